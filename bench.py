@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 x MXFP4 MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl cuda|reference]
+
+A step is one whole layer forward (router, top-k + gates, dispatch + E4M3
+quantisation, grouped linear1 + SwiGLU + requant, grouped linear2, combine) over
+one batch of T synthetic tokens already resident in HBM.  The default workload
+is the Mixtral-shaped layer (T=4096, H=4096, I=14336, E=8, k=2).  With N > 1
+(launched by torchrun) every rank runs an independent replica on its own GPU and
+its own token batch: the layer has no exchange step on one device, so there is
+no collective on the data path (weak scaling); ranks only meet for the timing
+barrier and the max-over-ranks reduction.
+
+`--impl reference` times the CPU oracle (float64 numpy, oracle/) on a bounded
+token sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fp8_fp4_moe_b200 import inputs as I  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOPS (% FP8 peak / % HBM) at T=1/512/8192/32768"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CPU_SAMPLE_TOKENS = {"tiny": 64, "mixtral": 8, "dsv3_t1": 1, "dsv3_t512": 2, "dsv3_t8192_zipf": 2,
+                     "dsv3_t32768": 2}
+REF_STEP_TOKENS = {"tiny": 64, "mixtral": 1, "dsv3_t1": 1, "dsv3_t512": 1, "dsv3_t8192_zipf": 1,
+                   "dsv3_t32768": 1}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm_sm100.cu", "common.cuh", "path_kernels.cu"):
+        with open(os.path.join(ROOT, "fp8_fp4_moe_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}@{workload}")
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return float(ent["bytes_per_launch"])
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_ids):
+        self.gpu_ids = gpu_ids
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ",".join(map(str, self.gpu_ids)), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1])]
+        mx = max((num(r[2]) or 0) for r in rows)
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def algorithmic_counts(w: I.Workload, counts):
+    """FLOPs and bytes of the layer and of each GEMM launch for the routed counts."""
+    touched = int(np.count_nonzero(counts))
+    rows = int(np.sum(counts))
+    H, I_ = w.H, w.I
+    w1_bytes = 2 * I_ * H // 2 + 2 * I_ * H // 32
+    w2_bytes = H * I_ // 2 + H * I_ // 32
+    return {
+        "layer_flops": w.flops(),
+        "layer_bytes": touched * (w1_bytes + w2_bytes) + w.E * H * 4 + w.T * H * 2 * 2,
+        "linear1_flops": 2.0 * rows * H * 2 * I_,
+        "linear1_bytes": touched * w1_bytes + rows * H + rows * I_,
+        "linear2_flops": 2.0 * rows * I_ * H,
+        "linear2_bytes": touched * w2_bytes + rows * I_ + rows * H * 2,
+        "touched_experts": touched,
+    }
+
+
+def cpu_baseline(w: I.Workload, n_tokens: int):
+    """The oracle as it stands, on all host cores, on a token sample of the workload."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe as M
+    x, W_r, bias = I.make_routing_inputs(w, 0)
+    rng = np.random.default_rng(0)
+    tokens = np.sort(rng.choice(w.T, size=min(n_tokens, w.T), replace=False))
+    x_np = x.view(torch.int16).numpy().view(np.uint16)
+    # expert weights of only the experts the sample touches (the rest are never read)
+    ids, _, _ = M.route(x_np[tokens], W_r.numpy(), bias.numpy(), w.k)
+    need = sorted(set(ids.ravel().tolist()) | ({w.E} if w.shared else set()))
+    W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device="cpu", experts=need)
+    t0 = time.perf_counter()
+    M.forward(x_np, W_r.numpy(), bias.numpy(), W1.numpy(), W1s.numpy(), W2.numpy(), W2s.numpy(), k=w.k,
+              shared=w.shared, tokens=tokens)
+    dt = time.perf_counter() - t0
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    return {"value": len(tokens) / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{w.name}: routing + dispatch of all {w.T} tokens, expert FFN + combine of "
+                      f"{len(tokens)} sampled tokens ({len(need)} experts), float64 numpy; {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe as M
+    w = I.WORKLOADS[args.workload]
+    x, W_r, bias = I.make_routing_inputs(w, 0)
+    x_np = x.view(torch.int16).numpy().view(np.uint16)
+    n_tok = REF_STEP_TOKENS[args.workload]
+    rng = np.random.default_rng(0)
+    samples = [np.sort(rng.choice(w.T, size=min(n_tok, w.T), replace=False))
+               for _ in range(args.steps + args.warmup)]
+    need = set()
+    for s in samples:
+        ids, _, _ = M.route(x_np[s], W_r.numpy(), bias.numpy(), w.k)
+        need |= set(ids.ravel().tolist())
+    if w.shared:
+        need.add(w.E)
+    W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device="cpu", experts=sorted(need))
+    args_np = (x_np, W_r.numpy(), bias.numpy(), W1.numpy(), W1s.numpy(), W2.numpy(), W2s.numpy())
+    for s in samples[:args.warmup]:
+        M.forward(*args_np, k=w.k, shared=w.shared, tokens=s)
+    t0 = time.perf_counter()
+    done = 0
+    for s in samples[args.warmup:]:
+        M.forward(*args_np, k=w.k, shared=w.shared, tokens=s)
+        done += len(s)
+    dt = time.perf_counter() - t0
+    value = done / dt
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": I.WORKLOADS[args.workload].description, "tokens_per_step": n_tok,
+                   "parallelism": "none (CPU oracle, rank 0)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{w.name}: per step routing + dispatch of all {w.T} tokens and the expert "
+                                   f"FFN + combine of {n_tok} sampled token(s), float64 numpy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+
+def run_cuda(args, rank, world, local_rank):
+    from fp8_fp4_moe_b200 import binding
+    w = I.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    _, W_r, bias = I.make_routing_inputs(w, 0)
+    x, _, _ = I.make_routing_inputs(w, 1000 + rank) if rank > 0 else I.make_routing_inputs(w, 0)
+    W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device=dev)
+    d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
+    plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared, device=dev)
+    plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 1)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        plan.forward(**d, out=out)
+    code, detail = plan.check_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} {detail}")
+    counts = plan.region("counts").cpu().numpy()
+
+    sampler = ClockSampler(list(range(world)) if rank == 0 else [local_rank])
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms, phases = [], []
+    for _ in range(args.steps):
+        flush.fill_(1)                                   # L2 scrub between timed steps (not timed)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        plan.forward(**d, out=out)
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms.append(ev0.elapsed_time(ev1))
+        phases.append(plan.phase_times())
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    code, detail = plan.check_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} {detail}")
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(total_ms, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+
+    # end to end through the public API: pinned host x -> device, forward, out -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        x_host = d["x"].cpu().pin_memory()
+        out_host = torch.empty(w.T, w.H, dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(d["x"])
+        d_e2e = dict(d)
+        d_e2e["x"] = x_dev
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e_ms = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            plan.forward(**d_e2e, out=out)
+            out_host.copy_(out, non_blocking=True)
+            ev1.record(stream)
+            ev1.synchronize()
+            e_ms.append(ev0.elapsed_time(ev1))
+        t = torch.tensor([sum(e_ms)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_total = float(t.item())
+        e2e = {"value": world * w.T * args.steps / (e2e_total / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+               "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+               "ms_per_step": e2e_total / args.steps}
+        code, detail = plan.check_status()
+        if code != 0:
+            raise RuntimeError(f"device status {code} {detail}")
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    fp8_sustained = 2.0 * peaks["bf16_tflops_sustained"]       # nominal FP8 : BF16 dense ratio 2
+    hbm = peaks["hbm_gbs"]
+    alg = algorithmic_counts(w, counts)
+    avg = {k: statistics.mean(p[k] for p in phases) for k in phases[0]}
+    ms = total_ms / args.steps
+    dominant = max(avg, key=avg.get)
+    dom_ms = avg[dominant]
+    if dominant in ("linear1", "linear2"):
+        flops = alg[f"{dominant}_flops"]
+        byts = alg[f"{dominant}_bytes"]
+        if flops / byts > fp8_sustained * 1e12 / (hbm * 1e9):
+            roof = {"bound": "tensor", "achieved": flops / (dom_ms * 1e-3) / 1e12, "peak": fp8_sustained,
+                    "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        byts = alg["layer_bytes"]
+        roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dominant
+    roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json: 2 x bf16_tflops_sustained (FP8 = 2 x BF16 dense)"
+                           if roof["unit"] == "TFLOP/s" else f"{peak_src} MEASURED_PEAKS.json hbm_gbs")
+    roof["traffic"] = ncu_traffic(dominant, w.name)
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, CPU_SAMPLE_TOKENS[w.name])
+
+    value = world * w.T * args.steps / (total_ms / 1e3)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3 x fp4e2m1 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": w.description, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
+                   "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+                   "parallelism": f"replicas x{world} (token-sharded, no collective)"},
+        "tflops": w.flops() / (ms * 1e-3) / 1e12,
+        "tflops_frac_fp8": w.flops() / (ms * 1e-3) / 1e12 / fp8_sustained,
+        "hbm_gbs": alg["layer_bytes"] / (ms * 1e-3) / 1e9,
+        "hbm_frac": alg["layer_bytes"] / (ms * 1e-3) / 1e9 / hbm,
+        "phases_ms": avg,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 7 * args.steps,
+        "clocks": clocks,
+        "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
+    }
+    return line
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_cuda(args, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

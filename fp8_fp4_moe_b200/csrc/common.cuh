@@ -1,0 +1,249 @@
+// Device-side building blocks shared by the sm_100a kernels of libmoe_b200:
+// status reporting, bounded waits, mbarrier / TMA / tcgen05 PTX wrappers and
+// the E4M3 / power-of-two-scale activation quantiser.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ------------------------------------------------------------------ status words
+// status[0] = error code (0 = ok), [1] = where, [2] = block, [3] = detail.
+// The first error wins (atomicCAS on word 0).
+enum : int { kStatusTimeout = -4, kStatusBounds = -6 };
+enum : uint32_t {
+  kWhereGemmProducer = 0x100, kWhereGemmSfLoader = 0x200, kWhereGemmMma = 0x300,
+  kWhereGemmEpilogue = 0x400, kWhereGemmDrain = 0x500
+};
+
+__device__ __forceinline__ void report_status(uint32_t* status, int code, uint32_t where, uint32_t detail) {
+  if (atomicCAS(status, 0u, (uint32_t)code) == 0u) {
+    status[1] = where;
+    status[2] = blockIdx.x;
+    status[3] = detail;
+    __threadfence();
+  }
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbarrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Control block every waiting role consults: a CTA-wide abort flag in shared
+// memory, the global status words and the wait limit.
+struct WaitCtl {
+  volatile int* abort_flag;   // shared memory
+  uint32_t* status;           // global
+  uint64_t timeout_ns;
+};
+
+// Wait for the phase with the given parity to complete.  Gives up (returns
+// false) when the CTA has been aborted or after ctl.timeout_ns, in which case
+// it records MOE_ERR_DEVICE_TIMEOUT with `where` and raises the abort flag.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl,
+                                          uint32_t where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*ctl.abort_flag) return false;
+    if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+      report_status(ctl.status, kStatusTimeout, where, parity);
+      *ctl.abort_flag = 1;
+      __threadfence_block();
+      return false;
+    }
+  }
+}
+
+// Same, but ignores the abort flag: used to drain our own async copies.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ TMA
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ cp.async (4 bytes)
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive on `bar` once every tcgen05 async operation issued so far by this thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D(tmem) (+)= A(smem) x B(smem)^T with per-32-K block scales read from tmem.
+__device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory into 32 lanes x 4 columns of tmem,
+// replicated into all four 32-lane sub-partitions.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane (base+i).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading/stride
+// byte offsets (16-byte units), version 1, layout type.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
+  d |= (uint64_t)(layout & 0x7u) << 61;   // 0 = no swizzle, 2 = 128-byte swizzle
+  return d;
+}
+constexpr uint32_t kLayoutNoSwizzle = 0;
+constexpr uint32_t kLayoutSwizzle128B = 2;
+
+// Instruction descriptor for kind::mxf8f6f4 block-scaled MMA, A = E4M3,
+// B = E2M1, both K-major, UE8M0 scales, fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id & 3u) << 4          // B scale-factor byte
+         | (0u << 7)                  // A format: E4M3
+         | (5u << 10)                 // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17) // N / 8
+         | (1u << 23)                 // scale format: UE8M0
+         | ((uint32_t)(M >> 4) << 24) // M / 16
+         | (a_sf_id & 3u) << 29;      // A scale-factor byte
+}
+
+// ------------------------------------------------------------------ activation quantiser
+// Power-of-two scale exponent: the smallest integer p with amax <= 448 * 2^p,
+// p = 0 when amax == 0, and p >= -126 so that 2^p is a normal fp32 and p + 127
+// is a valid UE8M0 code.  Works on the fp32 bit pattern: with amax = 1.f * 2^E,
+// 448 * 2^p >= amax  <=>  p >= E - 8 + (f > 0.75 ? 1 : 0) - ... ; computed exactly
+// by comparing the mantissa against 448 = 1.75 * 2^8.
+__device__ __forceinline__ int pow2_exp_e4m3(float amax) {
+  if (!(amax > 0.f)) return 0;
+  const uint32_t bits = __float_as_uint(amax);
+  int e = (int)((bits >> 23) & 0xFF);
+  uint32_t man = bits & 0x7FFFFF;
+  if (e == 0) {                      // subnormal amax = man * 2^-149: normalise
+    int lz = __clz(man) - 8;         // shift that brings the leading one to bit 23
+    man = (man << lz) & 0x7FFFFF;
+    e = 1 - lz;
+  }
+  // amax = (1 + man/2^23) * 2^(e-127).  448 * 2^p = 1.75 * 2^(p+8).
+  // If 1 + man/2^23 <= 1.75, p = (e-127) - 8 works and p-1 does not; else p = e-127-7.
+  const uint32_t m175 = 0x600000;    // 0.75 * 2^23
+  int p = (e - 127) - 8 + (man > m175 ? 1 : 0);
+  return p < -126 ? -126 : p;
+}
+
+// 2^-p as an exact fp32 (p in [-126, 127]).
+__device__ __forceinline__ float exp2_neg(int p) {
+  int be = 127 - p;                   // biased exponent of 2^-p, in [0, 253]
+  if (be <= 0) return __uint_as_float(0x00400000u >> (-be));   // not reached for p <= 126
+  return __uint_as_float((uint32_t)be << 23);
+}
+
+// Two fp32 -> packed E4M3 pair (low byte = a), round to nearest even, saturating.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  return (uint32_t)cvt_e4m3x2(a, b) | ((uint32_t)cvt_e4m3x2(c, d) << 16);
+}
+
+}  // namespace moe

@@ -1,0 +1,64 @@
+// Host-side launchers of the libmoe_b200 kernels (internal interface).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- grouped block-scaled GEMMs (gemm_sm100.cu) --------------------------------
+constexpr int kGemmBM = 128;      // rows (tokens) per tile
+constexpr int kGemmBN = 256;      // accumulator columns per tile
+constexpr int kGemmBK = 128;      // K per pipeline stage
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 224; // 7 warps: TMA, MMA, SF loader, 4 x epilogue
+
+struct GemmArgs {
+  int K;               // reduction length (H for linear1, I for linear2)
+  int N;               // linear1: I (SwiGLU width); linear2: H (output width)
+  int rows_b;          // B rows per expert (2I or H)
+  int n_experts;       // E + shared
+  int rows_total;      // R + shared * T
+  int n_tiles_n;       // linear1: I/128; linear2: ceil(H/256)
+  const int32_t* counts;       // [n_experts]
+  const int32_t* offsets;      // [n_experts + 1]
+  const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
+  const uint32_t* sfa;         // [rows_total][K/128], UE8M0 code in all 4 bytes
+  const uint8_t* sfb;          // [n_experts * rows_b][K/32] UE8M0
+  uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
+  uint32_t* hsf;               // linear1 out: [rows_total][I/128]
+  uint16_t* y;                 // linear2 out: [rows_total][H] bf16
+  uint32_t* status;
+  uint64_t timeout_ns;
+  int inject_fault;
+};
+
+size_t gemm_smem_bytes();
+cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attribute
+cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+                                cudaStream_t s);
+cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+                                cudaStream_t s);
+
+// ---- routing / dispatch / combine (path_kernels.cu) -----------------------------
+cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
+                                 cudaStream_t s);
+// mode 0: select from logits (+bias), write ids/gates, then rank.  mode 1: rank given ids.
+// mode 1 validates the given ids (range, distinct per token) and records MOE_ERR_DEBUG_BOUNDS in `status`.
+cudaError_t launch_topk_rank(int mode, const float* logits, const float* bias, int32_t* topk_ids, float* gates,
+                             int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
+                             cudaStream_t s);
+cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
+                                 int32_t* group_base, int32_t* mtile_start, int T, int E, int k, int shared,
+                                 cudaStream_t s);
+// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale words.
+cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
+                                 const int32_t* group_base, int32_t* slot_pos, int32_t* perm, uint8_t* xq,
+                                 uint32_t* xsf, int T, int H, int E, int k, int shared, cudaStream_t s);
+// Token-order quantisation (debug entry point).
+cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,
+                           int H, int k, int shared, cudaStream_t s);
+
+}  // namespace moe

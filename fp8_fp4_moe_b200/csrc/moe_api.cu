@@ -1,0 +1,413 @@
+// Host side of libmoe_b200.so: plans, workspace layout, argument checks, TMA
+// descriptors and the launch sequence of the layer forward.
+//
+// Launch sequence of moe_forward (one stream, no host synchronisation):
+//   router_logits -> topk_rank -> dispatch_scan -> scatter_quant
+//   -> grouped GEMM linear1 (+SwiGLU +E4M3 requant) -> grouped GEMM linear2 -> combine
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "../../include/moe_b200.h"
+#include "kernels.h"
+
+using namespace moe;
+
+struct moe_plan_s {
+  int T, H, I, E, k, shared, n;
+  long long R, rows;
+  int G;
+  // options
+  int max_sms = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int inject_fault = 0;
+  // workspace layout
+  size_t region_off[MOE_REGION_COUNT_];
+  size_t region_len[MOE_REGION_COUNT_];
+  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile;
+  size_t total;
+  // bound state
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  int device = -1;
+  int num_sms = 0;
+  alignas(64) CUtensorMap tmA1, tmA2, tmB1, tmB2;
+  const void* w1_cached = nullptr;
+  const void* w2_cached = nullptr;
+  // per-phase timing (MOE_OPT_PHASE_EVENTS)
+  int phase_events = 0;
+  bool events_ready = false;
+  bool events_recorded = false;
+  cudaEvent_t ev[MOE_PHASE_COUNT_ + 1];
+};
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  if (get_encode() != MOE_OK) return MOE_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <class T>
+T* at(moe_plan_t p, size_t off) {
+  return reinterpret_cast<T*>(p->ws + off);
+}
+template <class T>
+T* region(moe_plan_t p, int r) {
+  return at<T>(p, p->region_off[r]);
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int check_bound(moe_plan_t p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev != p->device) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+GemmArgs gemm_args(moe_plan_t p, int mode, const uint8_t* W_scales) {
+  GemmArgs a{};
+  a.n_experts = p->n;
+  a.rows_total = (int)p->rows;
+  a.counts = region<int32_t>(p, MOE_REGION_COUNTS);
+  a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
+  a.mtile_start = at<int32_t>(p, p->off_mtile);
+  a.sfb = W_scales;
+  a.status = region<uint32_t>(p, MOE_REGION_STATUS);
+  a.timeout_ns = p->timeout_ns;
+  if (mode == 1) {
+    a.K = p->H;
+    a.N = p->I;
+    a.rows_b = 2 * p->I;
+    a.n_tiles_n = p->I / 128;
+    a.sfa = region<uint32_t>(p, MOE_REGION_XSF);
+    a.hq = region<uint8_t>(p, MOE_REGION_HQ);
+    a.hsf = region<uint32_t>(p, MOE_REGION_HSF);
+    a.inject_fault = p->inject_fault;
+  } else {
+    a.K = p->I;
+    a.N = p->H;
+    a.rows_b = p->H;
+    a.n_tiles_n = (p->H + kGemmBN - 1) / kGemmBN;
+    a.sfa = region<uint32_t>(p, MOE_REGION_HSF);
+    a.y = region<uint16_t>(p, MOE_REGION_Y);
+    a.inject_fault = 0;
+  }
+  return a;
+}
+
+int gemm_grid(moe_plan_t p, int n_tiles_n) {
+  const long long mt_bound = (p->rows + kGemmBM - 1) / kGemmBM + p->n;
+  long long tiles = mt_bound * n_tiles_n;
+  int sms = p->num_sms;
+  if (p->max_sms > 0 && p->max_sms < sms) sms = p->max_sms;
+  return (int)(tiles < sms ? tiles : sms);
+}
+
+// Record the event that closes phase `i` (event 0 opens the forward).
+void mark(moe_plan_t p, int i, cudaStream_t s) {
+  if (p->phase_events && p->events_ready) cudaEventRecord(p->ev[i], s);
+}
+
+// routing + dispatch + quantisation into the workspace
+int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias, cudaStream_t s) {
+  int32_t* ids = region<int32_t>(p, MOE_REGION_TOPK_IDS);
+  float* gates = region<float>(p, MOE_REGION_GATES);
+  cudaError_t e;
+  mark(p, 0, s);
+  if ((e = launch_router_logits(x, W_router, at<float>(p, p->off_logits), p->T, p->H, p->E, s)) != cudaSuccess)
+    return cuda_rc(e);
+  mark(p, 1 + MOE_PHASE_ROUTER, s);
+  if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, ids, gates, at<int32_t>(p, p->off_rank),
+                            at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E,
+                            p->k, s)) != cudaSuccess)
+    return cuda_rc(e);
+  mark(p, 1 + MOE_PHASE_TOPK, s);
+  if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
+                                region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
+                                at<int32_t>(p, p->off_mtile), p->T, p->E, p->k, p->shared, s)) != cudaSuccess)
+    return cuda_rc(e);
+  mark(p, 1 + MOE_PHASE_SCAN, s);
+  e = launch_scatter_quant(x, ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
+                           region<int32_t>(p, MOE_REGION_SLOT_POS), region<int32_t>(p, MOE_REGION_PERM),
+                           region<uint8_t>(p, MOE_REGION_XQ), region<uint32_t>(p, MOE_REGION_XSF), p->T, p->H,
+                           p->E, p->k, p->shared, s);
+  mark(p, 1 + MOE_PHASE_SCATTER_QUANT, s);
+  return cuda_rc(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (T < 1 || H < 128 || I < 128 || H % 128 || I % 128 || E < 1 || E > 1024 || k < 1 || k > 16 || k > E ||
+      (shared != 0 && shared != 1) || E + shared > 1024)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const long long R = (long long)T * k;
+  const long long rows = R + (long long)shared * T;
+  // 32-bit row indices and TMA coordinates
+  if (rows * (long long)(H > I ? H : I) > (1ll << 40) || rows >= (1ll << 31) ||
+      (long long)(E + shared) * 2 * I >= (1ll << 31) || (long long)(E + shared) * H >= (1ll << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  moe_plan_t p = new (std::nothrow) moe_plan_s();
+  if (!p) return MOE_ERR_INVALID_ARG;
+  p->T = T; p->H = H; p->I = I; p->E = E; p->k = k; p->shared = shared; p->n = E + shared;
+  p->R = R; p->rows = rows; p->G = (T + 31) / 32;
+  size_t off = 0;
+  auto add = [&](size_t bytes) {
+    size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    return o;
+  };
+  auto reg = [&](int r, size_t bytes) {
+    p->region_off[r] = add(bytes);
+    p->region_len[r] = bytes;
+  };
+  const size_t Tk = (size_t)T * k;
+  reg(MOE_REGION_STATUS, 16);
+  reg(MOE_REGION_TOPK_IDS, Tk * 4);
+  reg(MOE_REGION_GATES, Tk * 4);
+  reg(MOE_REGION_COUNTS, (size_t)p->n * 4);
+  reg(MOE_REGION_OFFSETS, (size_t)(p->n + 1) * 4);
+  reg(MOE_REGION_PERM, (size_t)R * 4);
+  reg(MOE_REGION_SLOT_POS, Tk * 4);
+  reg(MOE_REGION_XQ, (size_t)rows * H);
+  reg(MOE_REGION_XSF, (size_t)rows * (H / 128) * 4);
+  reg(MOE_REGION_HQ, (size_t)rows * I);
+  reg(MOE_REGION_HSF, (size_t)rows * (I / 128) * 4);
+  reg(MOE_REGION_Y, (size_t)rows * H * 2);
+  p->off_logits = add((size_t)T * E * 4);
+  p->off_rank = add(Tk * 4);
+  p->off_gcounts = add((size_t)p->G * E * 4);
+  p->off_gbase = add((size_t)p->G * E * 4);
+  p->off_mtile = add((size_t)(p->n + 1) * 4);
+  p->total = off;
+  *out = p;
+  return MOE_OK;
+}
+
+int moe_plan_set_option(moe_plan_t p, int key, long long value) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  switch (key) {
+    case MOE_OPT_MAX_SMS:
+      if (value < 0) return MOE_ERR_INVALID_ARG;
+      p->max_sms = (int)value;
+      return MOE_OK;
+    case MOE_OPT_TIMEOUT_NS:
+      if (value <= 0) return MOE_ERR_INVALID_ARG;
+      p->timeout_ns = (uint64_t)value;
+      return MOE_OK;
+    case MOE_OPT_INJECT_FAULT:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->inject_fault = (int)value;
+      return MOE_OK;
+    case MOE_OPT_ROUTER_TC:
+      return value == 0 ? MOE_OK : MOE_ERR_INVALID_ARG;
+    case MOE_OPT_PHASE_EVENTS:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->phase_events = (int)value;
+      return MOE_OK;
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+}
+
+size_t moe_workspace_bytes(moe_plan_t p) { return p ? p->total : 0; }
+
+int moe_workspace_region(moe_plan_t p, int r, size_t* offset, size_t* bytes) {
+  if (!p || r < 0 || r >= MOE_REGION_COUNT_ || !offset || !bytes) return MOE_ERR_INVALID_ARG;
+  *offset = p->region_off[r];
+  *bytes = p->region_len[r];
+  return MOE_OK;
+}
+
+int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!ws || bytes < p->total || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED_SHAPE;   // built for sm_100a only
+  if (gemm_prepare_device() != cudaSuccess) return MOE_ERR_CUDA;
+  p->ws = static_cast<uint8_t*>(ws);
+  p->ws_bytes = bytes;
+  p->device = dev;
+  p->num_sms = sms;
+  p->w1_cached = p->w2_cached = nullptr;
+  int rc = encode_2d(&p->tmA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_XQ), p->H, p->rows,
+                     p->H, 128, 128);
+  if (rc == MOE_OK)
+    rc = encode_2d(&p->tmA2, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_HQ), p->I, p->rows,
+                   p->I, 128, 128);
+  if (rc != MOE_OK) {
+    p->ws = nullptr;
+    return rc;
+  }
+  if (cudaMemset(region<uint32_t>(p, MOE_REGION_STATUS), 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float* bias, const uint8_t* W1,
+                const uint8_t* W1_scales, const uint8_t* W2, const uint8_t* W2_scales, void* out, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(x, 16) || !aligned(W_router, 16) || !aligned(bias, 4) || !aligned(W1, 32) ||
+      !aligned(W1_scales, 4) || !aligned(W2, 32) || !aligned(W2_scales, 4) || !aligned(out, 16))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (W1 != p->w1_cached) {
+    rc = encode_2d(&p->tmB1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W1, p->H, (uint64_t)p->n * 2 * p->I, p->H / 2,
+                   128, 128);
+    if (rc != MOE_OK) return rc;
+    p->w1_cached = W1;
+  }
+  if (W2 != p->w2_cached) {
+    rc = encode_2d(&p->tmB2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
+                   128, 256);
+    if (rc != MOE_OK) return rc;
+    p->w2_cached = W2;
+  }
+  if (p->phase_events && !p->events_ready) {
+    for (int i = 0; i <= MOE_PHASE_COUNT_; ++i)
+      if (cudaEventCreate(&p->ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+    p->events_ready = true;
+  }
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  if ((rc = run_front(p, xb, W_router, bias, s)) != MOE_OK) return rc;
+  GemmArgs a1 = gemm_args(p, 1, W1_scales);
+  if (launch_gemm_linear1(p->tmA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(p, 1 + MOE_PHASE_LINEAR1, s);
+  GemmArgs a2 = gemm_args(p, 2, W2_scales);
+  if (launch_gemm_linear2(p->tmA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(p, 1 + MOE_PHASE_LINEAR2, s);
+  cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
+                                 region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
+                                 p->shared, s);
+  mark(p, 1 + MOE_PHASE_COMBINE, s);
+  if (p->phase_events && p->events_ready) p->events_recorded = true;
+  return cuda_rc(e);
+}
+
+int moe_phase_times(moe_plan_t p, float* ms, int capacity) {
+  if (!p || !ms || capacity < MOE_PHASE_COUNT_) return MOE_ERR_INVALID_ARG;
+  if (!p->events_recorded) return MOE_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(p->ev[MOE_PHASE_COUNT_]) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int i = 0; i < MOE_PHASE_COUNT_; ++i)
+    if (cudaEventElapsedTime(&ms[i], p->ev[i], p->ev[i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_PHASE_COUNT_;
+}
+
+int moe_debug_routing(moe_plan_t p, const void* x, const float* W_router, const float* bias, int32_t* topk_ids,
+                      float* gates, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(x, 16) || !aligned(W_router, 4) || !aligned(bias, 4) || !aligned(topk_ids, 4) || !aligned(gates, 4))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_router_logits(static_cast<const uint16_t*>(x), W_router, at<float>(p, p->off_logits), p->T,
+                                       p->H, p->E, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, topk_ids, gates, at<int32_t>(p, p->off_rank),
+                       at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
+  return cuda_rc(e);
+}
+
+int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, int32_t* offsets, int32_t* perm,
+                       int32_t* slot_pos, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(topk_ids, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) ||
+      !aligned(slot_pos, 4))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_topk_rank(1, nullptr, nullptr, const_cast<int32_t*>(topk_ids), nullptr,
+                                   at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
+                                   region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), counts, offsets, at<int32_t>(p, p->off_gbase),
+                                at<int32_t>(p, p->off_mtile), p->T, p->E, p->k, p->shared, s)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase), slot_pos,
+                           perm, nullptr, nullptr, p->T, p->H, p->E, p->k, p->shared, s);
+  return cuda_rc(e);
+}
+
+int moe_debug_quant_x(moe_plan_t p, const void* x, uint8_t* xq, float* xs, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(x, 16) || !aligned(xq, 8) || !aligned(xs, 4)) return MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_quant_tokens(static_cast<const uint16_t*>(x), xq, xs, p->T, p->H,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int moe_check_status(moe_plan_t p, void* stream, uint32_t* detail) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t h[4] = {0, 0, 0, 0};
+  uint32_t* d = region<uint32_t>(p, MOE_REGION_STATUS);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(h, d, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(d, 0, sizeof(h)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (detail) std::memcpy(detail, h, sizeof(h));
+  return (int)(int32_t)h[0];
+}
+
+void moe_plan_destroy(moe_plan_t p) {
+  if (!p) return;
+  if (p->events_ready)
+    for (int i = 0; i <= MOE_PHASE_COUNT_; ++i) cudaEventDestroy(p->ev[i]);
+  delete p;
+}
+
+const char* moe_error_string(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or device";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_DEBUG_BOUNDS: return "device-side bounds check failed";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

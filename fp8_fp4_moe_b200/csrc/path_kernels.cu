@@ -1,0 +1,427 @@
+// Routing, dispatch (+ activation quantisation) and combine kernels.
+//
+// Router and gates: "전문가 혼합(Mixture of Experts; MoE)" lesson, "FFN 교체"
+// (the router is one linear layer giving a score per expert) and "Step 1: 라우터"
+// (selection by descending score + bias, gates = softmax over the selected
+// experts' original scores); the bias steers selection only ("부하 분산 문제").
+// Dispatch/combine: "Mega MoE" wiki, "한 줄 정의" -- on one device an in-HBM
+// permutation of token copies into expert-major order and a gather back.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+// --------------------------------------------------------------------------- router
+// logits[t][e] = sum_h x[t][h] * W_r[e][h], fp32 FMA on CUDA cores.
+// Block tile: 64 tokens x ET experts, K chunks of 32 staged in shared memory.
+template <int ET>
+__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                            const float* __restrict__ W, float* __restrict__ logits,
+                                                            int T, int H, int E) {
+  constexpr int TT = 64, KC = 32;
+  constexpr int EPT = ET / 16;           // experts per thread
+  __shared__ float xs[KC][TT + 1];
+  __shared__ float ws[KC][ET + 1];
+  const int t0 = blockIdx.x * TT;
+  const int e0 = blockIdx.y * ET;
+  const int tx = threadIdx.x % 16;       // expert lane
+  const int ty = threadIdx.x / 16;       // token group of 4
+  float acc[4][EPT];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = 0; k0 < H; k0 += KC) {
+    for (int idx = threadIdx.x; idx < TT * KC; idx += 256) {
+      const int tt = idx / KC, kk = idx % KC;
+      const int t = t0 + tt;
+      float v = 0.f;
+      if (t < T) v = __uint_as_float((uint32_t)x[(long)t * H + k0 + kk] << 16);
+      xs[kk][tt] = v;
+    }
+    for (int idx = threadIdx.x; idx < ET * KC; idx += 256) {
+      const int ee = idx / KC, kk = idx % KC;
+      const int e = e0 + ee;
+      ws[kk][ee] = (e < E) ? W[(long)e * H + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < KC; ++kk) {
+      float xv[4], wv[EPT];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) wv[j] = ws[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = e0 + tx + 16 * j;
+      if (e < E) logits[(long)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- top-k + rank
+// One block per group of 32 tokens; warp w selects for token 32*g + w.
+// Then warp 0 ranks the group's copies: lane = token, and each expert keeps a
+// 32-bit mask of the group's tokens that chose it.  A copy's rank inside its
+// expert is the number of lower lanes in that mask (ascending token order).
+__global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* __restrict__ logits,
+                                                         const float* __restrict__ bias, int32_t* topk_ids,
+                                                         float* gates, int32_t* __restrict__ local_rank,
+                                                         int32_t* __restrict__ group_counts, uint32_t* status,
+                                                         int T, int E, int k) {
+  __shared__ int32_t ids_s[32][16];
+  __shared__ uint32_t mask_s[1024];
+  const int g = blockIdx.x;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) mask_s[e] = 0u;
+  const int t = g * 32 + warp;
+  if (t < T) {
+    if (mode == 0) {
+      const float* row = logits + (long)t * E;
+      // k rounds of a warp arg-max over (score + bias), lower id on ties
+      float chosen_score = 0.f;   // unbiased score of this lane's slot (lane < k)
+      int chosen_id = -1;
+      uint32_t taken = 0u;        // bit i: expert lane + 32*i already selected (E <= 1024)
+      for (int j = 0; j < k; ++j) {
+        float best = -INFINITY;
+        int best_id = 0x7FFFFFFF;
+        int free_id = 0x7FFFFFFF;   // lowest unselected id (fallback when every score is NaN)
+        for (int i = 0, e = lane; e < E; ++i, e += 32) {
+          if (taken & (1u << i)) continue;
+          if (free_id == 0x7FFFFFFF) free_id = e;
+          const float b = row[e] + bias[e];
+          if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oid = __shfl_xor_sync(0xffffffffu, best_id, off);
+          if (ob > best || (ob == best && oid < best_id)) { best = ob; best_id = oid; }
+          free_id = min(free_id, __shfl_xor_sync(0xffffffffu, free_id, off));
+        }
+        if (best_id == 0x7FFFFFFF) best_id = free_id;   // k <= E guarantees free_id < E
+        if ((best_id & 31) == lane) taken |= 1u << (best_id >> 5);
+        if (lane == j) { chosen_id = best_id; chosen_score = row[best_id]; }
+      }
+      // softmax over the unbiased scores of the selected experts
+      float m = (lane < k) ? chosen_score : -INFINITY;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float ex = (lane < k) ? expf(chosen_score - m) : 0.f;
+      float sum = ex;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane < k) {
+        topk_ids[(long)t * k + lane] = chosen_id;
+        gates[(long)t * k + lane] = ex / sum;
+        ids_s[warp][lane] = chosen_id;
+      }
+    } else {
+      int id = (lane < k) ? topk_ids[(long)t * k + lane] : -1;
+      bool bad = lane < k && (id < 0 || id >= E);
+      for (int j = 0; j < k; ++j) {
+        const int other = __shfl_sync(0xffffffffu, id, j);
+        if (lane < k && j != lane && other == id) bad = true;
+      }
+      if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) report_status(status, kStatusBounds, 0x10, (uint32_t)t);
+        id = (lane < E) ? lane : 0;        // keep every index in range; results are void
+      }
+      if (lane < k) ids_s[warp][lane] = id;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int tt = g * 32 + lane;
+    if (tt < T)
+      for (int j = 0; j < k; ++j) atomicOr(&mask_s[ids_s[lane][j]], 1u << lane);
+    __syncwarp();
+    if (tt < T)
+      for (int j = 0; j < k; ++j)
+        local_rank[(long)tt * k + j] = __popc(mask_s[ids_s[lane][j]] & ((1u << lane) - 1u));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) group_counts[(long)g * E + e] = __popc(mask_s[e]);
+}
+
+// --------------------------------------------------------------------------- scan
+// One block.  counts[e] = sum over groups; offsets = exclusive scan over experts
+// (shared expert last, T rows); group_base[g][e] = offsets[e] + rows of e in
+// groups < g; mtile_start = exclusive scan of ceil(count/128).
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __restrict__ group_counts,
+                                                             int32_t* counts, int32_t* offsets,
+                                                             int32_t* group_base, int32_t* mtile_start, int T,
+                                                             int E, int k, int shared) {
+  __shared__ int32_t warp_sums[2][32];
+  const int G = (T + 31) / 32;
+  const int n = E + shared;
+  const int e = threadIdx.x;           // n <= 1025: thread 1024 never needed (E <= 1024, shared expert handled below)
+  int c = 0;
+  if (e < E) {
+    for (int g = 0; g < G; ++g) c += group_counts[(long)g * E + e];
+  } else if (e == E && shared) {
+    c = T;
+  }
+  // block-wide exclusive scans of c and of ceil(c/128)
+  int mt = (c + kGemmBM - 1) / kGemmBM;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int ic = c, im = mt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ic, off);
+    const int b = __shfl_up_sync(0xffffffffu, im, off);
+    if (lane >= off) { ic += a; im += b; }
+  }
+  if (lane == 31) { warp_sums[0][warp] = ic; warp_sums[1][warp] = im; }
+  __syncthreads();
+  if (warp == 0) {
+    int a = warp_sums[0][lane], b = warp_sums[1][lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int a2 = __shfl_up_sync(0xffffffffu, a, off);
+      const int b2 = __shfl_up_sync(0xffffffffu, b, off);
+      if (lane >= off) { a += a2; b += b2; }
+    }
+    warp_sums[0][lane] = a;
+    warp_sums[1][lane] = b;
+  }
+  __syncthreads();
+  const int base_c = (warp > 0 ? warp_sums[0][warp - 1] : 0) + ic - c;
+  const int base_m = (warp > 0 ? warp_sums[1][warp - 1] : 0) + im - mt;
+  if (e < n) {
+    counts[e] = c;
+    offsets[e] = base_c;
+    mtile_start[e] = base_m;
+  }
+  if (e == n - 1) {
+    offsets[n] = base_c + c;
+    mtile_start[n] = base_m + mt;
+  }
+  if (e < E) {
+    int run = base_c;
+    for (int g = 0; g < G; ++g) {
+      group_base[(long)g * E + e] = run;
+      run += group_counts[(long)g * E + e];
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- scatter + quant
+// One warp per token.  Positions: slot_pos[t][j] = group_base[g][e] + rank;
+// the shared expert's row for token t is R + t.  Quantisation: per 128-channel
+// block, smallest 2^p with amax <= 448 * 2^p (p >= -126; p = 0 if all zero),
+// codes = E4M3 round-to-nearest-even of x * 2^-p (exact scaling), written once
+// per destination row together with the block's UE8M0 code word.
+__global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __restrict__ x,
+                                                            const int32_t* __restrict__ topk_ids,
+                                                            const int32_t* __restrict__ local_rank,
+                                                            const int32_t* __restrict__ group_base,
+                                                            int32_t* slot_pos, int32_t* perm, uint8_t* xq,
+                                                            uint32_t* xsf, int T, int H, int E, int k, int shared) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const int g = t / 32;
+  const long R = (long)T * k;
+  int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
+  if (lane < k) {
+    const int e = topk_ids[(long)t * k + lane];
+    row = group_base[(long)g * E + e] + local_rank[(long)t * k + lane];
+    slot_pos[(long)t * k + lane] = row;
+    perm[row] = t * k + lane;
+  } else if (lane == k && shared) {
+    row = (int)(R + t);
+  }
+  if (x == nullptr) return;
+  const int ndst = k + shared;
+  const int kw = H / 128;
+  const uint16_t* xr = x + (long)t * H;
+  for (int cb = 0; cb < H; cb += 256) {
+    // 8 channels per lane; a 128-channel block spans 16 lanes.  Every lane runs
+    // every iteration (shuffles use the full mask); a half-warp past H idles.
+    const int c0 = cb + lane * 8;
+    const bool active = c0 < H;           // H % 128 == 0: whole half-warps
+    const uint4 raw = active ? *reinterpret_cast<const uint4*>(xr + c0) : make_uint4(0, 0, 0, 0);
+    float v[8];
+    v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(raw.z << 16); v[5] = __uint_as_float(raw.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(raw.w << 16); v[7] = __uint_as_float(raw.w & 0xFFFF0000u);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int p = pow2_exp_e4m3(amax);
+    const float sc = exp2_neg(p);
+    uint2 q;
+    q.x = pack_e4m3x4(v[0] * sc, v[1] * sc, v[2] * sc, v[3] * sc);
+    q.y = pack_e4m3x4(v[4] * sc, v[5] * sc, v[6] * sc, v[7] * sc);
+    const uint32_t code = (uint32_t)(p + 127) * 0x01010101u;
+    const int blk = c0 / 128;
+    for (int d = 0; d < ndst; ++d) {
+      const long r = __shfl_sync(0xffffffffu, row, d);
+      if (active) {
+        *reinterpret_cast<uint2*>(xq + r * H + c0) = q;
+        if ((lane & 15) == 0) xsf[r * kw + blk] = code;
+      }
+    }
+  }
+}
+
+// Token-order quantisation for the debug entry point: xq[t][H], xs[t][H/128] = 2^p.
+__global__ void __launch_bounds__(256) quant_tokens_kernel(const uint16_t* __restrict__ x, uint8_t* xq, float* xs,
+                                                           int T, int H) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const uint16_t* xr = x + (long)t * H;
+  for (int cb = 0; cb < H; cb += 256) {
+    const int c0 = cb + lane * 8;
+    const bool active = c0 < H;
+    const uint4 raw = active ? *reinterpret_cast<const uint4*>(xr + c0) : make_uint4(0, 0, 0, 0);
+    float v[8];
+    v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(raw.z << 16); v[5] = __uint_as_float(raw.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(raw.w << 16); v[7] = __uint_as_float(raw.w & 0xFFFF0000u);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int p = pow2_exp_e4m3(amax);
+    const float sc = exp2_neg(p);
+    uint2 q;
+    q.x = pack_e4m3x4(v[0] * sc, v[1] * sc, v[2] * sc, v[3] * sc);
+    q.y = pack_e4m3x4(v[4] * sc, v[5] * sc, v[6] * sc, v[7] * sc);
+    if (active) {
+      *reinterpret_cast<uint2*>(xq + (long)t * H + c0) = q;
+      if ((lane & 15) == 0) xs[(long)t * (H / 128) + c0 / 128] = exp2_neg(-p);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- combine
+// out[t] = bf16( sum_{j<k} gate[t][j] * row[slot_pos[t][j]] + shared * row[R + t] ),
+// fp32 accumulation in exactly that order (deterministic, no atomics).
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
+                                                      const int32_t* __restrict__ slot_pos,
+                                                      const float* __restrict__ gates, uint16_t* __restrict__ out,
+                                                      int T, int H, int k, int shared) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const long R = (long)T * k;
+  int my_row = 0;
+  float my_gate = 0.f;
+  if (lane < k) {
+    my_row = slot_pos[(long)t * k + lane];
+    my_gate = gates[(long)t * k + lane];
+  }
+  for (int cb = 0; cb < H; cb += 256) {
+    const int c0 = cb + lane * 8;
+    const bool active = c0 < H;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const long r = __shfl_sync(0xffffffffu, my_row, j);
+      const float gj = __shfl_sync(0xffffffffu, my_gate, j);
+      if (!active) continue;
+      const uint4 raw = *reinterpret_cast<const uint4*>(y + r * H + c0);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(gj, __uint_as_float(w[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(gj, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+      }
+    }
+    if (!active) continue;
+    if (shared) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(y + (R + t) * H + c0);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(w[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    }
+    uint4 o;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[0], acc[1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[2], acc[3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[4], acc[5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(acc[6], acc[7]);
+    o.x = *reinterpret_cast<uint32_t*>(&b0);
+    o.y = *reinterpret_cast<uint32_t*>(&b1);
+    o.z = *reinterpret_cast<uint32_t*>(&b2);
+    o.w = *reinterpret_cast<uint32_t*>(&b3);
+    *reinterpret_cast<uint4*>(out + (long)t * H + c0) = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
+                                 cudaStream_t s) {
+  if (E <= 16) {
+    dim3 grid((T + 63) / 64, (E + 15) / 16);
+    router_logits_kernel<16><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+  } else {
+    dim3 grid((T + 63) / 64, (E + 63) / 64);
+    router_logits_kernel<64><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_rank(int mode, const float* logits, const float* bias, int32_t* topk_ids, float* gates,
+                             int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
+                             cudaStream_t s) {
+  const int G = (T + 31) / 32;
+  topk_rank_kernel<<<G, 1024, 0, s>>>(mode, logits, bias, topk_ids, gates, local_rank, group_counts, status, T, E,
+                                      k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
+                                 int32_t* group_base, int32_t* mtile_start, int T, int E, int k, int shared,
+                                 cudaStream_t s) {
+  dispatch_scan_kernel<<<1, 1024, 0, s>>>(group_counts, counts, offsets, group_base, mtile_start, T, E, k, shared);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
+                                 const int32_t* group_base, int32_t* slot_pos, int32_t* perm, uint8_t* xq,
+                                 uint32_t* xsf, int T, int H, int E, int k, int shared, cudaStream_t s) {
+  scatter_quant_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, topk_ids, local_rank, group_base, slot_pos, perm, xq, xsf,
+                                                   T, H, E, k, shared);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s) {
+  quant_tokens_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, xq, xs, T, H);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,
+                           int H, int k, int shared, cudaStream_t s) {
+  combine_kernel<<<(T + 7) / 8, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

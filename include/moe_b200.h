@@ -1,0 +1,164 @@
+/*
+ * moe_b200.h -- C ABI of libmoe_b200.so: the forward pass of one
+ * Mixture-of-Experts FFN layer with FP8 (E4M3) activations and MXFP4 (E2M1 +
+ * UE8M0) expert weights on one NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (page title, section):
+ *   router scores, biased top-k selection, softmax gates over the unbiased
+ *   scores of the selected experts     -- "전문가 혼합(Mixture of Experts; MoE)"
+ *                                         lesson, "FFN 교체", "부하 분산 문제",
+ *                                         "Step 1: 라우터";
+ *   dispatch -> linear1 (FP8 x FP4) -> SwiGLU -> linear2 (FP8 x FP4) -> combine
+ *                                       -- "DeepSeek Mega MoE / DeepGEMM mega
+ *                                         kernel", "TL;DR" and the
+ *                                         "Thông số kỹ thuật" table; "Mega MoE"
+ *                                         wiki, "한 줄 정의";
+ *   an always-on shared expert          -- MoE lesson, "공유 전문가".
+ * On one device dispatch and combine are an in-memory permutation and gather.
+ *
+ * Conventions shared by every entry point
+ *   - All arrays are row-major and contiguous.  Every array pointer is a DEVICE
+ *     pointer on the device that was current when moe_set_workspace() ran,
+ *     16-byte aligned; W1 and W2 must be 32-byte aligned.  The caller owns all
+ *     memory (inputs, outputs, workspace) and the plan.  The library never
+ *     allocates device memory.
+ *   - Shapes: T tokens, hidden size H, expert intermediate size I, E routed
+ *     experts, k experts per token, shared in {0,1}; n = E + shared; R = T*k.
+ *     Constraints: T >= 1, H % 128 == 0, I % 128 == 0, 1 <= k <= min(E, 16),
+ *     1 <= E <= 1024.  Violations return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - x         bf16  [T, H]
+ *     W_router  fp32  [E, H]            routed experts only
+ *     bias      fp32  [E]               added to the scores for selection only
+ *     W1        uint8 [n, 2I, H/2]      MXFP4 codes; rows 0..I-1 = gate,
+ *                                       rows I..2I-1 = up; byte j of a row holds
+ *                                       element 2j (low nibble), 2j+1 (high)
+ *     W1_scales uint8 [n, 2I, H/32]     UE8M0, one per 32 consecutive K elements
+ *     W2        uint8 [n, H, I/2]       MXFP4 codes
+ *     W2_scales uint8 [n, H, I/32]      UE8M0
+ *     out       bf16  [T, H]
+ *     Expert index E is the shared expert when shared == 1.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All compute entry points are asynchronous and stream-ordered; they never
+ *     synchronise the host.  Device-side failures (bounded waits that ran out)
+ *     are recorded in the workspace and reported by moe_check_status().
+ *   - Return codes are the MOE_* values below.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_plan_s* moe_plan_t;
+
+enum moe_status_code {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,        /* NULL/misaligned pointer, bad option, plan state */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2,  /* shape outside the constraints above           */
+  MOE_ERR_CUDA = -3,               /* a CUDA runtime/driver call or launch failed    */
+  MOE_ERR_DEVICE_TIMEOUT = -4,     /* a device-side wait ran out (see check_status)  */
+  MOE_ERR_WORKSPACE = -5,          /* workspace missing or too small                 */
+  MOE_ERR_DEBUG_BOUNDS = -6        /* a device-side bounds check failed              */
+};
+
+enum moe_option {
+  MOE_OPT_MAX_SMS = 1,         /* persistent GEMM grid size cap (0 = all SMs)            */
+  MOE_OPT_TIMEOUT_NS = 2,      /* device wait limit in ns (default 2e9)                  */
+  MOE_OPT_INJECT_FAULT = 3,    /* test hook: 1 = the GEMM1 scale-factor loader withholds
+                                  its first arrival, so the MMA warp's bounded wait runs
+                                  out and the call reports MOE_ERR_DEVICE_TIMEOUT        */
+  MOE_OPT_ROUTER_TC = 4,       /* reserved: 1 = tensor-core router (default 0)           */
+  MOE_OPT_PHASE_EVENTS = 5     /* 1 = record a CUDA event after each kernel of moe_forward
+                                  on its stream, read back with moe_phase_times()        */
+};
+
+/* Phases of moe_forward, in launch order (moe_phase_times). */
+enum moe_phase {
+  MOE_PHASE_ROUTER = 0, MOE_PHASE_TOPK, MOE_PHASE_SCAN, MOE_PHASE_SCATTER_QUANT,
+  MOE_PHASE_LINEAR1, MOE_PHASE_LINEAR2, MOE_PHASE_COMBINE, MOE_PHASE_COUNT_
+};
+
+/* Workspace regions (moe_workspace_region) -- for tests and debugging. */
+enum moe_region {
+  MOE_REGION_STATUS = 0,   /* uint32 [4]: code, where, block, detail                      */
+  MOE_REGION_TOPK_IDS,     /* int32  [T, k]                                               */
+  MOE_REGION_GATES,        /* fp32   [T, k]                                               */
+  MOE_REGION_COUNTS,       /* int32  [n]                                                  */
+  MOE_REGION_OFFSETS,      /* int32  [n + 1]                                              */
+  MOE_REGION_PERM,         /* int32  [R]                                                  */
+  MOE_REGION_SLOT_POS,     /* int32  [T, k]                                               */
+  MOE_REGION_XQ,           /* uint8  [R + shared*T, H]   E4M3, dispatched row order       */
+  MOE_REGION_XSF,          /* uint32 [R + shared*T, H/128] UE8M0 code in all four bytes  */
+  MOE_REGION_HQ,           /* uint8  [R + shared*T, I]   E4M3 SwiGLU output               */
+  MOE_REGION_HSF,          /* uint32 [R + shared*T, I/128]                                */
+  MOE_REGION_Y,            /* bf16   [R + shared*T, H]   expert output rows               */
+  MOE_REGION_COUNT_
+};
+
+/* Create a plan for one layer shape.  Host only; touches no device.
+ * `out` receives a heap object the caller releases with moe_plan_destroy(). */
+int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out);
+
+/* Set a moe_option.  Returns MOE_ERR_INVALID_ARG for an unknown key/value. */
+int moe_plan_set_option(moe_plan_t plan, int key, long long value);
+
+/* Bytes of device workspace the plan needs (0 for a NULL plan). */
+size_t moe_workspace_bytes(moe_plan_t plan);
+
+/* Bind caller-allocated device workspace (>= moe_workspace_bytes, 256-byte
+ * aligned).  The device current at this call becomes the plan's device. */
+int moe_set_workspace(moe_plan_t plan, void* workspace, size_t bytes);
+
+/* Offset and size of a workspace region (moe_region) in bytes. */
+int moe_workspace_region(moe_plan_t plan, int region, size_t* offset, size_t* bytes);
+
+/* The whole layer: out = bf16( sum_j gate[t,j] * Expert_{id[t,j]}(x_t) + shared*Expert_E(x_t) ).
+ * Requantisation points: x -> E4M3 (per token per 128 channels, power-of-two
+ * scale), SwiGLU output -> E4M3 (same rule), expert rows -> bf16, out -> bf16. */
+int moe_forward(moe_plan_t plan, const void* x_bf16, const float* W_router, const float* bias,
+                const uint8_t* W1, const uint8_t* W1_scales,
+                const uint8_t* W2, const uint8_t* W2_scales,
+                void* out_bf16, void* stream);
+
+/* Routing only: topk_ids int32 [T,k] (descending biased score, lower id first
+ * on ties) and gates fp32 [T,k] (softmax over the selected unbiased scores). */
+int moe_debug_routing(moe_plan_t plan, const void* x_bf16, const float* W_router, const float* bias,
+                      int32_t* topk_ids, float* gates, void* stream);
+
+/* Dispatch only, from given topk_ids int32 [T,k] (each id in [0,E), distinct
+ * within a token): counts int32 [n], offsets int32 [n+1], perm int32 [R]
+ * (entry t*k+j at the row token t's j-th copy occupies), slot_pos int32 [T,k].
+ * Order: expert-major, ascending token id within an expert; shared rows last. */
+int moe_debug_dispatch(moe_plan_t plan, const int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                       int32_t* perm, int32_t* slot_pos, void* stream);
+
+/* Activation quantisation only, token order: xq uint8 [T,H] E4M3 codes and
+ * xs fp32 [T,H/128] power-of-two scales (smallest 2^p with amax <= 448*2^p,
+ * p >= -126; 1 for an all-zero block); x ~ decode(xq) * xs. */
+int moe_debug_quant_x(moe_plan_t plan, const void* x_bf16, uint8_t* xq, float* xs, void* stream);
+
+/* Kernel durations (ms) of the most recent moe_forward that ran with
+ * MOE_OPT_PHASE_EVENTS = 1, one per moe_phase, measured with CUDA events on
+ * that call's stream.  Waits for those events.  Returns the number of values
+ * written (MOE_PHASE_COUNT_), or a negative MOE_* code. */
+int moe_phase_times(moe_plan_t plan, float* ms, int capacity);
+
+/* Synchronise `stream`, then return the device-side status recorded since the
+ * last call (MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEBUG_BOUNDS) and clear it.
+ * `detail` (may be NULL) receives the 4 status words. */
+int moe_check_status(moe_plan_t plan, void* stream, uint32_t* detail);
+
+/* Release a plan (NULL is a no-op).  Does not free the workspace. */
+void moe_plan_destroy(moe_plan_t plan);
+
+/* Static string for a return code. */
+const char* moe_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

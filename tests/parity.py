@@ -1,0 +1,55 @@
+"""Shared helpers of the GPU parity tests: build cases, run the oracle, compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from fp8_fp4_moe_b200 import inputs as I
+from oracle import formats as F
+from oracle import moe as M
+from oracle import screen
+
+# Output tolerance of the layer (relative Frobenius, and max-abs relative to rms(out)).
+REL_FROB_TOL = 5e-3
+MAX_ABS_RMS_TOL = 2e-2
+
+
+def bits(x: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> uint16 numpy bit patterns (CPU)."""
+    return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def make_case(w: I.Workload, seed: int = 0, screened: bool = True, weight_device="cpu"):
+    if screened:
+        x, W_r, bias, _ = screen.screened_routing_inputs(w, seed)
+    else:
+        x, W_r, bias = I.make_routing_inputs(w, seed)
+    W1, W1s, W2, W2s = I.make_expert_weights(w, seed, device=weight_device)
+    return dict(x=x, W_router=W_r, bias=bias, W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
+
+
+def to_device(case: dict, device="cuda") -> dict:
+    return {k: v.to(device).contiguous() for k, v in case.items()}
+
+
+def oracle_forward(case: dict, w: I.Workload, tokens=None, keep_rows=False):
+    return M.forward(bits(case["x"]), case["W_router"].cpu().numpy(), case["bias"].cpu().numpy(),
+                     case["W1"].cpu().numpy(), case["W1_scales"].cpu().numpy(), case["W2"].cpu().numpy(),
+                     case["W2_scales"].cpu().numpy(), k=w.k, shared=w.shared, tokens=tokens, keep_rows=keep_rows)
+
+
+def output_errors(gpu_out_bits: np.ndarray, ref_y: np.ndarray):
+    got = F.bf16_to_f64(gpu_out_bits)
+    diff = got - ref_y
+    rms = float(np.sqrt(np.mean(ref_y ** 2)))
+    rel_frob = float(np.linalg.norm(diff) / max(np.linalg.norm(ref_y), 1e-300))
+    max_abs = float(np.max(np.abs(diff)))
+    return rel_frob, max_abs, rms
+
+
+def assert_output_close(gpu_out_bits, ref_y, what=""):
+    rel_frob, max_abs, rms = output_errors(gpu_out_bits, ref_y)
+    assert np.all(np.isfinite(F.bf16_to_f64(gpu_out_bits))), what
+    assert rel_frob <= REL_FROB_TOL, f"{what}: rel Frobenius {rel_frob:.3e}"
+    assert max_abs <= MAX_ABS_RMS_TOL * rms, f"{what}: max abs {max_abs:.3e} vs rms {rms:.3e}"
+    return rel_frob, max_abs, rms

@@ -1,0 +1,102 @@
+"""The C-ABI library builds, loads without a GPU and exports every declared entry point.
+
+Only host-side logic is exercised here (plans, shape validation, workspace
+layout, option checks); nothing launches a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_fp4_moe_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    assert sorted(names) == sorted(binding.EXPORTED)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _plan(L, *shape):
+    h = ctypes.c_void_p()
+    rc = L.moe_plan(*shape, ctypes.byref(h))
+    return rc, h
+
+
+@pytest.mark.parametrize("shape", [
+    (0, 256, 512, 8, 2, 0),      # T < 1
+    (64, 200, 512, 8, 2, 0),     # H % 128
+    (64, 256, 500, 8, 2, 0),     # I % 128
+    (64, 256, 512, 8, 9, 0),     # k > E
+    (64, 256, 512, 8, 0, 0),     # k < 1
+    (64, 256, 512, 32, 17, 0),   # k > 16
+    (64, 256, 512, 1025, 2, 0),  # E > 1024
+    (64, 256, 512, 1024, 2, 1),  # E + shared > 1024
+    (64, 256, 512, 8, 2, 2),     # shared not 0/1
+])
+def test_plan_rejects_unsupported_shapes(L, shape):
+    rc, h = _plan(L, *shape)
+    assert rc == binding.MOE_ERR_UNSUPPORTED_SHAPE and not h.value
+
+
+def test_workspace_layout_is_aligned_and_disjoint(L):
+    rc, h = _plan(L, 4096, 4096, 14336, 8, 2, 0)
+    assert rc == 0
+    total = L.moe_workspace_bytes(h)
+    T, H, I, k = 4096, 4096, 14336, 2
+    rows = T * k
+    spans = []
+    for name, r in binding.REGIONS.items():
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        assert L.moe_workspace_region(h, r, ctypes.byref(off), ctypes.byref(n)) == 0
+        assert off.value % 256 == 0 and off.value + n.value <= total
+        spans.append((off.value, off.value + n.value, name))
+    spans.sort()
+    for a, b in zip(spans, spans[1:]):
+        assert a[1] <= b[0], (a, b)
+    sizes = {name: e - s for s, e, name in spans}
+    assert sizes["xq"] == rows * H and sizes["hq"] == rows * I and sizes["y"] == rows * H * 2
+    off, n = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.moe_workspace_region(h, 99, ctypes.byref(off), ctypes.byref(n)) == binding.MOE_ERR_INVALID_ARG
+    L.moe_plan_destroy(h)
+
+
+def test_options_and_unbound_plan(L):
+    rc, h = _plan(L, 64, 256, 512, 8, 2, 0)
+    assert rc == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_MAX_SMS, 16) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TIMEOUT_NS, 0) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_INJECT_FAULT, 2) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, 12345, 1) == binding.MOE_ERR_INVALID_ARG
+    # no workspace bound yet: every compute entry point refuses before touching a device
+    null = [None] * 9
+    assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE
+    assert L.moe_debug_routing(h, *null[:6]) == binding.MOE_ERR_WORKSPACE
+    assert L.moe_set_workspace(h, None, 0) == binding.MOE_ERR_WORKSPACE
+    assert L.moe_forward(None, *null) == binding.MOE_ERR_INVALID_ARG
+    L.moe_plan_destroy(h)
+    L.moe_plan_destroy(None)
+
+
+def test_error_strings(L):
+    for code in range(-6, 1):
+        assert L.moe_error_string(code)
+    assert L.moe_error_string(-99) == b"unknown error"

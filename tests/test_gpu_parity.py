@@ -1,0 +1,257 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on seeded inputs.
+
+Bit-exact: routing ids, dispatch counts/offsets/perm/slot_pos, token-order and
+dispatched E4M3 activation codes and scales.  Within tolerance: gates (fp32 vs
+fp64 softmax) and layer outputs (relative Frobenius <= 5e-3, max-abs <=
+2e-2 * rms(out)).  Sizes span several tiles and ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_fp4_moe_b200 import binding
+from fp8_fp4_moe_b200 import inputs as I
+from oracle import formats as F
+from oracle import moe as M
+
+from parity import assert_output_close, bits, make_case, oracle_forward, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def W(name="t", T=64, H=256, I_=512, E=8, k=2, shared=0, router_std=0.02, bias="zeros"):
+    return I.Workload(name, T=T, H=H, I=I_, E=E, k=k, shared=shared, router_std=router_std, bias=bias)
+
+
+SMALL = {
+    "tiny": I.WORKLOADS["tiny"],
+    "ragged_shared": W("ragged_shared", T=333, H=384, I_=256, E=16, k=4, shared=1, router_std=0.05, bias="uniform"),
+    "t1_k1": W("t1_k1", T=1, H=256, I_=256, E=4, k=1),
+    "k_eq_E": W("k_eq_E", T=50, H=256, I_=384, E=6, k=6, shared=1),
+    "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
+}
+
+
+def plan_for(w):
+    return binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+
+
+# --------------------------------------------------------------------------- quantisation
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_shared"])
+def test_quant_x_bit_exact(cuda_lib, name):
+    w = SMALL[name]
+    x, _, _ = I.make_routing_inputs(w, 3)
+    x = x.clone()
+    x[0, :128] = 0.0                               # all-zero block
+    x[1, 128:256] = torch.tensor(1e-38).to(torch.bfloat16)   # tiny block -> clamped exponent
+    x[2, 5] = -0.0
+    x[2, 6] = -1e-30                               # rounds to -0 after scaling
+    x[min(3, w.T - 1), 7] = 3.0e38                 # huge value
+    p = plan_for(w)
+    xq, xs = p.debug_quant_x(x.cuda())
+    codes, exps = M.quantize_blocks(F.bf16_to_f64(bits(x)))
+    assert np.array_equal(xq.cpu().numpy(), codes)
+    assert np.array_equal(xs.cpu().numpy().astype(np.float64), np.ldexp(1.0, exps))
+
+
+# --------------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "t1_k1", "k_eq_E", "dsv3_like"])
+def test_routing_bit_exact(cuda_lib, name):
+    w = SMALL[name]
+    case = make_case(w, seed=5)
+    p = plan_for(w)
+    d = to_device(case)
+    ids, gates = p.debug_routing(d["x"], d["W_router"], d["bias"])
+    r_ids, r_gates, _ = M.route(bits(case["x"]), case["W_router"].numpy(), case["bias"].numpy(), w.k)
+    assert np.array_equal(ids.cpu().numpy(), r_ids)
+    np.testing.assert_allclose(gates.cpu().numpy(), r_gates, rtol=2e-6, atol=2e-7)
+
+
+def test_routing_exact_ties_lower_id(cuda_lib):
+    # dyadic router rows: fp32 and fp64 logits are exact and tie exactly
+    w = W("ties", T=40, H=256, I_=256, E=8, k=3)
+    x = torch.zeros(w.T, w.H, dtype=torch.bfloat16)
+    x[:, 0] = 1.0
+    x[:, 1] = torch.arange(w.T, dtype=torch.float32).remainder(4).to(torch.bfloat16)
+    Wr = torch.zeros(w.E, w.H)
+    Wr[:, 0] = torch.tensor([0.5, 0.5, 0.25, 0.5, 0.0, 0.25, 0.5, 0.125])
+    Wr[:, 1] = torch.tensor([0.0, 0.0, 0.125, 0.0, 0.25, 0.125, 0.0, 0.0])
+    bias = torch.tensor([0, 0, 0, 0, 0, 0, 0.25, 0], dtype=torch.float32)
+    p = plan_for(w)
+    ids, gates = p.debug_routing(x.cuda(), Wr.cuda(), bias.cuda())
+    r_ids, r_gates, _ = M.route(bits(x), Wr.numpy(), bias.numpy(), w.k)
+    assert np.array_equal(ids.cpu().numpy(), r_ids)
+    np.testing.assert_allclose(gates.cpu().numpy(), r_gates, rtol=1e-6, atol=1e-7)
+    assert r_ids[0].tolist() == [6, 0, 1]          # 0.75 > 0.5 == 0.5 (lower id first)
+
+
+# --------------------------------------------------------------------------- dispatch
+
+def _ids_case(T, E, k, kind, seed=0):
+    rng = np.random.default_rng(seed)
+    if kind == "random":
+        s = rng.normal(size=(T, E))
+    elif kind == "one_expert":      # every token picks expert 0 first (others empty but the top-k)
+        s = rng.normal(size=(T, E)) - 10 * np.arange(E)[None, :]
+    elif kind == "two_experts":
+        s = rng.normal(size=(T, E)) * 1e-3
+        s[:, 3] += 100
+        s[:, 1] += 50
+    else:
+        raise ValueError(kind)
+    return M.select_experts(s, np.zeros(E, np.float32), k)
+
+
+@pytest.mark.parametrize("T,E,k,shared,kind", [
+    (1, 4, 2, 0, "random"), (33, 8, 2, 1, "random"), (1000, 64, 8, 1, "random"), (4097, 16, 4, 0, "random"),
+    (300, 8, 1, 0, "one_expert"), (257, 32, 2, 1, "two_experts"), (64, 5, 5, 0, "random"),
+])
+def test_dispatch_bit_exact(cuda_lib, T, E, k, shared, kind):
+    ids = _ids_case(T, E, k, kind, seed=T)
+    w = W("d", T=T, H=256, I_=256, E=E, k=k, shared=shared)
+    p = plan_for(w)
+    counts, offsets, perm, slot_pos = p.debug_dispatch(torch.from_numpy(ids.astype(np.int32)).cuda())
+    rc, rof, rperm, rslot = M.dispatch(ids, E, shared)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), rof)
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    assert np.array_equal(slot_pos.cpu().numpy(), rslot)
+    assert p.check_status()[0] == 0
+
+
+def test_dispatch_flags_invalid_ids(cuda_lib):
+    w = W("bad", T=40, H=256, I_=256, E=8, k=2)
+    p = plan_for(w)
+    ids = torch.zeros(w.T, w.k, dtype=torch.int32)
+    ids[:, 1] = 1
+    ids[7, 1] = 8            # out of range
+    ids[9, 1] = 0            # duplicate within a token
+    p.debug_dispatch(ids.cuda())
+    code, detail = p.check_status()
+    assert code == binding.MOE_ERR_DEBUG_BOUNDS and detail[3] in (7, 9)
+    assert p.check_status()[0] == 0          # cleared
+
+
+# --------------------------------------------------------------------------- whole layer
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_matches_oracle(cuda_lib, name):
+    w = SMALL[name]
+    case = make_case(w, seed=7)
+    d = to_device(case)
+    p = plan_for(w)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref = oracle_forward(case, w)
+    # routing and dispatch inside the forward are bit-exact
+    assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
+    assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
+    assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
+    assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
+    # dispatched activation codes: row slot_pos[t, j] holds token t's codes
+    xq = p.region("xq").cpu().numpy()
+    xsf = p.region("xsf").cpu().numpy().view(np.uint32)
+    rows = ref["slot_pos"]
+    for j in range(w.k):
+        assert np.array_equal(xq[rows[:, j]], ref["xq"])
+        assert np.array_equal((xsf[rows[:, j]] & 0xFF).astype(np.int64) - 127, ref["xexp"])
+    if w.shared:
+        R = w.T * w.k
+        assert np.array_equal(xq[R:R + w.T], ref["xq"])
+    assert_output_close(bits(out), ref["y"], name)
+
+
+def test_forward_intermediates_match_oracle(cuda_lib):
+    w = SMALL["ragged_shared"]
+    case = make_case(w, seed=8)
+    d = to_device(case)
+    p = plan_for(w)
+    p.forward(**d)
+    ref = oracle_forward(case, w, keep_rows=True)
+    hq = p.region("hq").cpu().numpy()
+    hsf = p.region("hsf").cpu().numpy().view(np.uint32)
+    y = F.bf16_to_f64(bits(p.region("y")))
+    offsets = ref["offsets"]
+    agree = total = 0
+    for e, (lst, res) in ref["rows"].items():
+        # oracle rows for expert e are listed in token order == dispatch order
+        rows = np.arange(offsets[e], offsets[e + 1])
+        assert len(rows) == len(lst)
+        g_h = M.dequantize_blocks(hq[rows], (hsf[rows] & 0xFF).astype(np.int64) - 127)
+        r_h = M.dequantize_blocks(res["hq"], res["hexp"])
+        # an E4M3 code can flip by one step where fp32 and fp64 h straddle a rounding point
+        assert np.linalg.norm(g_h - r_h) <= 1e-2 * np.linalg.norm(r_h) + 1e-30, e
+        agree += int(np.sum(hq[rows] == res["hq"]))
+        total += hq[rows].size
+        ry = res["o"]
+        err = np.linalg.norm(y[rows] - ry) / max(np.linalg.norm(ry), 1e-300)
+        assert err < 5e-3, (e, err)
+    assert agree / total > 0.99         # codes differ only where fp32 and fp64 h straddle a rounding point
+
+
+def test_forward_is_deterministic(cuda_lib):
+    w = SMALL["dsv3_like"]
+    d = to_device(make_case(w, seed=9, screened=False))
+    p = plan_for(w)
+    a = p.forward(**d).clone()
+    b = p.forward(**d).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_forward_all_tokens_on_one_expert(cuda_lib):
+    # the bias forces every token onto expert 2 (many row tiles for one expert, others empty)
+    w = W("skew", T=700, H=256, I_=384, E=8, k=1, shared=1)
+    case = make_case(w, seed=2, screened=False)
+    case["bias"] = torch.tensor([0, 0, 50, 0, 0, 0, 0, 0], dtype=torch.float32)
+    d = to_device(case)
+    p = plan_for(w)
+    out = p.forward(**d)
+    ref = oracle_forward(case, w)
+    assert ref["counts"].tolist() == [0, 0, 700, 0, 0, 0, 0, 0, 700]
+    assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
+    assert_output_close(bits(out), ref["y"], "skew")
+
+
+def test_token_permutation_permutes_output(cuda_lib):
+    w = SMALL["ragged_shared"]
+    case = make_case(w, seed=4, screened=False)
+    d = to_device(case)
+    p = plan_for(w)
+    a = p.forward(**d).clone()
+    pi = torch.randperm(w.T, generator=torch.Generator().manual_seed(0))
+    d2 = dict(d)
+    d2["x"] = d["x"][pi.cuda()].contiguous()
+    b = p.forward(**d2)
+    assert torch.equal(b.view(torch.int16), a[pi.cuda()].view(torch.int16))
+
+
+def test_doubling_w2_scales_doubles_output(cuda_lib):
+    w = SMALL["tiny"]
+    d = to_device(make_case(w, seed=6, screened=False))
+    p = plan_for(w)
+    a = p.forward(**d).clone().float()
+    d["W2_scales"] = d["W2_scales"] + 1
+    b = p.forward(**d).float()
+    assert torch.equal(b, 2 * a)
+
+
+# --------------------------------------------------------------------------- failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    w = SMALL["tiny"]
+    case = make_case(w, seed=1)
+    d = to_device(case)
+    p = plan_for(w)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 50_000_000)      # 50 ms
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 1)             # scale factors of one stage never arrive
+    p.forward(**d)
+    code, detail = p.check_status()
+    assert code == binding.MOE_ERR_DEVICE_TIMEOUT
+    assert detail[1] & 0xF00 in (0x300, 0x400, 0x100, 0x200)
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 0)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 2_000_000_000)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    assert_output_close(bits(out), oracle_forward(case, w)["y"], "after timeout")
