@@ -27,8 +27,9 @@ MOE_OPT_MAX_SMS = 1
 MOE_OPT_TIMEOUT_NS = 2
 MOE_OPT_INJECT_FAULT = 3
 MOE_OPT_PHASE_EVENTS = 5
+MOE_OPT_STATIC_WEIGHTS = 6
 
-PHASES = ["router", "topk_rank", "scan", "scatter_quant", "linear1", "linear2", "combine"]
+PHASES = ["router", "topk_rank", "scan", "scatter_quant", "prepare", "linear1", "linear2", "combine"]
 
 REGIONS = {
     "status": 0, "topk_ids": 1, "gates": 2, "counts": 3, "offsets": 4, "perm": 5, "slot_pos": 6,
@@ -38,7 +39,7 @@ REGIONS = {
 EXPORTED = [
     "moe_plan", "moe_plan_set_option", "moe_workspace_bytes", "moe_set_workspace", "moe_workspace_region",
     "moe_forward", "moe_debug_routing", "moe_debug_dispatch", "moe_debug_quant_x", "moe_check_status",
-    "moe_plan_destroy", "moe_error_string", "moe_phase_times",
+    "moe_plan_destroy", "moe_error_string", "moe_phase_times", "moe_prepare_weights",
 ]
 
 _lib = None
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.moe_debug_quant_x.restype = i32
     L.moe_check_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.moe_check_status.restype = i32
+    L.moe_prepare_weights.argtypes = [vp] * 4
+    L.moe_prepare_weights.restype = i32
     L.moe_phase_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i32]
     L.moe_phase_times.restype = i32
     L.moe_plan_destroy.argtypes = [vp]
@@ -150,11 +153,11 @@ class Plan:
         raw = self.workspace[off.value:off.value + n.value]
         dt = {"status": torch.int32, "topk_ids": torch.int32, "gates": torch.float32, "counts": torch.int32,
               "offsets": torch.int32, "perm": torch.int32, "slot_pos": torch.int32, "xq": torch.uint8,
-              "xsf": torch.int32, "hq": torch.uint8, "hsf": torch.int32, "y": torch.bfloat16}[name]
+              "xsf": torch.uint8, "hq": torch.uint8, "hsf": torch.uint8, "y": torch.bfloat16}[name]
         v = raw.view(dt)
         shapes = {"topk_ids": (self.T, self.k), "gates": (self.T, self.k), "slot_pos": (self.T, self.k),
-                  "xq": (self.rows, self.H), "xsf": (self.rows, self.H // 128), "hq": (self.rows, self.I),
-                  "hsf": (self.rows, self.I // 128), "y": (self.rows, self.H)}
+                  "xq": (self.rows, self.H), "xsf": (-1, self.H // 128, 512), "hq": (self.rows, self.I),
+                  "hsf": (-1, self.I // 128, 512), "y": (self.rows, self.H)}
         return v.view(shapes[name]) if name in shapes else v
 
     def forward(self, x, W_router, bias, W1, W1_scales, W2, W2_scales, out=None, stream=None):
@@ -167,6 +170,11 @@ class Plan:
                                _ptr(W2_scales, torch.uint8, d), _ptr(out, torch.bfloat16, d), _stream_ptr(stream))
         _check(rc, "moe_forward")
         return out
+
+    def prepare_weights(self, W1_scales, W2_scales, stream=None):
+        d = self.device
+        _check(lib().moe_prepare_weights(self._h, _ptr(W1_scales, torch.uint8, d), _ptr(W2_scales, torch.uint8, d),
+                                         _stream_ptr(stream)), "moe_prepare_weights")
 
     def debug_routing(self, x, W_router, bias, stream=None):
         d = self.device

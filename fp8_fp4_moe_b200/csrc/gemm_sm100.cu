@@ -10,23 +10,26 @@
 // ("DeepSeek Mega MoE / DeepGEMM mega kernel", TL;DR and "Thông số kỹ thuật").
 //
 // Design (one CTA per SM, persistent, static round-robin over tiles):
-//   warp 0      TMA producer: A tile 128 x 128 B (SW128) and B tile
-//               256 x 128 FP4 elements, loaded with the 16U4_ALIGN16B type so
-//               the packed nibbles land in the padded shared-memory form the
-//               f8f6f4 MMA reads (128 bytes of shared memory per 128 elements);
+//   warp 0      TMA producer.  Per 128-deep K stage: the A tile 128 x 128 B
+//               (SW128), the B tile 256 x 128 FP4 elements loaded with the
+//               16U4_ALIGN16B type (packed nibbles land in the padded
+//               shared-memory form the f8f6f4 MMA reads: 128 bytes per 128
+//               elements), and the two scale-factor atoms of the stage as
+//               bulk copies (A: 512 B, B: 1024 B) from pre-tiled layouts;
 //   warp 1      TMEM owner and single-thread MMA issuer:
-//               tcgen05.mma.kind::mxf8f6f4.block_scale, M=128, N=256, K=32,
+//               tcgen05.cp of the scale atoms (32x128b.warpx4), then
+//               tcgen05.mma.kind::mxf8f6f4.block_scale M=128 N=256 K=32 x4,
 //               fp32 accumulator in TMEM columns [0, 256);
-//   warp 2      scale-factor loader: cp.async of the UE8M0 scale words into
-//               the 128-row x 4-block atom layout (row r at byte
-//               (r%32)*16 + (r/32)*4, block b at +b), copied to TMEM by the
-//               MMA thread with tcgen05.cp 32x128b.warpx4;
-//   warps 3..6  epilogue: tcgen05.ld of their 32-lane quarter, release the
-//               accumulator, then SwiGLU + requant (linear1) or bf16 (linear2)
-//               and stores.
+//   warps 2..9  epilogue, two warps per 32-lane TMEM quarter, each owning
+//               half of the accumulator columns: tcgen05.ld, release the
+//               accumulator, then SwiGLU + requant (linear1) or bf16 (linear2).
+// Scale-factor atom (128 rows x 4 K-blocks of 32): row r at byte
+// (r % 32) * 16 + (r / 32) * 4, block b at + b; copied to TMEM it gives row r
+// its scale at lane r % 32 (all four sub-partitions), column r / 32, byte b.
 // Tiles never cross experts: expert e owns rows [offsets[e], offsets[e+1]) of
-// the dispatched activations, split into ceil(n_e/128) row tiles; rows of a
-// tile past n_e are computed on whatever the loads return and never stored.
+// the dispatched activations, split into ceil(n_e/128) row tiles (global row
+// tile index mtile_start[e] + mt); rows of a tile past n_e are computed on
+// whatever the loads return and never stored.
 // Every wait is bounded (WaitCtl); on a timeout the CTA records
 // MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM, returns.
 #include "common.cuh"
@@ -37,28 +40,30 @@ namespace moe {
 namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK, S = kGemmStages;
+constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264;
 constexpr uint32_t kATileBytes = BM * BK;            // 16 KB
 constexpr uint32_t kBTileBytes = BN * BK;            // 32 KB in shared memory (unpacked FP4)
 constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
-// Transaction bytes per stage: A 16 KB + B counted at 4 bits per element (16 KB).
-constexpr uint32_t kStageTxBytes = BM * BK + BN * BK / 2;
+// Transaction bytes per stage: A 16 KB, B counted at 4 bits per element (16 KB), scale atoms.
+constexpr uint32_t kStageTxBytes = BM * BK + BN * BK / 2 + kSfaBytes + kSfbBytes;
 
 struct SmemLayout {
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + S * kATileBytes;
   static constexpr uint32_t sfa = b + S * kBTileBytes;
   static constexpr uint32_t sfb = sfa + S * kSfaBytes;
-  static constexpr uint32_t bars = sfb + S * kSfbBytes;
-  // full_tma[S], full_sf[S], empty[S], accf, acce, drain
-  static constexpr uint32_t n_bars = 3 * S + 3;
+  static constexpr uint32_t amax = sfb + S * kSfbBytes;           // [2 buffers][2 halves][128 rows] fp32
+  static constexpr uint32_t bars = amax + 2 * 2 * 128 * 4;
+  // full[S], empty[S], accf, acce, drain
+  static constexpr uint32_t n_bars = 2 * S + 3;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t total = misc + 16;
 };
 
 struct TileCoord {
-  int e, mt, nt, count, row0;
+  int e, mt, nt, count, row0, gmt;   // gmt = global row-tile index
 };
 
 __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
@@ -72,10 +77,12 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
   c.e = lo;
   c.count = __ldg(p.counts + lo);
   const int mtiles = (c.count + BM - 1) / BM;
-  const int local = tile - __ldg(p.mtile_start + lo) * p.n_tiles_n;
+  const int mstart = __ldg(p.mtile_start + lo);
+  const int local = tile - mstart * p.n_tiles_n;
   c.nt = local / mtiles;             // tiles of one expert: n-major, m fastest
   c.mt = local - c.nt * mtiles;
   c.row0 = __ldg(p.offsets + lo) + c.mt * BM;
+  c.gmt = mstart + c.mt;
   return c;
 }
 
@@ -88,40 +95,49 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
   return smem_desc(saddr, 16, 128, kLayoutNoSwizzle);
 }
 
+// Named barrier over the epilogue warps (ids 1..; 0 is __syncthreads).
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+}
+
 template <int MODE>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t tmem_base, int q,
-                                              int lane, uint64_t* acce) {
+                                              int half, int lane, uint64_t* acce, float* amax_s, int buf) {
   const int m = q * 32 + lane;                         // accumulator row = TMEM lane
   const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
   const bool valid = c.mt * BM + m < c.count;
   const long grow = (long)c.row0 + m;
   if constexpr (MODE == 1) {
-    float h[128];
-    float amax = 0.f;
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t g[32], u[32];
-      tmem_ld_32x32b_x32(t_row + kAccCol + ch * 32, g);
-      tmem_ld_32x32b_x32(t_row + kAccCol + 128 + ch * 32, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float gv = __uint_as_float(g[i]);
-        const float uv = __uint_as_float(u[i]);
-        const float hv = gv / (1.0f + expf(-gv)) * uv;   // silu(gate) * up
-        h[ch * 32 + i] = hv;
-        amax = fmaxf(amax, fabsf(hv));
-      }
-    }
+    // this warp: h channels [64*half, 64*half + 64) of the tile's 128
+    uint32_t g[64], u[64];
+    tmem_ld_32x32b_x32(t_row + kAccCol + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+    tmem_ld_32x32b_x32(t_row + kAccCol + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+    tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+    tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+    tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(acce);
+    if (lane == 0) mbar_arrive(acce);                  // accumulator may be overwritten now
+    float h[64];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float gv = __uint_as_float(g[i]);
+      const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);   // silu(gate) * up
+      h[i] = hv;
+      amax = fmaxf(amax, fabsf(hv));
+    }
+    // the 128-channel block's amax spans both halves: exchange through shared memory
+    float* slot = amax_s + buf * 256;
+    slot[half * 128 + m] = amax;
+    epi_bar();
+    amax = fmaxf(amax, slot[(half ^ 1) * 128 + m]);
     if (valid) {
       const int pexp = pow2_exp_e4m3(amax);
       const float sc = exp2_neg(pexp);
-      uint8_t* dst = p.hq + grow * p.N + (long)c.nt * 128;
+      uint8_t* dst = p.hq + grow * p.N + (long)c.nt * 128 + half * 64;
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
+      for (int v = 0; v < 4; ++v) {
         uint4 w;
         w.x = pack_e4m3x4(h[v * 16 + 0] * sc, h[v * 16 + 1] * sc, h[v * 16 + 2] * sc, h[v * 16 + 3] * sc);
         w.y = pack_e4m3x4(h[v * 16 + 4] * sc, h[v * 16 + 5] * sc, h[v * 16 + 6] * sc, h[v * 16 + 7] * sc);
@@ -129,14 +145,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
         w.w = pack_e4m3x4(h[v * 16 + 12] * sc, h[v * 16 + 13] * sc, h[v * 16 + 14] * sc, h[v * 16 + 15] * sc);
         *reinterpret_cast<uint4*>(dst + v * 16) = w;
       }
-      p.hsf[grow * (p.N / 128) + c.nt] = (uint32_t)(pexp + 127) * 0x01010101u;
+      if (half == 0) {
+        // scale word of (row tile gmt, K-tile nt of linear2) in the tiled atom layout
+        uint8_t* atom = reinterpret_cast<uint8_t*>(p.hsf) + ((long)c.gmt * (p.N / 128) + c.nt) * 512;
+        *reinterpret_cast<uint32_t*>(atom + (m % 32) * 16 + (m / 32) * 4) = (uint32_t)(pexp + 127) * 0x01010101u;
+      }
     }
   } else {
-    uint32_t packed[128];
+    // this warp: output columns [128*half, 128*half + 128)
+    uint32_t packed[64];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int ch = 0; ch < 4; ++ch) {
       uint32_t r[32];
-      tmem_ld_32x32b_x32(t_row + kAccCol + ch * 32, r);
+      tmem_ld_32x32b_x32(t_row + kAccCol + half * 128 + ch * 32, r);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -147,19 +168,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(acce);
-    if (valid) {
-      const int col0 = c.nt * BN;
+    const int col0 = c.nt * BN + half * 128;
+    if (valid && col0 < p.N) {
       uint16_t* dst = p.y + grow * p.N + col0;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        if (col0 + ch * 32 < p.N) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w = make_uint4(packed[ch * 16 + v * 4 + 0], packed[ch * 16 + v * 4 + 1],
-                                 packed[ch * 16 + v * 4 + 2], packed[ch * 16 + v * 4 + 3]);
-            *reinterpret_cast<uint4*>(dst + ch * 32 + v * 8) = w;
-          }
-        }
+      for (int v = 0; v < 16; ++v) {
+        uint4 w = make_uint4(packed[v * 4 + 0], packed[v * 4 + 1], packed[v * 4 + 2], packed[v * 4 + 3]);
+        *reinterpret_cast<uint4*>(dst + v * 8) = w;
       }
     }
   }
@@ -176,11 +191,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* b_s = smem + SmemLayout::b;
   uint8_t* sfa_s = smem + SmemLayout::sfa;
   uint8_t* sfb_s = smem + SmemLayout::sfb;
+  float* amax_s = reinterpret_cast<float*>(smem + SmemLayout::amax);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
-  uint64_t* full_tma = bars;
-  uint64_t* full_sf = bars + S;
-  uint64_t* empty = bars + 2 * S;
-  uint64_t* accf = bars + 3 * S;
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* accf = bars + 2 * S;
   uint64_t* acce = accf + 1;
   uint64_t* drain = accf + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
@@ -191,12 +206,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_tma[s], 1);
-      mbar_init(&full_sf[s], 32);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
-    mbar_init(acce, 4);
+    mbar_init(acce, kEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -218,39 +232,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int total_tiles = __ldg(p.mtile_start + p.n_experts) * p.n_tiles_n;
   const int KT = p.K / BK;
 
-  // per-stage fill counters of the TMA producer (for draining on abort)
-  uint32_t fills[S];
-#pragma unroll
-  for (int s = 0; s < S; ++s) fills[s] = 0;
-
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      uint32_t fills[S];
+#pragma unroll
+      for (int s = 0; s < S; ++s) fills[s] = 0;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      bool withhold = p.inject_fault != 0 && blockIdx.x == 0;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const TileCoord c = decode_tile(p, tile);
+        const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
+        const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_tma[stage], kStageTxBytes);
-          tma_load_2d(a_s + stage * kATileBytes, &tmA, kt * BK, c.row0, &full_tma[stage]);
-          if constexpr (MODE == 1) {
-            const int brow = c.e * p.rows_b + c.nt * 128;
-            tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full_tma[stage]);
-            tma_load_2d(b_s + stage * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full_tma[stage]);
+          if (withhold) {
+            withhold = false;            // test hook: this stage never fills
           } else {
-            const int brow = c.e * p.rows_b + c.nt * BN;
-            tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full_tma[stage]);
+            mbar_arrive_expect_tx(&full[stage], kStageTxBytes);
+            tma_load_2d(a_s + stage * kATileBytes, &tmA, kt * BK, c.row0, &full[stage]);
+            if constexpr (MODE == 1) {
+              const int brow = c.e * p.rows_b + c.nt * 128;
+              tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full[stage]);
+              tma_load_2d(b_s + stage * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full[stage]);
+            } else {
+              const int brow = c.e * p.rows_b + c.nt * BN;
+              tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full[stage]);
+            }
+            bulk_load(sfa_s + stage * kSfaBytes, sfa_tile + kt * kSfaBytes, kSfaBytes, &full[stage]);
+            bulk_load(sfb_s + stage * kSfbBytes, sfb_tile + kt * kSfbBytes, kSfbBytes, &full[stage]);
+            fills[stage] += 1;
           }
-          fills[stage] += 1;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
       // wait for our own bulk copies before the CTA may exit (abort path)
 #pragma unroll
       for (int s = 0; s < S; ++s) {
-        if (fills[s] > 0 && !mbar_wait_drain(&full_tma[s], (fills[s] - 1) & 1, p.timeout_ns)) {
+        if (fills[s] > 0 && !mbar_wait_drain(&full[s], (fills[s] - 1) & 1, p.timeout_ns)) {
           report_status(p.status, kStatusTimeout, kWhereGemmDrain, s);
         }
       }
@@ -265,13 +286,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(acce, acc_phase ^ 1, ctl, kWhereGemmMma)) break;
         tc_fence_after();
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full_tma[stage], phase, ctl, kWhereGemmMma + 1) ||
-              !mbar_wait(&full_sf[stage], phase, ctl, kWhereGemmMma + 2)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(&full[stage], phase, ctl, kWhereGemmMma + 1)) { ok = false; break; }
           tc_fence_after();
-          fence_proxy_async_smem();
           const uint32_t sfa_addr = smem_u32(sfa_s + stage * kSfaBytes);
           const uint32_t sfb_addr = smem_u32(sfb_s + stage * kSfbBytes);
           tc_cp_32x128b_warpx4(tmem_base + kSfaCol, sf_desc(sfa_addr));
@@ -296,62 +312,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_commit(drain);
       if (!mbar_wait_drain(drain, 0, p.timeout_ns)) report_status(p.status, kStatusTimeout, kWhereGemmDrain, 9);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale-factor loader
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    bool withhold = p.inject_fault != 0 && blockIdx.x == 0;
-    const int kw_a = p.K / 128;     // u32 words per activation row
-    const int kb_b = p.K / 32;      // bytes per weight scale row
-    const long wrow_max = (long)p.n_experts * p.rows_b - 1;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const TileCoord c = decode_tile(p, tile);
-      for (int kt = 0; kt < KT; ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmSfLoader)) { ok = false; break; }
-        if (withhold) {
-          // test hook: this stage's scale factors never arrive
-          withhold = false;
-        } else {
-          uint8_t* da = sfa_s + stage * kSfaBytes + lane * 16;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;
-            long grow = (long)c.row0 + r;
-            if (grow > p.rows_total - 1) grow = p.rows_total - 1;
-            cp_async_4(da + i * 4, p.sfa + grow * kw_a + kt);
-          }
-          uint8_t* db = sfb_s + stage * kSfbBytes + lane * 16;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int n = lane + 32 * i;
-            long wrow;
-            if constexpr (MODE == 1) {
-              wrow = (long)c.e * p.rows_b + (n < 128 ? c.nt * 128 + n : p.N + c.nt * 128 + (n - 128));
-            } else {
-              wrow = (long)c.e * p.rows_b + (long)c.nt * BN + n;
-            }
-            if (wrow > wrow_max) wrow = wrow_max;
-            cp_async_4(db + (i / 4) * 512 + (i % 4) * 4, p.sfb + wrow * kb_b + kt * 4);
-          }
-          cp_async_arrive_noinc(&full_sf[stage]);
-        }
-        if (++stage == S) { stage = 0; phase ^= 1; }
-      }
-    }
-    cp_async_wait_all();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 3..6)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int half = (warp - 2) / 4;      // which half of the accumulator columns
     uint32_t acc_phase = 0;
+    int buf = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const TileCoord c = decode_tile(p, tile);
       // warp-uniform decision: tcgen05.ld below is .sync.aligned
       const bool ok = mbar_wait(accf, acc_phase, ctl, kWhereGemmEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      epilogue_tile<MODE>(p, c, tmem_base, q, lane, acce);
+      epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf);
       acc_phase ^= 1;
+      buf ^= 1;
     }
   }
 
@@ -362,6 +337,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// Weight scale factors, canonical [n][rows_b][K/32] UE8M0 -> tiled atoms.
+// Block per (expert, 128-row group): the group's K/32-byte rows are staged in
+// shared memory, then written as K/128 atoms of 512 bytes (row r at byte
+// (r%32)*16 + (r/32)*4, its 4 K-blocks at +0..3).  linear1 groups pair gate
+// rows j.. and up rows I + j.. of one 128-channel block into a 1024-byte unit;
+// linear2 groups pair row blocks 2t and 2t+1 of a 256-row tile.
+__global__ void __launch_bounds__(256) tile_weight_scales_kernel(const uint8_t* __restrict__ src,
+                                                                 uint8_t* __restrict__ dst, int rows_b, int K,
+                                                                 int n_tiles_n, int mode, int N) {
+  extern __shared__ uint32_t sm[];                // [128 rows][K/128 words]
+  const int kw = K / 128;
+  const int e = blockIdx.y;
+  const int grp = blockIdx.x;                     // 128-row group within the expert's B rows
+  // which (n-tile, half) this group fills
+  int nt, hf, row_first;
+  if (mode == 1) {                                // rows_b = 2N: groups 0..N/128-1 gate, N/128.. up
+    const int ng = N / 128;
+    hf = grp >= ng;
+    nt = grp - hf * ng;
+    row_first = grp * 128;
+  } else {                                        // rows_b = H (=N): 256-row tiles, 2 halves
+    nt = grp / 2;
+    hf = grp % 2;
+    row_first = grp * 128;
+  }
+  const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src);
+  for (int i = threadIdx.x; i < 128 * kw; i += blockDim.x) {
+    const int r = i / kw, w = i % kw;
+    const int row = row_first + r;
+    sm[i] = row < rows_b ? s32[((long)e * rows_b + row) * kw + w] : 0x7F7F7F7Fu;
+  }
+  __syncthreads();
+  uint8_t* out = dst + ((long)e * n_tiles_n + nt) * kw * 1024 + hf * 512;
+  for (int i = threadIdx.x; i < 32 * kw; i += blockDim.x) {
+    const int kt = i / 32, r0 = i % 32;           // 16-byte chunk r0 of atom kt
+    uint4 v;
+    v.x = sm[(r0 + 0) * kw + kt];
+    v.y = sm[(r0 + 32) * kw + kt];
+    v.z = sm[(r0 + 64) * kw + kt];
+    v.w = sm[(r0 + 96) * kw + kt];
+    *reinterpret_cast<uint4*>(out + (long)kt * 1024 + r0 * 16) = v;
+  }
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
@@ -369,6 +388,8 @@ size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
 cudaError_t gemm_prepare_device() {
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)gemm_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tile_weight_scales_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)gemm_smem_bytes());
@@ -383,6 +404,16 @@ cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, cons
 cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s) {
   grouped_gemm_kernel<2><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
+                                      int n_tiles_n, int mode, int N, cudaStream_t s) {
+  const int groups = mode == 1 ? rows_b / 128 : n_tiles_n * 2;
+  const size_t smem = (size_t)128 * (K / 128) * 4;
+  if (smem > 128 * 1024) return cudaErrorInvalidValue;
+  dim3 grid(groups, n_experts);
+  tile_weight_scales_kernel<<<grid, 256, smem, s>>>(src, dst, rows_b, K, n_tiles_n, mode, N);
   return cudaGetLastError();
 }
 

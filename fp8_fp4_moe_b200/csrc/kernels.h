@@ -12,8 +12,14 @@ constexpr int kGemmBM = 128;      // rows (tokens) per tile
 constexpr int kGemmBN = 256;      // accumulator columns per tile
 constexpr int kGemmBK = 128;      // K per pipeline stage
 constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 224; // 7 warps: TMA, MMA, SF loader, 4 x epilogue
+constexpr int kGemmThreads = 320; // 10 warps: TMA, MMA, 8 x epilogue
 
+// Scale-factor atoms (the unit the MMA's scale copy reads): 128 rows x 4 K-blocks
+// of 32, row r at byte (r%32)*16 + (r/32)*4, K-block b at +b.
+//   activations: [row tile g = mtile_start[e] + mt][K/128] atoms of 512 B, the
+//                row's power-of-two code in all four bytes;
+//   weights:     [expert][n-tile][K/128] units of 1024 B (two atoms: the tile's
+//                B rows 0..127 and 128..255).
 struct GemmArgs {
   int K;               // reduction length (H for linear1, I for linear2)
   int N;               // linear1: I (SwiGLU width); linear2: H (output width)
@@ -24,10 +30,10 @@ struct GemmArgs {
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
   const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
-  const uint32_t* sfa;         // [rows_total][K/128], UE8M0 code in all 4 bytes
-  const uint8_t* sfb;          // [n_experts * rows_b][K/32] UE8M0
+  const uint8_t* sfa;          // activation scale atoms
+  const uint8_t* sfb;          // weight scale units
   uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
-  uint32_t* hsf;               // linear1 out: [rows_total][I/128]
+  uint32_t* hsf;               // linear1 out: activation scale atoms of hq (K = I)
   uint16_t* y;                 // linear2 out: [rows_total][H] bf16
   uint32_t* status;
   uint64_t timeout_ns;
@@ -35,7 +41,10 @@ struct GemmArgs {
 };
 
 size_t gemm_smem_bytes();
-cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attribute
+cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attributes
+// canonical UE8M0 weight scales [n][rows_b][K/32] -> weight scale units
+cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
+                                      int n_tiles_n, int mode, int N, cudaStream_t s);
 cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s);
 cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
@@ -52,10 +61,11 @@ cudaError_t launch_topk_rank(int mode, const float* logits, const float* bias, i
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int T, int E, int k, int shared,
                                  cudaStream_t s);
-// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale words.
+// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms.
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
-                                 const int32_t* group_base, int32_t* slot_pos, int32_t* perm, uint8_t* xq,
-                                 uint32_t* xsf, int T, int H, int E, int k, int shared, cudaStream_t s);
+                                 const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
+                                 int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
+                                 int k, int shared, cudaStream_t s);
 // Token-order quantisation (debug entry point).
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,

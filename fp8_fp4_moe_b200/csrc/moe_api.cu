@@ -24,10 +24,12 @@ struct moe_plan_s {
   int max_sms = 0;
   uint64_t timeout_ns = 2000000000ull;
   int inject_fault = 0;
+  int static_weights = 0;
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
-  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile;
+  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_w1sf, off_w2sf;
+  long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
   // bound state
   uint8_t* ws = nullptr;
@@ -37,6 +39,8 @@ struct moe_plan_s {
   alignas(64) CUtensorMap tmA1, tmA2, tmB1, tmB2;
   const void* w1_cached = nullptr;
   const void* w2_cached = nullptr;
+  const void* w1s_prepared = nullptr;   // weight scales the prepared units were built from
+  const void* w2s_prepared = nullptr;
   // per-phase timing (MOE_OPT_PHASE_EVENTS)
   int phase_events = 0;
   bool events_ready = false;
@@ -95,14 +99,13 @@ int check_bound(moe_plan_t p) {
   return MOE_OK;
 }
 
-GemmArgs gemm_args(moe_plan_t p, int mode, const uint8_t* W_scales) {
+GemmArgs gemm_args(moe_plan_t p, int mode) {
   GemmArgs a{};
   a.n_experts = p->n;
   a.rows_total = (int)p->rows;
   a.counts = region<int32_t>(p, MOE_REGION_COUNTS);
   a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
   a.mtile_start = at<int32_t>(p, p->off_mtile);
-  a.sfb = W_scales;
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
   if (mode == 1) {
@@ -110,7 +113,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode, const uint8_t* W_scales) {
     a.N = p->I;
     a.rows_b = 2 * p->I;
     a.n_tiles_n = p->I / 128;
-    a.sfa = region<uint32_t>(p, MOE_REGION_XSF);
+    a.sfa = region<uint8_t>(p, MOE_REGION_XSF);
+    a.sfb = at<uint8_t>(p, p->off_w1sf);
     a.hq = region<uint8_t>(p, MOE_REGION_HQ);
     a.hsf = region<uint32_t>(p, MOE_REGION_HSF);
     a.inject_fault = p->inject_fault;
@@ -119,7 +123,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode, const uint8_t* W_scales) {
     a.N = p->H;
     a.rows_b = p->H;
     a.n_tiles_n = (p->H + kGemmBN - 1) / kGemmBN;
-    a.sfa = region<uint32_t>(p, MOE_REGION_HSF);
+    a.sfa = region<uint8_t>(p, MOE_REGION_HSF);
+    a.sfb = at<uint8_t>(p, p->off_w2sf);
     a.y = region<uint16_t>(p, MOE_REGION_Y);
     a.inject_fault = 0;
   }
@@ -159,16 +164,37 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
     return cuda_rc(e);
   mark(p, 1 + MOE_PHASE_SCAN, s);
   e = launch_scatter_quant(x, ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
+                           region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile),
                            region<int32_t>(p, MOE_REGION_SLOT_POS), region<int32_t>(p, MOE_REGION_PERM),
-                           region<uint8_t>(p, MOE_REGION_XQ), region<uint32_t>(p, MOE_REGION_XSF), p->T, p->H,
+                           region<uint8_t>(p, MOE_REGION_XQ), region<uint8_t>(p, MOE_REGION_XSF), p->T, p->H,
                            p->E, p->k, p->shared, s);
   mark(p, 1 + MOE_PHASE_SCATTER_QUANT, s);
   return cuda_rc(e);
 }
 
+// Weight scale factors -> the tiled units the GEMMs bulk-load (both weights).
+int prepare_weights(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_scales, cudaStream_t s) {
+  cudaError_t e = launch_tile_weight_scales(W1_scales, at<uint8_t>(p, p->off_w1sf), p->n, 2 * p->I, p->H,
+                                            p->I / 128, 1, p->I, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_tile_weight_scales(W2_scales, at<uint8_t>(p, p->off_w2sf), p->n, p->H, p->I,
+                                (p->H + kGemmBN - 1) / kGemmBN, 2, p->H, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  p->w1s_prepared = W1_scales;
+  p->w2s_prepared = W2_scales;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int moe_prepare_weights(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_scales, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(W1_scales, 4) || !aligned(W2_scales, 4)) return MOE_ERR_INVALID_ARG;
+  return prepare_weights(p, W1_scales, W2_scales, static_cast<cudaStream_t>(stream));
+}
 
 int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   if (!out) return MOE_ERR_INVALID_ARG;
@@ -205,15 +231,18 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   reg(MOE_REGION_PERM, (size_t)R * 4);
   reg(MOE_REGION_SLOT_POS, Tk * 4);
   reg(MOE_REGION_XQ, (size_t)rows * H);
-  reg(MOE_REGION_XSF, (size_t)rows * (H / 128) * 4);
+  p->mt_cap = (rows + kGemmBM - 1) / kGemmBM + p->n;
+  reg(MOE_REGION_XSF, (size_t)p->mt_cap * (H / 128) * 512);
   reg(MOE_REGION_HQ, (size_t)rows * I);
-  reg(MOE_REGION_HSF, (size_t)rows * (I / 128) * 4);
+  reg(MOE_REGION_HSF, (size_t)p->mt_cap * (I / 128) * 512);
   reg(MOE_REGION_Y, (size_t)rows * H * 2);
   p->off_logits = add((size_t)T * E * 4);
   p->off_rank = add(Tk * 4);
   p->off_gcounts = add((size_t)p->G * E * 4);
   p->off_gbase = add((size_t)p->G * E * 4);
   p->off_mtile = add((size_t)(p->n + 1) * 4);
+  p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
+  p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
   p->total = off;
   *out = p;
   return MOE_OK;
@@ -233,6 +262,10 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
     case MOE_OPT_INJECT_FAULT:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->inject_fault = (int)value;
+      return MOE_OK;
+    case MOE_OPT_STATIC_WEIGHTS:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->static_weights = (int)value;
       return MOE_OK;
     case MOE_OPT_ROUTER_TC:
       return value == 0 ? MOE_OK : MOE_ERR_INVALID_ARG;
@@ -271,6 +304,7 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   p->device = dev;
   p->num_sms = sms;
   p->w1_cached = p->w2_cached = nullptr;
+  p->w1s_prepared = p->w2s_prepared = nullptr;
   int rc = encode_2d(&p->tmA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_XQ), p->H, p->rows,
                      p->H, 128, 128);
   if (rc == MOE_OK)
@@ -311,10 +345,14 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
   }
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   if ((rc = run_front(p, xb, W_router, bias, s)) != MOE_OK) return rc;
-  GemmArgs a1 = gemm_args(p, 1, W1_scales);
+  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
+    if ((rc = prepare_weights(p, W1_scales, W2_scales, s)) != MOE_OK) return rc;
+  }
+  mark(p, 1 + MOE_PHASE_PREPARE, s);
+  GemmArgs a1 = gemm_args(p, 1);
   if (launch_gemm_linear1(p->tmA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(p, 1 + MOE_PHASE_LINEAR1, s);
-  GemmArgs a2 = gemm_args(p, 2, W2_scales);
+  GemmArgs a2 = gemm_args(p, 2);
   if (launch_gemm_linear2(p->tmA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(p, 1 + MOE_PHASE_LINEAR2, s);
   cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
@@ -338,7 +376,7 @@ int moe_debug_routing(moe_plan_t p, const void* x, const float* W_router, const 
                       float* gates, void* stream) {
   int rc = check_bound(p);
   if (rc != MOE_OK) return rc;
-  if (!aligned(x, 16) || !aligned(W_router, 4) || !aligned(bias, 4) || !aligned(topk_ids, 4) || !aligned(gates, 4))
+  if (!aligned(x, 16) || !aligned(W_router, 16) || !aligned(bias, 4) || !aligned(topk_ids, 4) || !aligned(gates, 4))
     return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_router_logits(static_cast<const uint16_t*>(x), W_router, at<float>(p, p->off_logits), p->T,
@@ -364,7 +402,8 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), counts, offsets, at<int32_t>(p, p->off_gbase),
                                 at<int32_t>(p, p->off_mtile), p->T, p->E, p->k, p->shared, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase), slot_pos,
+  e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
+                           region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile), slot_pos,
                            perm, nullptr, nullptr, p->T, p->H, p->E, p->k, p->shared, s);
   return cuda_rc(e);
 }

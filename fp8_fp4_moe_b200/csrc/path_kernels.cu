@@ -74,6 +74,54 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
   }
 }
 
+// Warp per (token, chunk of EC experts): for few experts or few tokens, where
+// the tiled kernel above has too little parallelism.  Lane l covers channels
+// [c + 8l, c + 8l + 8) of every 256-channel slice; W rows stream through L1/L2.
+template <int EC>
+__global__ void __launch_bounds__(256) router_logits_warp_kernel(const uint16_t* __restrict__ x,
+                                                                 const float* __restrict__ W,
+                                                                 float* __restrict__ logits, int T, int H, int E) {
+  const int lane = threadIdx.x % 32;
+  const int n_chunks = (E + EC - 1) / EC;
+  const long n_items = (long)T * n_chunks;
+  for (long item = (long)blockIdx.x * 8 + threadIdx.x / 32; item < n_items; item += (long)gridDim.x * 8) {
+    const int t = (int)(item / n_chunks);
+    const int e0 = (int)(item % n_chunks) * EC;
+    float acc[EC];
+#pragma unroll
+    for (int j = 0; j < EC; ++j) acc[j] = 0.f;
+    const uint16_t* xr = x + (long)t * H;
+    for (int cb = 0; cb < H; cb += 256) {
+      const int c0 = cb + lane * 8;
+      if (c0 >= H) break;                       // no shuffles inside this loop
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xr + c0));
+      float xv[8];
+      xv[0] = __uint_as_float(raw.x << 16); xv[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+      xv[2] = __uint_as_float(raw.y << 16); xv[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+      xv[4] = __uint_as_float(raw.z << 16); xv[5] = __uint_as_float(raw.z & 0xFFFF0000u);
+      xv[6] = __uint_as_float(raw.w << 16); xv[7] = __uint_as_float(raw.w & 0xFFFF0000u);
+#pragma unroll
+      for (int j = 0; j < EC; ++j) {
+        if (e0 + j < E) {
+          const float4* wr = reinterpret_cast<const float4*>(W + (long)(e0 + j) * H + c0);
+          const float4 w0 = __ldg(wr), w1 = __ldg(wr + 1);
+          float a = acc[j];
+          a = fmaf(xv[0], w0.x, a); a = fmaf(xv[1], w0.y, a); a = fmaf(xv[2], w0.z, a); a = fmaf(xv[3], w0.w, a);
+          a = fmaf(xv[4], w1.x, a); a = fmaf(xv[5], w1.y, a); a = fmaf(xv[6], w1.z, a); a = fmaf(xv[7], w1.w, a);
+          acc[j] = a;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < EC; ++j) {
+      float v = acc[j];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0 && e0 + j < E) logits[(long)t * E + e0 + j] = v;
+    }
+  }
+}
+
 // --------------------------------------------------------------------------- top-k + rank
 // One block per group of 32 tokens; warp w selects for token 32*g + w.
 // Then warp 0 ranks the group's copies: lane = token, and each expert keeps a
@@ -231,25 +279,36 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
                                                             const int32_t* __restrict__ topk_ids,
                                                             const int32_t* __restrict__ local_rank,
                                                             const int32_t* __restrict__ group_base,
+                                                            const int32_t* __restrict__ offsets,
+                                                            const int32_t* __restrict__ mtile_start,
                                                             int32_t* slot_pos, int32_t* perm, uint8_t* xq,
-                                                            uint32_t* xsf, int T, int H, int E, int k, int shared) {
+                                                            uint8_t* xsf, int T, int H, int E, int k, int shared) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x * 8 + warp;
   if (t >= T) return;
   const int g = t / 32;
   const long R = (long)T * k;
+  const int kw = H / 128;
   int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
+  int e = -1;
   if (lane < k) {
-    const int e = topk_ids[(long)t * k + lane];
+    e = topk_ids[(long)t * k + lane];
     row = group_base[(long)g * E + e] + local_rank[(long)t * k + lane];
     slot_pos[(long)t * k + lane] = row;
     perm[row] = t * k + lane;
   } else if (lane == k && shared) {
+    e = E;
     row = (int)(R + t);
   }
   if (x == nullptr) return;
+  // this destination row's word inside its row tile's scale atoms
+  long sf_off = 0;
+  if (e >= 0) {
+    const int rank = row - offsets[e];
+    const int r = rank % 128;
+    sf_off = ((long)(mtile_start[e] + rank / 128) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
+  }
   const int ndst = k + shared;
-  const int kw = H / 128;
   const uint16_t* xr = x + (long)t * H;
   for (int cb = 0; cb < H; cb += 256) {
     // 8 channels per lane; a 128-channel block spans 16 lanes.  Every lane runs
@@ -276,9 +335,10 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
     const int blk = c0 / 128;
     for (int d = 0; d < ndst; ++d) {
       const long r = __shfl_sync(0xffffffffu, row, d);
+      const long so = __shfl_sync(0xffffffffu, sf_off, d);
       if (active) {
         *reinterpret_cast<uint2*>(xq + r * H + c0) = q;
-        if ((lane & 15) == 0) xsf[r * kw + blk] = code;
+        if ((lane & 15) == 0) *reinterpret_cast<uint32_t*>(xsf + so + (long)blk * 512) = code;
       }
     }
   }
@@ -379,7 +439,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
                                  cudaStream_t s) {
-  if (E <= 16) {
+  if (E <= 32 || (long)T * E <= 16384) {
+    // warp per (token, expert chunk); chunks of 2 when few tokens must cover many experts
+    const int ec = (E <= 32) ? 8 : 2;
+    const long items = (long)T * ((E + ec - 1) / ec);
+    const long blocks = (items + 7) / 8;
+    const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
+    if (ec == 8) router_logits_warp_kernel<8><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+    else router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+  } else if (E <= 16) {
     dim3 grid((T + 63) / 64, (E + 15) / 16);
     router_logits_kernel<16><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
   } else {
@@ -406,10 +474,11 @@ cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, i
 }
 
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
-                                 const int32_t* group_base, int32_t* slot_pos, int32_t* perm, uint8_t* xq,
-                                 uint32_t* xsf, int T, int H, int E, int k, int shared, cudaStream_t s) {
-  scatter_quant_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, topk_ids, local_rank, group_base, slot_pos, perm, xq, xsf,
-                                                   T, H, E, k, shared);
+                                 const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
+                                 int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
+                                 int k, int shared, cudaStream_t s) {
+  scatter_quant_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, topk_ids, local_rank, group_base, offsets, mtile_start,
+                                                   slot_pos, perm, xq, xsf, T, H, E, k, shared);
   return cudaGetLastError();
 }
 

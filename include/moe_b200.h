@@ -68,17 +68,24 @@ enum moe_status_code {
 enum moe_option {
   MOE_OPT_MAX_SMS = 1,         /* persistent GEMM grid size cap (0 = all SMs)            */
   MOE_OPT_TIMEOUT_NS = 2,      /* device wait limit in ns (default 2e9)                  */
-  MOE_OPT_INJECT_FAULT = 3,    /* test hook: 1 = the GEMM1 scale-factor loader withholds
-                                  its first arrival, so the MMA warp's bounded wait runs
-                                  out and the call reports MOE_ERR_DEVICE_TIMEOUT        */
+  MOE_OPT_INJECT_FAULT = 3,    /* test hook: 1 = the linear1 TMA producer of one CTA never
+                                  fills its first pipeline stage, so the MMA warp's
+                                  bounded wait runs out and the call reports
+                                  MOE_ERR_DEVICE_TIMEOUT                                  */
   MOE_OPT_ROUTER_TC = 4,       /* reserved: 1 = tensor-core router (default 0)           */
-  MOE_OPT_PHASE_EVENTS = 5     /* 1 = record a CUDA event after each kernel of moe_forward
+  MOE_OPT_PHASE_EVENTS = 5,    /* 1 = record a CUDA event after each kernel of moe_forward
                                   on its stream, read back with moe_phase_times()        */
+  MOE_OPT_STATIC_WEIGHTS = 6   /* 1 = the caller promises that W1_scales / W2_scales do not
+                                  change between calls that pass the same pointers:
+                                  moe_forward then reuses the tiled scale units built by
+                                  the last moe_prepare_weights (or forward) from those
+                                  pointers.  0 (default): every forward rebuilds them.   */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */
 enum moe_phase {
   MOE_PHASE_ROUTER = 0, MOE_PHASE_TOPK, MOE_PHASE_SCAN, MOE_PHASE_SCATTER_QUANT,
+  MOE_PHASE_PREPARE,     /* weight scale re-layout (zero when reused, MOE_OPT_STATIC_WEIGHTS) */
   MOE_PHASE_LINEAR1, MOE_PHASE_LINEAR2, MOE_PHASE_COMBINE, MOE_PHASE_COUNT_
 };
 
@@ -92,12 +99,20 @@ enum moe_region {
   MOE_REGION_PERM,         /* int32  [R]                                                  */
   MOE_REGION_SLOT_POS,     /* int32  [T, k]                                               */
   MOE_REGION_XQ,           /* uint8  [R + shared*T, H]   E4M3, dispatched row order       */
-  MOE_REGION_XSF,          /* uint32 [R + shared*T, H/128] UE8M0 code in all four bytes  */
+  MOE_REGION_XSF,          /* scale atoms of XQ: [row tile][H/128] x 512 B, see below    */
   MOE_REGION_HQ,           /* uint8  [R + shared*T, I]   E4M3 SwiGLU output               */
-  MOE_REGION_HSF,          /* uint32 [R + shared*T, I/128]                                */
+  MOE_REGION_HSF,          /* scale atoms of HQ: [row tile][I/128] x 512 B               */
   MOE_REGION_Y,            /* bf16   [R + shared*T, H]   expert output rows               */
   MOE_REGION_COUNT_
 };
+
+/* Scale atoms.  Expert e's dispatched rows [offsets[e], offsets[e+1]) form
+ * ceil(count/128) row tiles; row tile g = (sum of the row tiles of experts
+ * before e) + rank/128 holds the row of rank `rank` inside the expert at
+ * r = rank % 128.  Atom (g, kt) is 512 bytes; the row's UE8M0 code (p + 127)
+ * for channels [128 kt, 128 kt + 128) sits in all four bytes at offset
+ * (r % 32) * 16 + (r / 32) * 4.  Bytes of rows past the expert's count are
+ * unspecified. */
 
 /* Create a plan for one layer shape.  Host only; touches no device.
  * `out` receives a heap object the caller releases with moe_plan_destroy(). */
@@ -123,6 +138,12 @@ int moe_forward(moe_plan_t plan, const void* x_bf16, const float* W_router, cons
                 const uint8_t* W1, const uint8_t* W1_scales,
                 const uint8_t* W2, const uint8_t* W2_scales,
                 void* out_bf16, void* stream);
+
+/* Re-lay out the UE8M0 weight scales (canonical [n][rows][K/32]) into the
+ * tiled units the GEMMs load, inside the workspace.  moe_forward does this
+ * itself on every call unless MOE_OPT_STATIC_WEIGHTS is 1 and the pointers
+ * match the last preparation.  Asynchronous on `stream`. */
+int moe_prepare_weights(moe_plan_t plan, const uint8_t* W1_scales, const uint8_t* W2_scales, void* stream);
 
 /* Routing only: topk_ids int32 [T,k] (descending biased score, lower id first
  * on ties) and gates fp32 [T,k] (softmax over the selected unbiased scores). */

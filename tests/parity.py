@@ -53,3 +53,26 @@ def assert_output_close(gpu_out_bits, ref_y, what=""):
     assert rel_frob <= REL_FROB_TOL, f"{what}: rel Frobenius {rel_frob:.3e}"
     assert max_abs <= MAX_ABS_RMS_TOL * rms, f"{what}: max abs {max_abs:.3e} vs rms {rms:.3e}"
     return rel_frob, max_abs, rms
+
+
+def untile_scales(atoms, counts, offsets) -> np.ndarray:
+    """Per-row UE8M0 codes [rows, K/128] from scale atoms [row tiles, K/128, 512] (uint8).
+
+    Row tile g of expert e = (row tiles of experts before e) + rank // 128; the
+    row's code sits at byte (r % 32) * 16 + (r // 32) * 4 of the atom, r = rank % 128.
+    """
+    atoms = np.asarray(atoms, dtype=np.uint8)
+    counts = np.asarray(counts, dtype=np.int64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    mt = (counts + 127) // 128
+    mstart = np.concatenate([[0], np.cumsum(mt)])
+    rows = int(offsets[-1])
+    out = np.zeros((rows, atoms.shape[1]), dtype=np.int64)
+    for e in range(len(counts)):
+        for rank in range(int(counts[e])):
+            g = mstart[e] + rank // 128
+            r = rank % 128
+            word = atoms[g, :, (r % 32) * 16 + (r // 32) * 4:(r % 32) * 16 + (r // 32) * 4 + 4]
+            assert np.all(word == word[:, :1]), "code replicated in all four bytes"
+            out[offsets[e] + rank] = word[:, 0]
+    return out

@@ -14,7 +14,7 @@ from fp8_fp4_moe_b200 import inputs as I
 from oracle import formats as F
 from oracle import moe as M
 
-from parity import assert_output_close, bits, make_case, oracle_forward, to_device
+from parity import assert_output_close, bits, make_case, oracle_forward, to_device, untile_scales
 
 pytestmark = pytest.mark.gpu
 
@@ -152,11 +152,11 @@ def test_forward_matches_oracle(cuda_lib, name):
     assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
     # dispatched activation codes: row slot_pos[t, j] holds token t's codes
     xq = p.region("xq").cpu().numpy()
-    xsf = p.region("xsf").cpu().numpy().view(np.uint32)
+    xsf = untile_scales(p.region("xsf").cpu().numpy(), ref["counts"], ref["offsets"])
     rows = ref["slot_pos"]
     for j in range(w.k):
         assert np.array_equal(xq[rows[:, j]], ref["xq"])
-        assert np.array_equal((xsf[rows[:, j]] & 0xFF).astype(np.int64) - 127, ref["xexp"])
+        assert np.array_equal(xsf[rows[:, j]] - 127, ref["xexp"])
     if w.shared:
         R = w.T * w.k
         assert np.array_equal(xq[R:R + w.T], ref["xq"])
@@ -171,7 +171,7 @@ def test_forward_intermediates_match_oracle(cuda_lib):
     p.forward(**d)
     ref = oracle_forward(case, w, keep_rows=True)
     hq = p.region("hq").cpu().numpy()
-    hsf = p.region("hsf").cpu().numpy().view(np.uint32)
+    hsf = untile_scales(p.region("hsf").cpu().numpy(), ref["counts"], ref["offsets"])
     y = F.bf16_to_f64(bits(p.region("y")))
     offsets = ref["offsets"]
     agree = total = 0
@@ -179,7 +179,7 @@ def test_forward_intermediates_match_oracle(cuda_lib):
         # oracle rows for expert e are listed in token order == dispatch order
         rows = np.arange(offsets[e], offsets[e + 1])
         assert len(rows) == len(lst)
-        g_h = M.dequantize_blocks(hq[rows], (hsf[rows] & 0xFF).astype(np.int64) - 127)
+        g_h = M.dequantize_blocks(hq[rows], hsf[rows] - 127)
         r_h = M.dequantize_blocks(res["hq"], res["hexp"])
         # an E4M3 code can flip by one step where fp32 and fp64 h straddle a rounding point
         assert np.linalg.norm(g_h - r_h) <= 1e-2 * np.linalg.norm(r_h) + 1e-30, e
@@ -235,6 +235,28 @@ def test_doubling_w2_scales_doubles_output(cuda_lib):
     d["W2_scales"] = d["W2_scales"] + 1
     b = p.forward(**d).float()
     assert torch.equal(b, 2 * a)
+
+
+def test_static_weights_reuse_prepared_scales(cuda_lib):
+    w = SMALL["ragged_shared"]
+    case = make_case(w, seed=12, screened=False)
+    d = to_device(case)
+    p = plan_for(w)
+    ref = p.forward(**d).clone()
+    p.set_option(binding.MOE_OPT_STATIC_WEIGHTS, 1)
+    p.prepare_weights(d["W1_scales"], d["W2_scales"])
+    a = p.forward(**d).clone()
+    assert torch.equal(a.view(torch.int16), ref.view(torch.int16))
+    # in-place change of the scales is only seen after an explicit prepare
+    d["W2_scales"].add_(1)
+    stale = p.forward(**d).clone()
+    assert torch.equal(stale.view(torch.int16), ref.view(torch.int16))
+    p.prepare_weights(d["W1_scales"], d["W2_scales"])
+    b = p.forward(**d).float()
+    assert torch.equal(b, 2 * ref.float())
+    p.set_option(binding.MOE_OPT_STATIC_WEIGHTS, 0)
+    c = p.forward(**d).float()
+    assert torch.equal(c, b)
 
 
 # --------------------------------------------------------------------------- failure detection
