@@ -39,7 +39,7 @@ REGIONS = {
 EXPORTED = [
     "moe_plan", "moe_plan_set_option", "moe_workspace_bytes", "moe_set_workspace", "moe_workspace_region",
     "moe_forward", "moe_debug_routing", "moe_debug_dispatch", "moe_debug_quant_x", "moe_check_status",
-    "moe_plan_destroy", "moe_error_string", "moe_phase_times", "moe_prepare_weights",
+    "moe_plan_destroy", "moe_error_string", "moe_phase_times", "moe_prepare_weights", "moe_route_noalloc",
 ]
 
 _lib = None
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.moe_debug_quant_x.restype = i32
     L.moe_check_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.moe_check_status.restype = i32
+    L.moe_route_noalloc.argtypes = [i32, i32, i32, i32] + [vp] * 6
+    L.moe_route_noalloc.restype = i32
     L.moe_prepare_weights.argtypes = [vp] * 4
     L.moe_prepare_weights.restype = i32
     L.moe_phase_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i32]
@@ -118,6 +120,24 @@ def _stream_ptr(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def route_noalloc(x, W_router, bias, k: int, topk_ids=None, gates=None, stream=None):
+    """Routing through moe_route_noalloc: no plan, no workspace, no device allocation
+    inside the library (the outputs are the caller's; pass them to avoid any
+    allocation here too).  Returns (topk_ids int32 [T,k], gates fp32 [T,k])."""
+    d = x.device
+    T, H = x.shape
+    E = W_router.shape[0]
+    if topk_ids is None:
+        topk_ids = torch.empty(T, k, dtype=torch.int32, device=d)
+    if gates is None:
+        gates = torch.empty(T, k, dtype=torch.float32, device=d)
+    rc = lib().moe_route_noalloc(T, H, E, k, _ptr(x, torch.bfloat16, d), _ptr(W_router, torch.float32, d),
+                                 _ptr(bias, torch.float32, d), _ptr(topk_ids, torch.int32, d),
+                                 _ptr(gates, torch.float32, d), _stream_ptr(stream))
+    _check(rc, "moe_route_noalloc")
+    return topk_ids, gates
 
 
 class Plan:

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["gemm_sm100.cu", "path_kernels.cu", "moe_api.cu"]
+SOURCES = ["gemm_sm100.cu", "path_kernels.cu", "moe_api.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

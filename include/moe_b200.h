@@ -150,6 +150,35 @@ int moe_prepare_weights(moe_plan_t plan, const uint8_t* W1_scales, const uint8_t
 int moe_debug_routing(moe_plan_t plan, const void* x_bf16, const float* W_router, const float* bias,
                       int32_t* topk_ids, float* gates, void* stream);
 
+/* Routing without any device allocation.  The pages describe no counterpart:
+ * this entry point exists for callers that cannot allocate device memory when
+ * they need a routing decision -- e.g. code running while another component
+ * owns the CUDA allocator (a serving loop with a fixed, pre-carved memory
+ * pool), hooks that must not call back into an allocator, or runtimes that only
+ * hand over raw stream and buffer pointers.  It needs no plan and no workspace.
+ *
+ * Computes exactly what moe_debug_routing computes (same kernels): topk_ids
+ * int32 [T,k] and gates fp32 [T,k] from x bf16 [T,H], W_router fp32 [E,H] and
+ * bias fp32 [E], all device pointers supplied by the caller (x and W_router
+ * 16-byte aligned).  Its intermediates live in one fixed scratch array of
+ * MOE_ROUTE_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library's device memory;
+ * every device that loads the library holds that array until the process
+ * exits.  The call needs
+ *     r(T*E*4) + r(T*k*4) + r(ceil(T/32)*E*4) + 256  bytes,  r(v) = v rounded up to 256,
+ * and returns MOE_ERR_WORKSPACE (nothing launched) when that exceeds the array
+ * -- about 15,000 tokens at E = 256, k = 8.  Shapes as for moe_plan
+ * (MOE_ERR_UNSUPPORTED_SHAPE otherwise).  Calls no allocating routine.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and leave their intermediates in it:
+ * calls whose kernels can overlap on the GPU (different streams without
+ * ordering between them) race on it, so order them on one stream or by events.
+ * Asynchronous on `stream`. */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int moe_route_noalloc(int T, int H, int E, int k, const void* x_bf16, const float* W_router, const float* bias,
+                      int32_t* topk_ids, float* gates, void* stream);
+
 /* Dispatch only, from given topk_ids int32 [T,k] (each id in [0,E), distinct
  * within a token): counts int32 [n], offsets int32 [n+1], perm int32 [R]
  * (entry t*k+j at the row token t's j-th copy occupies), slot_pos int32 [T,k].
