@@ -122,6 +122,68 @@ __global__ void __launch_bounds__(256) router_logits_warp_kernel(const uint16_t*
   }
 }
 
+// Few experts (E <= 8) with W_router small enough for shared memory: stage it
+// once per block, then each warp takes 4 tokens at a time so every W value read
+// from shared memory feeds 4 FMAs.
+constexpr int kSmemRouterMaxBytes = 200 * 1024;
+__global__ void __launch_bounds__(256) router_logits_smem_kernel(const uint16_t* __restrict__ x,
+                                                                 const float* __restrict__ W,
+                                                                 float* __restrict__ logits, int T, int H, int E) {
+  extern __shared__ float4 w_s4[];
+  const float* w_s = reinterpret_cast<const float*>(w_s4);
+  const int n4 = E * H / 4;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) w_s4[i] = __ldg(reinterpret_cast<const float4*>(W) + i);
+  __syncthreads();
+  const int lane = threadIdx.x % 32;
+  const int groups = (T + 3) / 4;
+  for (int grp = blockIdx.x * 8 + threadIdx.x / 32; grp < groups; grp += gridDim.x * 8) {
+    const int t0 = grp * 4;
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int cb = 0; cb < H; cb += 256) {
+      const int c0 = cb + lane * 8;
+      if (c0 >= H) break;                       // no shuffles inside this loop
+      float xv[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (t0 + i < T) raw = __ldg(reinterpret_cast<const uint4*>(x + (long)(t0 + i) * H + c0));
+        xv[i][0] = __uint_as_float(raw.x << 16); xv[i][1] = __uint_as_float(raw.x & 0xFFFF0000u);
+        xv[i][2] = __uint_as_float(raw.y << 16); xv[i][3] = __uint_as_float(raw.y & 0xFFFF0000u);
+        xv[i][4] = __uint_as_float(raw.z << 16); xv[i][5] = __uint_as_float(raw.z & 0xFFFF0000u);
+        xv[i][6] = __uint_as_float(raw.w << 16); xv[i][7] = __uint_as_float(raw.w & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < E) {
+          const float4 w0 = *reinterpret_cast<const float4*>(w_s + (long)j * H + c0);
+          const float4 w1 = *reinterpret_cast<const float4*>(w_s + (long)j * H + c0 + 4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float a = acc[i][j];
+            a = fmaf(xv[i][0], w0.x, a); a = fmaf(xv[i][1], w0.y, a); a = fmaf(xv[i][2], w0.z, a);
+            a = fmaf(xv[i][3], w0.w, a); a = fmaf(xv[i][4], w1.x, a); a = fmaf(xv[i][5], w1.y, a);
+            a = fmaf(xv[i][6], w1.z, a); a = fmaf(xv[i][7], w1.w, a);
+            acc[i][j] = a;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = acc[i][j];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0 && j < E && t0 + i < T) logits[(long)(t0 + i) * E + j] = v;
+      }
+  }
+}
+
 // --------------------------------------------------------------------------- top-k + rank
 // One block per group of 32 tokens; warp w selects for token 32*g + w.
 // Then warp 0 ranks the group's copies: lane = token, and each expert keeps a
@@ -439,7 +501,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
                                  cudaStream_t s) {
-  if (E <= 32 || (long)T * E <= 16384) {
+  if (E <= 8 && (size_t)E * H * 4 <= kSmemRouterMaxBytes && T >= 64) {
+    static bool attr_set[64] = {};      // the shared-memory opt-in, once per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(router_logits_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kSmemRouterMaxBytes);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    const int groups = (T + 3) / 4;
+    int grid = (groups + 7) / 8;
+    if (grid > 148) grid = 148;
+    router_logits_smem_kernel<<<grid, 256, (size_t)E * H * 4, s>>>(x, W_r, logits, T, H, E);
+  } else if (E <= 32 || (long)T * E <= 16384) {
     // warp per (token, expert chunk); chunks of 2 when few tokens must cover many experts
     const int ec = (E <= 32) ? 8 : 2;
     const long items = (long)T * ((E + ec - 1) / ec);

@@ -12,6 +12,17 @@ from oracle import screen
 # Output tolerance of the layer (relative Frobenius, and max-abs relative to rms(out)).
 REL_FROB_TOL = 5e-3
 MAX_ABS_RMS_TOL = 2e-2
+# Gates: fp32 router logits over up to H = 7168 products differ from fp64 by
+# ~1e-6..1e-5; a softmax gate's relative error is at most twice the largest
+# logit error.
+GATE_RTOL, GATE_ATOL = 1e-4, 1e-6
+
+
+def bf16_half_ulp(y):
+    """Half the bf16 spacing at |y|: the rounding error any bf16 output may carry."""
+    a = np.abs(np.asarray(y, dtype=np.float64))
+    _, e = np.frexp(np.maximum(a, 2.0 ** -126))     # a in [2^(e-1), 2^e)
+    return np.ldexp(1.0, e - 1 - 8)
 
 
 def bits(x: torch.Tensor) -> np.ndarray:
@@ -48,10 +59,23 @@ def output_errors(gpu_out_bits: np.ndarray, ref_y: np.ndarray):
 
 
 def assert_output_close(gpu_out_bits, ref_y, what=""):
+    """Relative Frobenius <= 5e-3 and, per element, |out - y| <= 2e-2 * rms(y) on top of
+    the half-ulp the bf16 output format itself may need at that element.
+
+    y is the oracle's float64 output before its final bf16 rounding.  The
+    half-ulp allowance matters only in the tail: at |y| >= 5.12 * rms the bf16
+    rounding alone (up to 2^-8 |y|) exceeds 2e-2 * rms, which a full-size
+    output (millions of values) reaches even when computed exactly.
+    """
     rel_frob, max_abs, rms = output_errors(gpu_out_bits, ref_y)
-    assert np.all(np.isfinite(F.bf16_to_f64(gpu_out_bits))), what
+    got = F.bf16_to_f64(gpu_out_bits)
+    assert np.all(np.isfinite(got)), what
     assert rel_frob <= REL_FROB_TOL, f"{what}: rel Frobenius {rel_frob:.3e}"
-    assert max_abs <= MAX_ABS_RMS_TOL * rms, f"{what}: max abs {max_abs:.3e} vs rms {rms:.3e}"
+    excess = np.abs(got - ref_y) - bf16_half_ulp(ref_y)
+    worst = int(np.argmax(excess))
+    assert excess.flat[worst] <= MAX_ABS_RMS_TOL * rms, (
+        f"{what}: |out - y| beyond the bf16 half-ulp {excess.flat[worst]:.3e} > {MAX_ABS_RMS_TOL} * rms "
+        f"({rms:.3e}) at y={ref_y.flat[worst]:.5f}, out={got.flat[worst]:.5f}; raw max abs {max_abs:.3e}")
     return rel_frob, max_abs, rms
 
 

@@ -12,7 +12,7 @@ import torch
 from fp8_fp4_moe_b200 import binding
 from fp8_fp4_moe_b200 import inputs as I
 
-from parity import assert_output_close, bits, make_case, oracle_forward
+from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, oracle_forward
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -39,7 +39,7 @@ def test_full_size_sampled_parity(cuda_lib, name):
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
     assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
     assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
-    np.testing.assert_allclose(p.region("gates").cpu().numpy(), ref["gates"], rtol=2e-6, atol=2e-7)
+    np.testing.assert_allclose(p.region("gates").cpu().numpy(), ref["gates"], rtol=GATE_RTOL, atol=GATE_ATOL)
     got = bits(out)[tokens]
     assert_output_close(got, ref["y"], name)
     assert torch.isfinite(out.float()).all()

@@ -14,7 +14,7 @@ from fp8_fp4_moe_b200 import inputs as I
 from oracle import formats as F
 from oracle import moe as M
 
-from parity import assert_output_close, bits, make_case, oracle_forward, to_device, untile_scales
+from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, oracle_forward, to_device, untile_scales
 
 pytestmark = pytest.mark.gpu
 
@@ -66,7 +66,7 @@ def test_routing_bit_exact(cuda_lib, name):
     ids, gates = p.debug_routing(d["x"], d["W_router"], d["bias"])
     r_ids, r_gates, _ = M.route(bits(case["x"]), case["W_router"].numpy(), case["bias"].numpy(), w.k)
     assert np.array_equal(ids.cpu().numpy(), r_ids)
-    np.testing.assert_allclose(gates.cpu().numpy(), r_gates, rtol=2e-6, atol=2e-7)
+    np.testing.assert_allclose(gates.cpu().numpy(), r_gates, rtol=GATE_RTOL, atol=GATE_ATOL)
 
 
 def test_routing_exact_ties_lower_id(cuda_lib):
