@@ -17,7 +17,8 @@ namespace moe {
 enum : int { kStatusTimeout = -4, kStatusBounds = -6 };
 enum : uint32_t {
   kWhereGemmProducer = 0x100, kWhereGemmSfLoader = 0x200, kWhereGemmMma = 0x300,
-  kWhereGemmEpilogue = 0x400, kWhereGemmDrain = 0x500
+  kWhereGemmEpilogue = 0x400, kWhereGemmDrain = 0x500, kWhereRouterProducer = 0x600, kWhereRouterMma = 0x700,
+  kWhereRouterEpilogue = 0x800
 };
 
 __device__ __forceinline__ void report_status(uint32_t* status, int code, uint32_t where, uint32_t detail) {
@@ -150,6 +151,26 @@ __device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
+}
+
+// D(tmem) (+)= A(smem) x B(smem)^T, bf16 operands, fp32 accumulator.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::f16: A = B = bf16, both K-major, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4)                    // accumulator format: f32
+         | (1u << 7)                  // A format: bf16
+         | (1u << 10)                 // B format: bf16
+         | ((uint32_t)(N >> 3) << 17) // N / 8
+         | ((uint32_t)(M >> 4) << 24); // M / 16
 }
 
 // Copy 32 rows x 16 bytes of shared memory into 32 lanes x 4 columns of tmem,

@@ -381,7 +381,171 @@ __global__ void __launch_bounds__(256) tile_weight_scales_kernel(const uint8_t* 
   }
 }
 
+// ------------------------------------------------------------------ router on tensor cores
+// logits[t][e] = sum_h x[t][h] * (W_hi[e][h] + W_lo[e][h]) with W = W_hi + W_lo + r, W_hi and W_lo
+// bf16 (|r| <= 2^-18 |W|): two bf16 MMAs per K slice into one fp32 accumulator.
+// One CTA per (128-token, 128-expert) tile: warp 0 TMA, warp 1 MMA (+TMEM), warps 2..5 epilogue.
+constexpr int RBK = 64;                                 // bf16 elements per stage = 128 bytes
+constexpr int RBN = 128;
+constexpr int RS = 4;
+constexpr uint32_t kRTile = 128 * 128;                  // bytes of one 128-row x 128-byte tile
+
+struct RouterSmem {
+  static constexpr uint32_t a = 0;
+  static constexpr uint32_t bh = a + RS * kRTile;
+  static constexpr uint32_t bl = bh + RS * kRTile;
+  static constexpr uint32_t bars = bl + RS * kRTile;    // full[RS], empty[RS], accf, drain
+  static constexpr uint32_t misc = bars + (2 * RS + 2) * 8;
+  static constexpr uint32_t total = misc + 16;
+};
+
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
+                     const __grid_constant__ CUtensorMap tmWlo, const RouterArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_s = smem + RouterSmem::a;
+  uint8_t* bh_s = smem + RouterSmem::bh;
+  uint8_t* bl_s = smem + RouterSmem::bl;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RouterSmem::bars);
+  uint64_t* empty = full + RS;
+  uint64_t* accf = full + 2 * RS;
+  uint64_t* drain = accf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RouterSmem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RouterSmem::misc + 4);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * RBN;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  const int KT = p.H / RBK;
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t fills[RS];
+#pragma unroll
+      for (int s = 0; s < RS; ++s) fills[s] = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereRouterProducer)) break;
+        mbar_arrive_expect_tx(&full[stage], 3 * kRTile);
+        tma_load_2d(a_s + stage * kRTile, &tmX, kt * RBK, m0, &full[stage]);
+        tma_load_2d(bh_s + stage * kRTile, &tmWhi, kt * RBK, n0, &full[stage]);
+        tma_load_2d(bl_s + stage * kRTile, &tmWlo, kt * RBK, n0, &full[stage]);
+        fills[stage] += 1;
+        if (++stage == RS) { stage = 0; phase ^= 1; }
+      }
+#pragma unroll
+      for (int s = 0; s < RS; ++s)
+        if (fills[s] > 0 && !mbar_wait_drain(&full[s], (fills[s] - 1) & 1, p.timeout_ns))
+          report_status(p.status, kStatusTimeout, kWhereGemmDrain, 0x20 + s);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      constexpr uint32_t idesc = idesc_bf16(128, RBN);
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!mbar_wait(&full[stage], phase, ctl, kWhereRouterMma)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(a_s + stage * kRTile);
+        const uint32_t bh_addr = smem_u32(bh_s + stage * kRTile);
+        const uint32_t bl_addr = smem_u32(bl_s + stage * kRTile);
+#pragma unroll
+        for (int kb = 0; kb < RBK / 16; ++kb)
+          tc_mma_bf16(tmem_base, sw128_desc(a_addr + kb * 32), sw128_desc(bh_addr + kb * 32), idesc, (kt | kb) != 0);
+#pragma unroll
+        for (int kb = 0; kb < RBK / 16; ++kb)
+          tc_mma_bf16(tmem_base, sw128_desc(a_addr + kb * 32), sw128_desc(bl_addr + kb * 32), idesc, 1);
+        tc_commit(&empty[stage]);
+        if (++stage == RS) { stage = 0; phase ^= 1; }
+      }
+      if (ok) tc_commit(accf);
+      tc_commit(drain);
+      if (!mbar_wait_drain(drain, 0, p.timeout_ns)) report_status(p.status, kStatusTimeout, kWhereGemmDrain, 0x29);
+    }
+  } else {
+    const int q = warp & 3;
+    const bool ok = mbar_wait(accf, 0, ctl, kWhereRouterEpilogue);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const int t = m0 + q * 32 + lane;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+#pragma unroll
+      for (int ch = 0; ch < RBN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + ch * 32, r);
+        tmem_ld_wait();
+        const int e0 = n0 + ch * 32;
+        if (t < p.T) {
+          float* dst = p.logits + (long)t * p.E + e0;
+          if (e0 + 32 <= p.E) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              *reinterpret_cast<float4*>(dst + 4 * v) =
+                  make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                              __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (e0 + i < p.E) dst[i] = __uint_as_float(r[i]);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 128);
+  }
+}
+
+// W fp32 -> (hi, lo) bf16 with hi = bf16(W), lo = bf16(W - hi) (W - hi is exact in fp32).
+__global__ void split_router_weights_kernel(const float* __restrict__ W, __nv_bfloat16* __restrict__ hi,
+                                            __nv_bfloat16* __restrict__ lo, long n) {
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const float w = W[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(w);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(w - __bfloat162float(h));
+  }
+}
+
 }  // namespace
+
+size_t router_tc_smem_bytes() { return RouterSmem::total + 1024; }
+
+cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
+                             const RouterArgs& args, cudaStream_t s) {
+  dim3 grid((args.E + RBN - 1) / RBN, (args.T + 127) / 128);
+  router_tc_kernel<<<grid, kRouterThreads, router_tc_smem_bytes(), s>>>(x, whi, wlo, args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* lo, long n, cudaStream_t s) {
+  split_router_weights_kernel<<<296, 256, 0, s>>>(W, reinterpret_cast<__nv_bfloat16*>(hi),
+                                                  reinterpret_cast<__nv_bfloat16*>(lo), n);
+  return cudaGetLastError();
+}
 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
 
@@ -390,6 +554,9 @@ cudaError_t gemm_prepare_device() {
                                        (int)gemm_smem_bytes());
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tile_weight_scales_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)router_tc_smem_bytes());
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)gemm_smem_bytes());

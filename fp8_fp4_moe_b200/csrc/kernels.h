@@ -50,6 +50,21 @@ cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, cons
 cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s);
 
+// ---- router on tensor cores (gemm_sm100.cu) -------------------------------------
+constexpr int kRouterThreads = 192;   // 6 warps: TMA, MMA, 4 x epilogue
+struct RouterArgs {
+  int T, H, E;
+  float* logits;                      // [T][E] fp32
+  uint32_t* status;
+  uint64_t timeout_ns;
+};
+size_t router_tc_smem_bytes();
+// x bf16 [T][H] and W_hi / W_lo bf16 [E][H] as 128-byte-swizzled TMA maps (box 64 x 128).
+cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
+                             const RouterArgs& args, cudaStream_t s);
+// W fp32 [n] -> hi = bf16(W), lo = bf16(W - hi)
+cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* lo, long n, cudaStream_t s);
+
 // ---- routing / dispatch / combine (path_kernels.cu) -----------------------------
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
                                  cudaStream_t s);

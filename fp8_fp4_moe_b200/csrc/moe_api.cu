@@ -25,10 +25,11 @@ struct moe_plan_s {
   uint64_t timeout_ns = 2000000000ull;
   int inject_fault = 0;
   int static_weights = 0;
+  int router_tc = 1;
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
-  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_w1sf, off_w2sf;
+  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_w1sf, off_w2sf, off_whi, off_wlo;
   long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
   // bound state
@@ -36,7 +37,9 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   int device = -1;
   int num_sms = 0;
-  alignas(64) CUtensorMap tmA1, tmA2, tmB1, tmB2;
+  alignas(64) CUtensorMap tmA1, tmA2, tmB1, tmB2, tmX, tmWhi, tmWlo;
+  const void* x_cached = nullptr;        // tmX encodes this x pointer
+  const void* wr_prepared = nullptr;     // W_router the hi/lo split was made from
   const void* w1_cached = nullptr;
   const void* w2_cached = nullptr;
   const void* w1s_prepared = nullptr;   // weight scales the prepared units were built from
@@ -144,14 +147,37 @@ void mark(moe_plan_t p, int i, cudaStream_t s) {
   if (p->phase_events && p->events_ready) cudaEventRecord(p->ev[i], s);
 }
 
+// Tensor-core router for enough tokens and a multiple of 16 experts; CUDA cores otherwise.
+bool use_tc_router(moe_plan_t p) { return p->router_tc && p->T >= 256 && p->E >= 16 && p->E % 16 == 0; }
+
+// logits [T][E] fp32 into the workspace
+int run_router(moe_plan_t p, const uint16_t* x, const float* W_router, cudaStream_t s) {
+  if (!use_tc_router(p))
+    return cuda_rc(launch_router_logits(x, W_router, at<float>(p, p->off_logits), p->T, p->H, p->E, s));
+  if (!p->static_weights || W_router != p->wr_prepared) {
+    if (launch_split_router_weights(W_router, at<uint16_t>(p, p->off_whi), at<uint16_t>(p, p->off_wlo),
+                                    (long)p->E * p->H, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    p->wr_prepared = W_router;
+  }
+  if (x != p->x_cached) {
+    int rc = encode_2d(&p->tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, p->H, p->T, 2ull * p->H, 64, 128);
+    if (rc != MOE_OK) return rc;
+    p->x_cached = x;
+  }
+  RouterArgs ra{p->T, p->H, p->E, at<float>(p, p->off_logits), region<uint32_t>(p, MOE_REGION_STATUS),
+                p->timeout_ns};
+  return cuda_rc(launch_router_tc(p->tmX, p->tmWhi, p->tmWlo, ra, s));
+}
+
 // routing + dispatch + quantisation into the workspace
 int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias, cudaStream_t s) {
   int32_t* ids = region<int32_t>(p, MOE_REGION_TOPK_IDS);
   float* gates = region<float>(p, MOE_REGION_GATES);
   cudaError_t e;
   mark(p, 0, s);
-  if ((e = launch_router_logits(x, W_router, at<float>(p, p->off_logits), p->T, p->H, p->E, s)) != cudaSuccess)
-    return cuda_rc(e);
+  int rc = run_router(p, x, W_router, s);
+  if (rc != MOE_OK) return rc;
   mark(p, 1 + MOE_PHASE_ROUTER, s);
   if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, ids, gates, at<int32_t>(p, p->off_rank),
                             at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E,
@@ -243,6 +269,8 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_mtile = add((size_t)(p->n + 1) * 4);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
+  p->off_whi = add((size_t)E * H * 2);
+  p->off_wlo = add((size_t)E * H * 2);
   p->total = off;
   *out = p;
   return MOE_OK;
@@ -268,7 +296,9 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       p->static_weights = (int)value;
       return MOE_OK;
     case MOE_OPT_ROUTER_TC:
-      return value == 0 ? MOE_OK : MOE_ERR_INVALID_ARG;
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->router_tc = (int)value;
+      return MOE_OK;
     case MOE_OPT_PHASE_EVENTS:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->phase_events = (int)value;
@@ -305,11 +335,18 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   p->num_sms = sms;
   p->w1_cached = p->w2_cached = nullptr;
   p->w1s_prepared = p->w2s_prepared = nullptr;
+  p->x_cached = p->wr_prepared = nullptr;
   int rc = encode_2d(&p->tmA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_XQ), p->H, p->rows,
                      p->H, 128, 128);
   if (rc == MOE_OK)
     rc = encode_2d(&p->tmA2, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_HQ), p->I, p->rows,
                    p->I, 128, 128);
+  if (rc == MOE_OK)
+    rc = encode_2d(&p->tmWhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, at<uint16_t>(p, p->off_whi), p->H, p->E,
+                   2ull * p->H, 64, 128);
+  if (rc == MOE_OK)
+    rc = encode_2d(&p->tmWlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, at<uint16_t>(p, p->off_wlo), p->H, p->E,
+                   2ull * p->H, 64, 128);
   if (rc != MOE_OK) {
     p->ws = nullptr;
     return rc;
@@ -379,10 +416,9 @@ int moe_debug_routing(moe_plan_t p, const void* x, const float* W_router, const 
   if (!aligned(x, 16) || !aligned(W_router, 16) || !aligned(bias, 4) || !aligned(topk_ids, 4) || !aligned(gates, 4))
     return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_router_logits(static_cast<const uint16_t*>(x), W_router, at<float>(p, p->off_logits), p->T,
-                                       p->H, p->E, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, topk_ids, gates, at<int32_t>(p, p->off_rank),
+  rc = run_router(p, static_cast<const uint16_t*>(x), W_router, s);
+  if (rc != MOE_OK) return rc;
+  cudaError_t e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, topk_ids, gates, at<int32_t>(p, p->off_rank),
                        at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   return cuda_rc(e);
 }

@@ -72,14 +72,18 @@ enum moe_option {
                                   fills its first pipeline stage, so the MMA warp's
                                   bounded wait runs out and the call reports
                                   MOE_ERR_DEVICE_TIMEOUT                                  */
-  MOE_OPT_ROUTER_TC = 4,       /* reserved: 1 = tensor-core router (default 0)           */
+  MOE_OPT_ROUTER_TC = 4,       /* 1 (default): router logits on tensor cores when T >= 256
+                                  and E % 16 == 0, as x (bf16) times W_router split into two
+                                  bf16 parts (hi = bf16(W), lo = bf16(W - hi); |residual| <=
+                                  2^-18 |W|) accumulated in fp32; 0: fp32 FMA on CUDA cores */
   MOE_OPT_PHASE_EVENTS = 5,    /* 1 = record a CUDA event after each kernel of moe_forward
                                   on its stream, read back with moe_phase_times()        */
-  MOE_OPT_STATIC_WEIGHTS = 6   /* 1 = the caller promises that W1_scales / W2_scales do not
-                                  change between calls that pass the same pointers:
-                                  moe_forward then reuses the tiled scale units built by
-                                  the last moe_prepare_weights (or forward) from those
-                                  pointers.  0 (default): every forward rebuilds them.   */
+  MOE_OPT_STATIC_WEIGHTS = 6   /* 1 = the caller promises that W_router / W1_scales /
+                                  W2_scales do not change between calls that pass the same
+                                  pointers: moe_forward then reuses the tiled scale units
+                                  and the split router weights built by the last
+                                  moe_prepare_weights (or forward) from those pointers.
+                                  0 (default): every forward rebuilds them.              */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */
@@ -157,7 +161,8 @@ int moe_debug_routing(moe_plan_t plan, const void* x_bf16, const float* W_router
  * pool), hooks that must not call back into an allocator, or runtimes that only
  * hand over raw stream and buffer pointers.  It needs no plan and no workspace.
  *
- * Computes exactly what moe_debug_routing computes (same kernels): topk_ids
+ * Computes exactly what moe_debug_routing computes with MOE_OPT_ROUTER_TC = 0
+ * (same kernels: the fp32 CUDA-core router, then the same top-k): topk_ids
  * int32 [T,k] and gates fp32 [T,k] from x bf16 [T,H], W_router fp32 [E,H] and
  * bias fp32 [E], all device pointers supplied by the caller (x and W_router
  * 16-byte aligned).  Its intermediates live in one fixed scratch array of

@@ -29,6 +29,8 @@ SMALL = {
     "t1_k1": W("t1_k1", T=1, H=256, I_=256, E=4, k=1),
     "k_eq_E": W("k_eq_E", T=50, H=256, I_=384, E=6, k=6, shared=1),
     "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
+    # T >= 256 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
+    "tc_router": W("tc_router", T=300, H=1024, I_=256, E=48, k=4, shared=1, router_std=0.02, bias="uniform"),
 }
 
 
@@ -57,7 +59,7 @@ def test_quant_x_bit_exact(cuda_lib, name):
 
 # --------------------------------------------------------------------------- routing
 
-@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "t1_k1", "k_eq_E", "dsv3_like"])
+@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "t1_k1", "k_eq_E", "dsv3_like", "tc_router"])
 def test_routing_bit_exact(cuda_lib, name):
     w = SMALL[name]
     case = make_case(w, seed=5)

@@ -24,6 +24,7 @@ GATE_RTOL, GATE_ATOL = 2e-6, 2e-7
 def test_route_noalloc_matches_plan_routing_on_two_calls(cuda_lib):
     w = I.Workload("noalloc", T=333, H=512, I=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform")
     plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+    plan.set_option(binding.MOE_OPT_ROUTER_TC, 0)      # the router kernels the entry point runs
     ids = torch.empty(w.T, w.k, dtype=torch.int32, device="cuda")
     gates = torch.empty(w.T, w.k, dtype=torch.float32, device="cuda")
     for seed in (21, 22):
