@@ -55,7 +55,8 @@ struct SmemLayout {
   static constexpr uint32_t sfa = b + S * kBTileBytes;
   static constexpr uint32_t sfb = sfa + S * kSfaBytes;
   static constexpr uint32_t amax = sfb + S * kSfbBytes;           // [2 buffers][2 halves][128 rows] fp32
-  static constexpr uint32_t bars = amax + 2 * 2 * 128 * 4;
+  static constexpr uint32_t stage_out = amax + 2 * 2 * 128 * 4;   // [8 epilogue warps][32 rows][64 B]
+  static constexpr uint32_t bars = stage_out + 8 * 2048;
   // full[S], empty[S], accf, acce, drain
   static constexpr uint32_t n_bars = 2 * S + 3;
   static constexpr uint32_t misc = bars + n_bars * 8;
@@ -100,13 +101,35 @@ __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
 }
 
+// Store 64 bytes of each of the warp's 32 rows (lane l holds row l's bytes in v[0..3]) so that
+// every global store instruction writes whole 32-byte sectors: the chunk goes through a
+// 2 KB per-warp shared buffer (16-byte pieces XOR-swizzled against bank conflicts) and
+// comes back with 4 lanes per row.  dst0 = address of lane 0's row, row_stride in bytes;
+// only rows with row_ok set (in the owning lane) are written.
+__device__ __forceinline__ void store_rows_64b(uint8_t* buf, const uint4 (&v)[4], uint8_t* dst0, long row_stride,
+                                               bool row_ok, int lane) {
+  const uint32_t okmask = __ballot_sync(0xffffffffu, row_ok);
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16)) = v[c];
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int r = it * 8 + (lane >> 2);
+    const int c = lane & 3;
+    const uint4 w = *reinterpret_cast<const uint4*>(buf + r * 64 + ((c ^ ((r >> 1) & 3)) * 16));
+    if (okmask & (1u << r)) *reinterpret_cast<uint4*>(dst0 + r * row_stride + c * 16) = w;
+  }
+  __syncwarp();
+}
+
 template <int MODE>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t tmem_base, int q,
-                                              int half, int lane, uint64_t* acce, float* amax_s, int buf) {
+                                              int half, int lane, uint64_t* acce, float* amax_s, int buf,
+                                              uint8_t* obuf) {
   const int m = q * 32 + lane;                         // accumulator row = TMEM lane
   const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
   const bool valid = c.mt * BM + m < c.count;
-  const long grow = (long)c.row0 + m;
   if constexpr (MODE == 1) {
     // this warp: h channels [64*half, 64*half + 64) of the tile's 128
     uint32_t g[64], u[64];
@@ -132,19 +155,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     slot[half * 128 + m] = amax;
     epi_bar();
     amax = fmaxf(amax, slot[(half ^ 1) * 128 + m]);
-    if (valid) {
-      const int pexp = pow2_exp_e4m3(amax);
-      const float sc = exp2_neg(pexp);
-      uint8_t* dst = p.hq + grow * p.N + (long)c.nt * 128 + half * 64;
+    const int pexp = pow2_exp_e4m3(amax);
+    const float sc = exp2_neg(pexp);
+    uint4 w[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_e4m3x4(h[v * 16 + 0] * sc, h[v * 16 + 1] * sc, h[v * 16 + 2] * sc, h[v * 16 + 3] * sc);
-        w.y = pack_e4m3x4(h[v * 16 + 4] * sc, h[v * 16 + 5] * sc, h[v * 16 + 6] * sc, h[v * 16 + 7] * sc);
-        w.z = pack_e4m3x4(h[v * 16 + 8] * sc, h[v * 16 + 9] * sc, h[v * 16 + 10] * sc, h[v * 16 + 11] * sc);
-        w.w = pack_e4m3x4(h[v * 16 + 12] * sc, h[v * 16 + 13] * sc, h[v * 16 + 14] * sc, h[v * 16 + 15] * sc);
-        *reinterpret_cast<uint4*>(dst + v * 16) = w;
-      }
+    for (int v = 0; v < 4; ++v) {
+      w[v].x = pack_e4m3x4(h[v * 16 + 0] * sc, h[v * 16 + 1] * sc, h[v * 16 + 2] * sc, h[v * 16 + 3] * sc);
+      w[v].y = pack_e4m3x4(h[v * 16 + 4] * sc, h[v * 16 + 5] * sc, h[v * 16 + 6] * sc, h[v * 16 + 7] * sc);
+      w[v].z = pack_e4m3x4(h[v * 16 + 8] * sc, h[v * 16 + 9] * sc, h[v * 16 + 10] * sc, h[v * 16 + 11] * sc);
+      w[v].w = pack_e4m3x4(h[v * 16 + 12] * sc, h[v * 16 + 13] * sc, h[v * 16 + 14] * sc, h[v * 16 + 15] * sc);
+    }
+    store_rows_64b(obuf, w, p.hq + (long)(c.row0 + q * 32) * p.N + (long)c.nt * 128 + half * 64, p.N, valid, lane);
+    if (valid) {
       if (half == 0) {
         // scale word of (row tile gmt, K-tile nt of linear2) in the tiled atom layout
         uint8_t* atom = reinterpret_cast<uint8_t*>(p.hsf) + ((long)c.gmt * (p.N / 128) + c.nt) * 512;
@@ -169,12 +191,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     __syncwarp();
     if (lane == 0) mbar_arrive(acce);
     const int col0 = c.nt * BN + half * 128;
-    if (valid && col0 < p.N) {
-      uint16_t* dst = p.y + grow * p.N + col0;
+    uint8_t* dst0 = reinterpret_cast<uint8_t*>(p.y + (long)(c.row0 + q * 32) * p.N + col0);
 #pragma unroll
-      for (int v = 0; v < 16; ++v) {
-        uint4 w = make_uint4(packed[v * 4 + 0], packed[v * 4 + 1], packed[v * 4 + 2], packed[v * 4 + 3]);
-        *reinterpret_cast<uint4*>(dst + v * 8) = w;
+    for (int ch = 0; ch < 4; ++ch) {
+      if (col0 + ch * 32 < p.N) {                      // warp-uniform column tail
+        uint4 w[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          w[v] = make_uint4(packed[ch * 16 + v * 4 + 0], packed[ch * 16 + v * 4 + 1], packed[ch * 16 + v * 4 + 2],
+                            packed[ch * 16 + v * 4 + 3]);
+        store_rows_64b(obuf, w, dst0 + ch * 64, (long)p.N * 2, valid, lane);
       }
     }
   }
@@ -316,6 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;      // which half of the accumulator columns
+    uint8_t* obuf = smem + SmemLayout::stage_out + (warp - 2) * 2048;
     uint32_t acc_phase = 0;
     int buf = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
@@ -324,7 +351,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool ok = mbar_wait(accf, acc_phase, ctl, kWhereGemmEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf);
+      epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf, obuf);
       acc_phase ^= 1;
       buf ^= 1;
     }
