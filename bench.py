@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch kernels one by one (no CUDA graph replay)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for ncu captures)")
     return ap.parse_args()
@@ -250,7 +251,8 @@ def run_cuda(args, rank, world, local_rank):
     W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device=dev)
     d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
     plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared, device=dev)
-    plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 1)
+    # launch the forward's kernels as one recorded CUDA graph (per pointer set)
+    plan.set_option(binding.MOE_OPT_GRAPH, 0 if args.no_graph else 1)
     out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -277,7 +279,7 @@ def run_cuda(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    step_ms, phases = [], []
+    step_ms = []
     for _ in range(args.steps):
         flush.fill_(1)                                   # L2 scrub between timed steps (not timed)
         ev0 = torch.cuda.Event(enable_timing=True)
@@ -287,7 +289,6 @@ def run_cuda(args, rank, world, local_rank):
         ev1.record(stream)
         ev1.synchronize()
         step_ms.append(ev0.elapsed_time(ev1))
-        phases.append(plan.phase_times())
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -299,6 +300,17 @@ def run_cuda(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.all_reduce(total_ms, op=torch.distributed.ReduceOp.MAX)
     total_ms = float(total_ms.item())
+
+    # Per-kernel times for the roofline: CUDA events recorded on the forward's stream
+    # between its kernels (graph replay is off while the events are on).
+    plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 1)
+    phases = []
+    for _ in range(min(args.steps, 20)):
+        flush.fill_(1)
+        plan.forward(**d, out=out)
+        phases.append(plan.phase_times())
+    plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 0)
+    plan.set_option(binding.MOE_OPT_GRAPH, 0 if args.no_graph else 1)
 
     # end to end through the public API: pinned host x -> device, forward, out -> pinned host
     # Every step copies its tokens host -> device, runs the layer and copies the
@@ -410,6 +422,9 @@ def run_cuda(args, rank, world, local_rank):
         "config": {"workload": w.description + ("" if args.tokens is None else f" (T overridden to {w.T})"),
                    "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
                    "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+                   "launch": "kernels launched one by one" if args.no_graph else
+                             "CUDA graph replay of the 7 kernels (MOE_OPT_GRAPH)",
+                   "phase_times": "separate pass, CUDA events between kernels, 20 steps",
                    "weight_scales": f"re-laid out once before timing ({prepare_ms:.3f} ms), reused "
                                     "(MOE_OPT_STATIC_WEIGHTS)",
                    "parallelism": f"replicas x{world} (token-sharded, no collective)"},

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "../../include/moe_b200.h"
 #include "kernels.h"
@@ -44,6 +45,14 @@ struct moe_plan_s {
   const void* w2_cached = nullptr;
   const void* w1s_prepared = nullptr;   // weight scales the prepared units were built from
   const void* w2s_prepared = nullptr;
+  // MOE_OPT_GRAPH: recorded launch sequences, keyed by the forward's pointers
+  int use_graph = 0;
+  struct GraphEntry {
+    const void* key[8];
+    cudaGraphExec_t exec;
+  };
+  std::vector<GraphEntry> graphs;
+  cudaStream_t cap_stream = nullptr;
   // per-phase timing (MOE_OPT_PHASE_EVENTS)
   int phase_events = 0;
   bool events_ready = false;
@@ -211,6 +220,67 @@ int prepare_weights(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_sc
   return MOE_OK;
 }
 
+// The forward's launch sequence on stream s (TMA maps already current).
+int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias,
+                   const uint8_t* W1_scales, const uint8_t* W2_scales, void* out, cudaStream_t s) {
+  int rc = run_front(p, x, W_router, bias, s);
+  if (rc != MOE_OK) return rc;
+  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
+    if ((rc = prepare_weights(p, W1_scales, W2_scales, s)) != MOE_OK) return rc;
+  }
+  mark(p, 1 + MOE_PHASE_PREPARE, s);
+  GemmArgs a1 = gemm_args(p, 1);
+  if (launch_gemm_linear1(p->tmA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(p, 1 + MOE_PHASE_LINEAR1, s);
+  GemmArgs a2 = gemm_args(p, 2);
+  if (launch_gemm_linear2(p->tmA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(p, 1 + MOE_PHASE_LINEAR2, s);
+  cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
+                                 region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
+                                 p->shared, s);
+  mark(p, 1 + MOE_PHASE_COMBINE, s);
+  if (p->phase_events && p->events_ready) p->events_recorded = true;
+  return cuda_rc(e);
+}
+
+void drop_graphs(moe_plan_t p) {
+  for (auto& g : p->graphs) cudaGraphExecDestroy(g.exec);
+  p->graphs.clear();
+}
+
+// MOE_OPT_GRAPH: replay the launch sequence recorded for this exact argument set,
+// recording it (on a private stream) the first time.
+int forward_graph(moe_plan_t p, const void* x, const float* W_router, const float* bias, const uint8_t* W1,
+                  const uint8_t* W1_scales, const uint8_t* W2, const uint8_t* W2_scales, void* out, cudaStream_t s) {
+  const void* key[8] = {x, W_router, bias, W1, W1_scales, W2, W2_scales, out};
+  for (auto& g : p->graphs)
+    if (std::memcmp(g.key, key, sizeof(key)) == 0) return cuda_rc(cudaGraphLaunch(g.exec, s));
+  if (!p->cap_stream && cudaStreamCreateWithFlags(&p->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamBeginCapture(p->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ERR_CUDA;
+  int rc = launch_forward(p, static_cast<const uint16_t*>(x), W_router, bias, W1_scales, W2_scales, out,
+                          p->cap_stream);
+  cudaGraph_t graph = nullptr;
+  cudaError_t e = cudaStreamEndCapture(p->cap_stream, &graph);
+  if (rc != MOE_OK || e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return rc != MOE_OK ? rc : MOE_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (p->graphs.size() >= 4) {
+    cudaGraphExecDestroy(p->graphs.front().exec);
+    p->graphs.erase(p->graphs.begin());
+  }
+  moe_plan_s::GraphEntry ge;
+  std::memcpy(ge.key, key, sizeof(key));
+  ge.exec = exec;
+  p->graphs.push_back(ge);
+  return cuda_rc(cudaGraphLaunch(exec, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -278,7 +348,12 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
 
 int moe_plan_set_option(moe_plan_t p, int key, long long value) {
   if (!p) return MOE_ERR_INVALID_ARG;
+  drop_graphs(p);                       // recorded sequences depend on the options
   switch (key) {
+    case MOE_OPT_GRAPH:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->use_graph = (int)value;
+      return MOE_OK;
     case MOE_OPT_MAX_SMS:
       if (value < 0) return MOE_ERR_INVALID_ARG;
       p->max_sms = (int)value;
@@ -329,6 +404,7 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED_SHAPE;   // built for sm_100a only
   if (gemm_prepare_device() != cudaSuccess) return MOE_ERR_CUDA;
+  drop_graphs(p);
   p->ws = static_cast<uint8_t*>(ws);
   p->ws_bytes = bytes;
   p->device = dev;
@@ -380,24 +456,13 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
       if (cudaEventCreate(&p->ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
     p->events_ready = true;
   }
-  const uint16_t* xb = static_cast<const uint16_t*>(x);
-  if ((rc = run_front(p, xb, W_router, bias, s)) != MOE_OK) return rc;
-  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
-    if ((rc = prepare_weights(p, W1_scales, W2_scales, s)) != MOE_OK) return rc;
+  if (p->use_graph && !p->phase_events) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (st == cudaStreamCaptureStatusNone) return forward_graph(p, x, W_router, bias, W1, W1_scales, W2, W2_scales,
+                                                                out, s);
   }
-  mark(p, 1 + MOE_PHASE_PREPARE, s);
-  GemmArgs a1 = gemm_args(p, 1);
-  if (launch_gemm_linear1(p->tmA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
-  mark(p, 1 + MOE_PHASE_LINEAR1, s);
-  GemmArgs a2 = gemm_args(p, 2);
-  if (launch_gemm_linear2(p->tmA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
-  mark(p, 1 + MOE_PHASE_LINEAR2, s);
-  cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
-                                 region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
-                                 p->shared, s);
-  mark(p, 1 + MOE_PHASE_COMBINE, s);
-  if (p->phase_events && p->events_ready) p->events_recorded = true;
-  return cuda_rc(e);
+  return launch_forward(p, static_cast<const uint16_t*>(x), W_router, bias, W1_scales, W2_scales, out, s);
 }
 
 int moe_phase_times(moe_plan_t p, float* ms, int capacity) {
@@ -467,6 +532,8 @@ int moe_check_status(moe_plan_t p, void* stream, uint32_t* detail) {
 
 void moe_plan_destroy(moe_plan_t p) {
   if (!p) return;
+  drop_graphs(p);
+  if (p->cap_stream) cudaStreamDestroy(p->cap_stream);
   if (p->events_ready)
     for (int i = 0; i <= MOE_PHASE_COUNT_; ++i) cudaEventDestroy(p->ev[i]);
   delete p;

@@ -345,9 +345,13 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
                                                             const int32_t* __restrict__ mtile_start,
                                                             int32_t* slot_pos, int32_t* perm, uint8_t* xq,
                                                             uint8_t* xsf, int T, int H, int E, int k, int shared) {
+  // one warp per (token, 256-channel slice); the slice-0 warp also records the positions
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
+  const int n_slices = (x == nullptr) ? 1 : (H + 255) / 256;
+  const long item = (long)blockIdx.x * 8 + warp;
+  if (item >= (long)T * n_slices) return;
+  const int t = (int)(item / n_slices);
+  const int slice = (int)(item % n_slices);
   const int g = t / 32;
   const long R = (long)T * k;
   const int kw = H / 128;
@@ -356,8 +360,10 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
   if (lane < k) {
     e = topk_ids[(long)t * k + lane];
     row = group_base[(long)g * E + e] + local_rank[(long)t * k + lane];
-    slot_pos[(long)t * k + lane] = row;
-    perm[row] = t * k + lane;
+    if (slice == 0) {
+      slot_pos[(long)t * k + lane] = row;
+      perm[row] = t * k + lane;
+    }
   } else if (lane == k && shared) {
     e = E;
     row = (int)(R + t);
@@ -372,10 +378,10 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
   }
   const int ndst = k + shared;
   const uint16_t* xr = x + (long)t * H;
-  for (int cb = 0; cb < H; cb += 256) {
+  {
     // 8 channels per lane; a 128-channel block spans 16 lanes.  Every lane runs
-    // every iteration (shuffles use the full mask); a half-warp past H idles.
-    const int c0 = cb + lane * 8;
+    // the shuffles (full mask); a half-warp past H idles.
+    const int c0 = slice * 256 + lane * 8;
     const bool active = c0 < H;           // H % 128 == 0: whole half-warps
     const uint4 raw = active ? *reinterpret_cast<const uint4*>(xr + c0) : make_uint4(0, 0, 0, 0);
     float v[8];
@@ -446,9 +452,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                                                       const int32_t* __restrict__ slot_pos,
                                                       const float* __restrict__ gates, uint16_t* __restrict__ out,
                                                       int T, int H, int k, int shared) {
+  // one warp per (token, 256-channel slice)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
+  const int n_slices = (H + 255) / 256;
+  const long item = (long)blockIdx.x * 8 + warp;
+  if (item >= (long)T * n_slices) return;
+  const int t = (int)(item / n_slices);
+  const int slice = (int)(item % n_slices);
   const long R = (long)T * k;
   int my_row = 0;
   float my_gate = 0.f;
@@ -456,8 +466,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     my_row = slot_pos[(long)t * k + lane];
     my_gate = gates[(long)t * k + lane];
   }
-  for (int cb = 0; cb < H; cb += 256) {
-    const int c0 = cb + lane * 8;
+  {
+    const int c0 = slice * 256 + lane * 8;
     const bool active = c0 < H;
     float acc[8];
 #pragma unroll
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         acc[2 * i + 1] = fmaf(gj, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
       }
     }
-    if (!active) continue;
+    if (!active) return;                 // no shuffles below
     if (shared) {
       const uint4 raw = *reinterpret_cast<const uint4*>(y + (R + t) * H + c0);
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -553,7 +563,9 @@ cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, con
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
                                  int k, int shared, cudaStream_t s) {
-  scatter_quant_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, topk_ids, local_rank, group_base, offsets, mtile_start,
+  const long items = (long)T * (x == nullptr ? 1 : (H + 255) / 256);
+  scatter_quant_kernel<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(x, topk_ids, local_rank, group_base, offsets,
+                                                                   mtile_start,
                                                    slot_pos, perm, xq, xsf, T, H, E, k, shared);
   return cudaGetLastError();
 }
@@ -565,7 +577,8 @@ cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T
 
 cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,
                            int H, int k, int shared, cudaStream_t s) {
-  combine_kernel<<<(T + 7) / 8, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  const long items = (long)T * ((H + 255) / 256);
+  combine_kernel<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
   return cudaGetLastError();
 }
 

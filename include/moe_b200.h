@@ -78,12 +78,19 @@ enum moe_option {
                                   2^-18 |W|) accumulated in fp32; 0: fp32 FMA on CUDA cores */
   MOE_OPT_PHASE_EVENTS = 5,    /* 1 = record a CUDA event after each kernel of moe_forward
                                   on its stream, read back with moe_phase_times()        */
-  MOE_OPT_STATIC_WEIGHTS = 6   /* 1 = the caller promises that W_router / W1_scales /
+  MOE_OPT_STATIC_WEIGHTS = 6,  /* 1 = the caller promises that W_router / W1_scales /
                                   W2_scales do not change between calls that pass the same
                                   pointers: moe_forward then reuses the tiled scale units
                                   and the split router weights built by the last
                                   moe_prepare_weights (or forward) from those pointers.
                                   0 (default): every forward rebuilds them.              */
+  MOE_OPT_GRAPH = 7            /* 1 = moe_forward records its launch sequence as a CUDA
+                                  graph the first time it sees a set of argument pointers
+                                  (up to 4 sets per plan) and replays it on later calls,
+                                  removing per-kernel launch overhead.  Not used while the
+                                  caller's stream is capturing or MOE_OPT_PHASE_EVENTS is
+                                  1.  The CUDA runtime may reserve memory for the recorded
+                                  graphs; changing any option drops them.  Default 0.    */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -261,6 +261,27 @@ def test_static_weights_reuse_prepared_scales(cuda_lib):
     assert torch.equal(c, b)
 
 
+def test_graph_replay_matches_direct_launches(cuda_lib):
+    w = SMALL["dsv3_like"]
+    d = to_device(make_case(w, seed=13, screened=False))
+    p = plan_for(w)
+    ref = p.forward(**d).clone()
+    p.set_option(binding.MOE_OPT_GRAPH, 1)
+    out = torch.empty_like(ref)
+    for _ in range(3):                                  # record, then replay
+        out.zero_()
+        p.forward(**d, out=out)
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # a replay reads the current contents of the same buffers
+    x2 = make_case(w, seed=14, screened=False)["x"].cuda()
+    d["x"].copy_(x2)
+    p.forward(**d, out=out)
+    p.set_option(binding.MOE_OPT_GRAPH, 0)
+    ref2 = p.forward(**d).clone()
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+    assert p.check_status()[0] == 0
+
+
 # --------------------------------------------------------------------------- failure detection
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
