@@ -208,7 +208,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
 
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles
@@ -242,7 +242,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&tmA.m[i]);
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
@@ -272,13 +273,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const TileCoord c = decode_tile(p, tile);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
+        const int rows_here = min(BM, c.count - c.mt * BM);
+        const int a_sel = rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
+        const uint32_t a_box = 16u << a_sel;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
           if (withhold) {
             withhold = false;            // test hook: this stage never fills
           } else {
-            mbar_arrive_expect_tx(&full[stage], kStageTxBytes);
-            tma_load_2d(a_s + stage * kATileBytes, &tmA, kt * BK, c.row0, &full[stage]);
+            // A rows of this tile that belong to the expert decide the box height; the MMA
+            // still reads 128 rows, the rest are leftovers whose accumulator rows are dropped
+            mbar_arrive_expect_tx(&full[stage], kStageTxBytes - kATileBytes + a_box * BK);
+            tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
             if constexpr (MODE == 1) {
               const int brow = c.e * p.rows_b + c.nt * 128;
               tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full[stage]);
@@ -589,13 +595,13 @@ cudaError_t gemm_prepare_device() {
                               (int)gemm_smem_bytes());
 }
 
-cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s) {
   grouped_gemm_kernel<1><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s) {
   grouped_gemm_kernel<2><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
   return cudaGetLastError();

@@ -45,9 +45,14 @@ cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attribut
 // canonical UE8M0 weight scales [n][rows_b][K/32] -> weight scale units
 cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
                                       int n_tiles_n, int mode, int N, cudaStream_t s);
-cudaError_t launch_gemm_linear1(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+// A-operand tensor maps of one activation matrix with box heights 16, 32, 64, 128 rows
+// (the producer picks the smallest box that covers the tile's rows of its expert).
+struct AMaps {
+  CUtensorMap m[4];
+};
+cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s);
-cudaError_t launch_gemm_linear2(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int grid,
+cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s);
 
 // ---- router on tensor cores (gemm_sm100.cu) -------------------------------------

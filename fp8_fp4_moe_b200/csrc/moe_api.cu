@@ -38,7 +38,8 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   int device = -1;
   int num_sms = 0;
-  alignas(64) CUtensorMap tmA1, tmA2, tmB1, tmB2, tmX, tmWhi, tmWlo;
+  alignas(64) AMaps amA1, amA2;
+  alignas(64) CUtensorMap tmB1, tmB2, tmX, tmWhi, tmWlo;
   const void* x_cached = nullptr;        // tmX encodes this x pointer
   const void* wr_prepared = nullptr;     // W_router the hi/lo split was made from
   const void* w1_cached = nullptr;
@@ -230,10 +231,10 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
   }
   mark(p, 1 + MOE_PHASE_PREPARE, s);
   GemmArgs a1 = gemm_args(p, 1);
-  if (launch_gemm_linear1(p->tmA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(p, 1 + MOE_PHASE_LINEAR1, s);
   GemmArgs a2 = gemm_args(p, 2);
-  if (launch_gemm_linear2(p->tmA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(p, 1 + MOE_PHASE_LINEAR2, s);
   cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
                                  region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
@@ -412,11 +413,14 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   p->w1_cached = p->w2_cached = nullptr;
   p->w1s_prepared = p->w2s_prepared = nullptr;
   p->x_cached = p->wr_prepared = nullptr;
-  int rc = encode_2d(&p->tmA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_XQ), p->H, p->rows,
-                     p->H, 128, 128);
-  if (rc == MOE_OK)
-    rc = encode_2d(&p->tmA2, CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_HQ), p->I, p->rows,
-                   p->I, 128, 128);
+  int rc = MOE_OK;
+  for (int i = 0; i < 4 && rc == MOE_OK; ++i) {
+    rc = encode_2d(&p->amA1.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_XQ), p->H, p->rows,
+                   p->H, 128, 16u << i);
+    if (rc == MOE_OK)
+      rc = encode_2d(&p->amA2.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, region<uint8_t>(p, MOE_REGION_HQ), p->I,
+                     p->rows, p->I, 128, 16u << i);
+  }
   if (rc == MOE_OK)
     rc = encode_2d(&p->tmWhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, at<uint16_t>(p, p->off_whi), p->H, p->E,
                    2ull * p->H, 64, 128);

@@ -207,15 +207,35 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
       float chosen_score = 0.f;   // unbiased score of this lane's slot (lane < k)
       int chosen_id = -1;
       uint32_t taken = 0u;        // bit i: expert lane + 32*i already selected (E <= 1024)
+      float cached[8];            // E <= 256: this lane's biased scores, read once
+      const bool use_cache = E <= 256;
+      if (use_cache) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = lane + 32 * i;
+          cached[i] = (e < E) ? row[e] + bias[e] : 0.f;
+        }
+      }
       for (int j = 0; j < k; ++j) {
         float best = -INFINITY;
         int best_id = 0x7FFFFFFF;
         int free_id = 0x7FFFFFFF;   // lowest unselected id (fallback when every score is NaN)
-        for (int i = 0, e = lane; e < E; ++i, e += 32) {
-          if (taken & (1u << i)) continue;
-          if (free_id == 0x7FFFFFFF) free_id = e;
-          const float b = row[e] + bias[e];
-          if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
+        if (use_cache) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (e >= E || (taken & (1u << i))) continue;
+            if (free_id == 0x7FFFFFFF) free_id = e;
+            const float b = cached[i];
+            if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
+          }
+        } else {
+          for (int i = 0, e = lane; e < E; ++i, e += 32) {
+            if (taken & (1u << i)) continue;
+            if (free_id == 0x7FFFFFFF) free_id = e;
+            const float b = row[e] + bias[e];
+            if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
+          }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -526,13 +546,14 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
     if (grid > 148) grid = 148;
     router_logits_smem_kernel<<<grid, 256, (size_t)E * H * 4, s>>>(x, W_r, logits, T, H, E);
   } else if (E <= 32 || (long)T * E <= 16384) {
-    // warp per (token, expert chunk); chunks of 2 when few tokens must cover many experts
-    const int ec = (E <= 32) ? 8 : 2;
+    // warp per (token, expert chunk); one expert per warp when few tokens must cover many experts
+    const int ec = (E <= 32) ? 8 : ((long)T * E <= 4096 ? 1 : 2);
     const long items = (long)T * ((E + ec - 1) / ec);
     const long blocks = (items + 7) / 8;
     const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
     if (ec == 8) router_logits_warp_kernel<8><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
-    else router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+    else if (ec == 2) router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+    else router_logits_warp_kernel<1><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
   } else if (E <= 16) {
     dim3 grid((T + 63) / 64, (E + 15) / 16);
     router_logits_kernel<16><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
