@@ -53,13 +53,19 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch kernels one by one (no CUDA graph replay)")
+    ap.add_argument("--opt", action="append", default=[], metavar="NAME=VALUE",
+                    help="plan option, e.g. SWAP_ROWS=0 or PREFETCH=4 (MOE_OPT_<NAME>); repeatable")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for ncu captures)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (with --tokens: a decode-shaped case with fewer experts in HBM)")
     return ap.parse_args()
 
 
 def workload(args) -> I.Workload:
     w = I.WORKLOADS[args.workload]
+    if args.experts is not None:
+        w = w.with_experts(args.experts)
     return w if args.tokens is None else w.with_tokens(args.tokens)
 
 
@@ -249,10 +255,14 @@ def run_cuda(args, rank, world, local_rank):
     _, W_r, bias = I.make_routing_inputs(w, 0)
     x, _, _ = I.make_routing_inputs(w, 1000 + rank) if rank > 0 else I.make_routing_inputs(w, 0)
     W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device=dev)
+    torch.cuda.empty_cache()        # return the quantiser's temporaries: only live tensors stay on the device
     d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
     plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared, device=dev)
     # launch the forward's kernels as one recorded CUDA graph (per pointer set)
     plan.set_option(binding.MOE_OPT_GRAPH, 0 if args.no_graph else 1)
+    for kv in args.opt:
+        name, value = kv.split("=", 1)
+        plan.set_option(getattr(binding, "MOE_OPT_" + name.upper()), int(value))
     out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -399,7 +409,8 @@ def run_cuda(args, rank, world, local_rank):
     roof["kernel"] = dominant
     roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json: 2 x {bf16_key} (FP8 = 2 x BF16 dense)"
                            if roof["unit"] == "TFLOP/s" else f"{peak_src} MEASURED_PEAKS.json hbm_gbs")
-    roof["traffic"] = ncu_traffic(dominant, args.workload) if args.tokens is None else None
+    resized = args.tokens is not None or args.experts is not None
+    roof["traffic"] = ncu_traffic(dominant, args.workload) if not resized else None
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -419,7 +430,7 @@ def run_cuda(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8e4m3 x fp4e2m1 (fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": w.description + ("" if args.tokens is None else f" (T overridden to {w.T})"),
+        "config": {"workload": w.description + ("" if not resized else f" (resized to T={w.T}, E={w.E})"),
                    "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
                    "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
                    "launch": "kernels launched one by one" if args.no_graph else
@@ -427,7 +438,8 @@ def run_cuda(args, rank, world, local_rank):
                    "phase_times": "separate pass, CUDA events between kernels, 20 steps",
                    "weight_scales": f"re-laid out once before timing ({prepare_ms:.3f} ms), reused "
                                     "(MOE_OPT_STATIC_WEIGHTS)",
-                   "parallelism": f"replicas x{world} (token-sharded, no collective)"},
+                   "parallelism": f"replicas x{world} (token-sharded, no collective)",
+                   "options": args.opt},
         "tflops": w.flops() / (ms * 1e-3) / 1e12,
         "tflops_frac_fp8": w.flops() / (ms * 1e-3) / 1e12 / fp8_sustained,
         "fp8_peak_tflops": fp8_sustained,

@@ -117,6 +117,15 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Bring a tensor-map box / a contiguous range into L2 without waiting for it.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* gmem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -192,6 +201,15 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "r"(taddr)
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading/stride
@@ -211,10 +229,13 @@ constexpr uint32_t kLayoutSwizzle128B = 2;
 
 // Instruction descriptor for kind::mxf8f6f4 block-scaled MMA, A = E4M3,
 // B = E2M1, both K-major, UE8M0 scales, fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+// Operand format codes of kind::mxf8f6f4.
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id,
+                                                     uint32_t a_fmt = kFmtE4M3, uint32_t b_fmt = kFmtE2M1) {
   return (b_sf_id & 3u) << 4          // B scale-factor byte
-         | (0u << 7)                  // A format: E4M3
-         | (5u << 10)                 // B format: E2M1
+         | (a_fmt << 7)               // A format
+         | (b_fmt << 10)              // B format
          | ((uint32_t)(N >> 3) << 17) // N / 8
          | (1u << 23)                 // scale format: UE8M0
          | ((uint32_t)(M >> 4) << 24) // M / 16

@@ -57,14 +57,15 @@ struct SmemLayout {
   static constexpr uint32_t amax = sfb + S * kSfbBytes;           // [2 buffers][2 halves][128 rows] fp32
   static constexpr uint32_t stage_out = amax + 2 * 2 * 128 * 4;   // [8 epilogue warps][32 rows][64 B]
   static constexpr uint32_t bars = stage_out + 8 * 2048;
-  // full[S], empty[S], accf, acce, drain
-  static constexpr uint32_t n_bars = 2 * S + 3;
+  // full[S], empty[S], accf[2], acce[2], drain
+  static constexpr uint32_t n_bars = 2 * S + 5;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t total = misc + 16;
 };
 
 struct TileCoord {
   int e, mt, nt, count, row0, gmt;   // gmt = global row-tile index
+  int rows;                          // rows of the expert in this tile (1..128)
 };
 
 __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
@@ -84,7 +85,33 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
   c.mt = local - c.nt * mtiles;
   c.row0 = __ldg(p.offsets + lo) + c.mt * BM;
   c.gmt = mstart + c.mt;
+  c.rows = min(BM, c.count - c.mt * BM);
   return c;
+}
+
+// Accumulator slots: TMEM columns [0, 128) and [128, 256).  A tile with at most
+// swap_rows rows of its expert is computed transposed (weights as the M = 128
+// operand, the tile's tokens as N = 32 or 64) into one slot, alternating between
+// the two; any other tile takes both slots (M = 128 tokens, N = 256).  The MMA
+// issuer and the epilogue walk the same tile sequence and keep one use counter
+// per slot, so both derive the same mbarrier parities.
+struct SlotPlan {
+  bool swap;
+  int lo, hi;        // slots [lo, hi] this tile uses
+  int nt_tok;        // swapped tiles: token columns (MMA N)
+};
+__device__ __forceinline__ SlotPlan plan_slots(const GemmArgs& p, const TileCoord& c, int& next_slot) {
+  SlotPlan s;
+  s.swap = c.rows <= p.swap_rows;
+  s.nt_tok = c.rows <= 32 ? 32 : 64;
+  if (s.swap) {
+    s.lo = s.hi = next_slot;
+    next_slot ^= 1;
+  } else {
+    s.lo = 0;
+    s.hi = 1;
+  }
+  return s;
 }
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -140,7 +167,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(acce);                  // accumulator may be overwritten now
+    if (lane == 0) {                                   // accumulator may be overwritten now
+      mbar_arrive(&acce[0]);
+      mbar_arrive(&acce[1]);
+    }
     float h[64];
     float amax = 0.f;
 #pragma unroll
@@ -189,7 +219,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(acce);
+    if (lane == 0) {
+      mbar_arrive(&acce[0]);
+      mbar_arrive(&acce[1]);
+    }
     const int col0 = c.nt * BN + half * 128;
     uint8_t* dst0 = reinterpret_cast<uint8_t*>(p.y + (long)(c.row0 + q * 32) * p.N + col0);
 #pragma unroll
@@ -202,6 +235,98 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
                             packed[ch * 16 + v * 4 + 3]);
         store_rows_64b(obuf, w, dst0 + ch * 64, (long)p.N * 2, valid, lane);
       }
+    }
+  }
+}
+
+// Lane l ends with the maximum over the warp's 32 lanes of a[l % TW] (TW = 16 or 32):
+// each step keeps half of the values and folds in the partner's copy of the other half.
+template <int TW>
+__device__ __forceinline__ float warp_transpose_max(float (&a)[TW], int lane) {
+  if constexpr (TW == 16) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = fmaxf(a[i], __shfl_xor_sync(0xffffffffu, a[i], 16));
+  }
+#pragma unroll
+  for (int s = TW / 2; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? a[i] : a[i + s];
+      const float keep = upper ? a[i + s] : a[i];
+      a[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, s));
+    }
+  }
+  return a[0];
+}
+
+// Epilogue of a transposed tile: TMEM lane = weight row (channel), column = token.
+//   linear1: gate accumulator in slot columns [0, NT), up in [64, 64 + NT); warp (q, half)
+//            owns channels q*32 + lane of the tile's 128 and tokens [half*NT/2, half*NT/2 + NT/2);
+//            the per-token amax over the 128 channels goes through shared memory.
+//   linear2: rows 0..127 of the 256-row weight tile in slot columns [0, NT), rows 128..255 in
+//            [64, 64 + NT); warp (q, half) owns output channels half*128 + q*32 + lane, all tokens.
+// Per token, a warp's 32 channels are consecutive in the output row: one store instruction
+// covers 32 bytes (linear1) or 64 bytes (linear2).
+template <int MODE, int NT>
+__device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord& c, uint32_t acc, int q, int half,
+                                              int lane, uint64_t* acce_slot, float* amax_s, int buf) {
+  const uint32_t t_lane = acc + ((uint32_t)(q * 32) << 16);
+  if constexpr (MODE == 1) {
+    constexpr int TW = NT / 2;
+    uint32_t g[TW], u[TW];
+    if constexpr (TW == 16) {
+      tmem_ld_32x32b_x16(t_lane + half * TW, g);
+      tmem_ld_32x32b_x16(t_lane + 64 + half * TW, u);
+    } else {
+      tmem_ld_32x32b_x32(t_lane + half * TW, g);
+      tmem_ld_32x32b_x32(t_lane + 64 + half * TW, u);
+    }
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_slot);
+    float h[TW], a[TW];
+#pragma unroll
+    for (int j = 0; j < TW; ++j) {
+      const float gv = __uint_as_float(g[j]);
+      h[j] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[j]);   // silu(gate) * up
+      a[j] = fabsf(h[j]);
+    }
+    const int tl = lane % TW;                    // this lane's token within the warp's range
+    const int tok = half * TW + tl;              // token row within the tile
+    float* slot = amax_s + buf * 256;            // [quarter][64 tokens]
+    const float am_q = warp_transpose_max<TW>(a, lane);
+    if (lane < TW) slot[q * 64 + tok] = am_q;
+    epi_bar();
+    const float am = fmaxf(fmaxf(slot[tok], slot[64 + tok]), fmaxf(slot[128 + tok], slot[192 + tok]));
+    const int pexp = pow2_exp_e4m3(am);
+    const float sc = exp2_neg(pexp);
+    if (q == 0 && lane < TW && tok < c.rows) {
+      uint8_t* atom = reinterpret_cast<uint8_t*>(p.hsf) + ((long)c.gmt * (p.N / 128) + c.nt) * 512;
+      *reinterpret_cast<uint32_t*>(atom + (tok % 32) * 16 + (tok / 32) * 4) = (uint32_t)(pexp + 127) * 0x01010101u;
+    }
+    uint8_t* dst = p.hq + (long)(c.row0 + half * TW) * p.N + (long)c.nt * 128 + q * 32 + lane;
+#pragma unroll
+    for (int j = 0; j < TW; ++j) {
+      const float sj = __shfl_sync(0xffffffffu, sc, j);
+      const uint8_t b = (uint8_t)(cvt_e4m3x2(h[j] * sj, 0.f) & 0xFF);
+      if (half * TW + j < c.rows) dst[(long)j * p.N] = b;
+    }
+  } else {
+    uint32_t r[NT];
+    tmem_ld_32x32b_x32(t_lane + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    if constexpr (NT == 64) tmem_ld_32x32b_x32(t_lane + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acce_slot);
+    const int col = c.nt * BN + half * 128 + q * 32 + lane;
+    if (col < p.N) {
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (long)c.row0 * p.N + col;
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+        if (j < c.rows) dst[(long)j * p.N] = __float2bfloat16_rn(__uint_as_float(r[j]));
     }
   }
 }
@@ -221,9 +346,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
-  uint64_t* accf = bars + 2 * S;
-  uint64_t* acce = accf + 1;
-  uint64_t* drain = accf + 2;
+  uint64_t* accf = bars + 2 * S;      // [2] accumulator slot full
+  uint64_t* acce = accf + 2;          // [2] accumulator slot empty
+  uint64_t* drain = accf + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 4);
 
@@ -235,8 +360,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accf, 1);
-    mbar_init(acce, kEpiWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], kEpiWarps);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -269,6 +396,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       bool withhold = p.inject_fault != 0 && blockIdx.x == 0;
+      // L2 prefetch cursor: walks this CTA's (tile, K stage) sequence p.prefetch stages ahead of
+      // the loads, so weight tiles stream from HBM into L2 while the shared-memory ring is full
+      int pf_tile = blockIdx.x, pf_kt = 0;
+      TileCoord pc{};
+      if (pf_tile < total_tiles) pc = decode_tile(p, pf_tile);
+      auto prefetch_next = [&]() {
+        if (pf_tile >= total_tiles) return;
+        if constexpr (MODE == 1) {
+          const int brow = pc.e * p.rows_b + pc.nt * 128;
+          tma_prefetch_l2_2d(&tmB, pf_kt * BK, brow);
+          tma_prefetch_l2_2d(&tmB, pf_kt * BK, brow + p.N);
+        } else {
+          tma_prefetch_l2_2d(&tmB, pf_kt * BK, pc.e * p.rows_b + pc.nt * BN);
+        }
+        bulk_prefetch_l2(p.sfb + (((long)pc.e * p.n_tiles_n + pc.nt) * KT + pf_kt) * kSfbBytes, kSfbBytes);
+        if (++pf_kt == KT) {
+          pf_kt = 0;
+          pf_tile += gridDim.x;
+          if (pf_tile < total_tiles) pc = decode_tile(p, pf_tile);
+        }
+      };
+      for (int i = 0; i < p.prefetch; ++i) prefetch_next();
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const TileCoord c = decode_tile(p, tile);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
@@ -297,6 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bulk_load(sfb_s + stage * kSfbBytes, sfb_tile + kt * kSfbBytes, kSfbBytes, &full[stage]);
             fills[stage] += 1;
           }
+          if (p.prefetch > 0) prefetch_next();
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -312,11 +462,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0;
+      uint32_t uses0 = 0, uses1 = 0;      // completed uses of each accumulator slot
+      int next_slot = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(acce, acc_phase ^ 1, ctl, kWhereGemmMma)) break;
+        const TileCoord c = decode_tile(p, tile);
+        const SlotPlan sp = plan_slots(p, c, next_slot);
+        for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
+          ok = mbar_wait(&acce[sl], ((sl ? uses1 : uses0) & 1) ^ 1, ctl, kWhereGemmMma);
+        if (!ok) break;
         tc_fence_after();
+        const uint32_t acc = tmem_base + kAccCol + sp.lo * 128;
+        const uint32_t id_swap0 = idesc_mxf8f6f4(BM, sp.nt_tok, 0, 0, kFmtE2M1, kFmtE4M3);
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&full[stage], phase, ctl, kWhereGemmMma + 1)) { ok = false; break; }
           tc_fence_after();
@@ -327,18 +485,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_cp_32x128b_warpx4(tmem_base + kSfbCol + 4, sf_desc(sfb_addr + 512));
           const uint32_t a_addr = smem_u32(a_s + stage * kATileBytes);
           const uint32_t b_addr = smem_u32(b_s + stage * kBTileBytes);
+          if (sp.swap) {
+            // weights (E2M1, rows 0..127 and 128..255 of the B stage) as A, tokens (E4M3) as B;
+            // the weight scale atoms are the A scales, the token atom the B scales
 #pragma unroll
-          for (int kb = 0; kb < BK / 32; ++kb) {
-            tc_mma_mxf8f6f4(tmem_base + kAccCol, sw128_desc(a_addr + kb * 32), sw128_desc(b_addr + kb * 32),
-                            idesc_mxf8f6f4(BM, BN, kb, kb), tmem_base + kSfaCol, tmem_base + kSfbCol,
-                            (kt | kb) != 0);
+            for (int kb = 0; kb < BK / 32; ++kb) {
+              const uint32_t id = id_swap0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
+              tc_mma_mxf8f6f4(acc, sw128_desc(b_addr + kb * 32), sw128_desc(a_addr + kb * 32), id,
+                              tmem_base + kSfbCol, tmem_base + kSfaCol, (kt | kb) != 0);
+              tc_mma_mxf8f6f4(acc + 64, sw128_desc(b_addr + kBTileBytes / 2 + kb * 32),
+                              sw128_desc(a_addr + kb * 32), id, tmem_base + kSfbCol + 4, tmem_base + kSfaCol,
+                              (kt | kb) != 0);
+            }
+          } else {
+#pragma unroll
+            for (int kb = 0; kb < BK / 32; ++kb) {
+              tc_mma_mxf8f6f4(acc, sw128_desc(a_addr + kb * 32), sw128_desc(b_addr + kb * 32),
+                              idesc_mxf8f6f4(BM, BN, kb, kb), tmem_base + kSfaCol, tmem_base + kSfbCol,
+                              (kt | kb) != 0);
+            }
           }
           tc_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(accf);
-        acc_phase ^= 1;
+        for (int sl = sp.lo; sl <= sp.hi; ++sl) tc_commit(&accf[sl]);
+        uses0 += sp.lo == 0;
+        uses1 += sp.hi == 1;
       }
       // all MMAs this thread issued have finished once `drain` completes
       tc_commit(drain);
@@ -349,16 +522,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;      // which half of the accumulator columns
     uint8_t* obuf = smem + SmemLayout::stage_out + (warp - 2) * 2048;
-    uint32_t acc_phase = 0;
+    uint32_t uses0 = 0, uses1 = 0;
+    int next_slot = 0;
     int buf = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const TileCoord c = decode_tile(p, tile);
+      const SlotPlan sp = plan_slots(p, c, next_slot);
+      bool ok = true;
+      for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
+        ok = mbar_wait(&accf[sl], (sl ? uses1 : uses0) & 1, ctl, kWhereGemmEpilogue);
       // warp-uniform decision: tcgen05.ld below is .sync.aligned
-      const bool ok = mbar_wait(accf, acc_phase, ctl, kWhereGemmEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf, obuf);
-      acc_phase ^= 1;
+      if (sp.swap) {
+        const uint32_t acc = tmem_base + kAccCol + sp.lo * 128;
+        if (sp.nt_tok == 32)
+          epilogue_swap<MODE, 32>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
+        else
+          epilogue_swap<MODE, 64>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
+      } else {
+        epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf, obuf);
+      }
+      uses0 += sp.lo == 0;
+      uses1 += sp.hi == 1;
       buf ^= 1;
     }
   }
@@ -448,6 +634,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RouterSmem::misc + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int m0 = blockIdx.y * 128, n0 = blockIdx.x * RBN;
+  // K split blockIdx.z of gridDim.z: stages [kt0, kt0 + KT), partial logits in slice blockIdx.z
+  const int KT = p.H / RBK / (int)gridDim.z;
+  const int kt0 = (int)blockIdx.z * KT;
+  float* const logits = p.logits + (long)blockIdx.z * p.T * p.E;
   if (threadIdx.x == 0) {
     for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
@@ -467,7 +657,6 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-  const int KT = p.H / RBK;
   if (warp == 0) {
     if (lane == 0) {
       uint32_t fills[RS];
@@ -478,9 +667,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereRouterProducer)) break;
         mbar_arrive_expect_tx(&full[stage], 3 * kRTile);
-        tma_load_2d(a_s + stage * kRTile, &tmX, kt * RBK, m0, &full[stage]);
-        tma_load_2d(bh_s + stage * kRTile, &tmWhi, kt * RBK, n0, &full[stage]);
-        tma_load_2d(bl_s + stage * kRTile, &tmWlo, kt * RBK, n0, &full[stage]);
+        const int kx = (kt0 + kt) * RBK;
+        tma_load_2d(a_s + stage * kRTile, &tmX, kx, m0, &full[stage]);
+        tma_load_2d(bh_s + stage * kRTile, &tmWhi, kx, n0, &full[stage]);
+        tma_load_2d(bl_s + stage * kRTile, &tmWlo, kx, n0, &full[stage]);
         fills[stage] += 1;
         if (++stage == RS) { stage = 0; phase ^= 1; }
       }
@@ -528,7 +718,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         tmem_ld_wait();
         const int e0 = n0 + ch * 32;
         if (t < p.T) {
-          float* dst = p.logits + (long)t * p.E + e0;
+          float* dst = logits + (long)t * p.E + e0;
           if (e0 + 32 <= p.E) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
@@ -567,9 +757,20 @@ __global__ void split_router_weights_kernel(const float* __restrict__ W, __nv_bf
 
 size_t router_tc_smem_bytes() { return RouterSmem::total + 1024; }
 
+int router_tc_splits(int T, int H, int E) {
+  if (E > kTopkMaxSplitE) return 1;
+  const long tiles = (long)((T + 127) / 128) * ((E + RBN - 1) / RBN);
+  const int kt = H / RBK;
+  int best = 1;
+  for (int s = 2; s <= 16; ++s)
+    if (kt % s == 0 && tiles * s <= 148 && (long)s * T * E <= (4l << 20)) best = s;
+  return best;
+}
+
 cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
                              const RouterArgs& args, cudaStream_t s) {
-  dim3 grid((args.E + RBN - 1) / RBN, (args.T + 127) / 128);
+  if (args.k_splits < 1 || (args.H / RBK) % args.k_splits != 0) return cudaErrorInvalidValue;
+  dim3 grid((args.E + RBN - 1) / RBN, (args.T + 127) / 128, args.k_splits);
   router_tc_kernel<<<grid, kRouterThreads, router_tc_smem_bytes(), s>>>(x, whi, wlo, args);
   return cudaGetLastError();
 }

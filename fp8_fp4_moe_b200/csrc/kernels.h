@@ -27,6 +27,8 @@ struct GemmArgs {
   int n_experts;       // E + shared
   int rows_total;      // R + shared * T
   int n_tiles_n;       // linear1: I/128; linear2: ceil(H/256)
+  int swap_rows;       // tiles with at most this many expert rows run transposed (0, 32 or 64)
+  int prefetch;        // weight K stages the producer prefetches into L2 ahead of its loads
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
   const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
@@ -59,12 +61,18 @@ cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const Gemm
 constexpr int kRouterThreads = 192;   // 6 warps: TMA, MMA, 4 x epilogue
 struct RouterArgs {
   int T, H, E;
-  float* logits;                      // [T][E] fp32
+  int k_splits;                       // K split into this many equal parts (divides H / 64)
+  float* logits;                      // [k_splits][T][E] fp32 partial sums
   uint32_t* status;
   uint64_t timeout_ns;
 };
 size_t router_tc_smem_bytes();
+// K splits of the tensor-core router for a T x E problem: enough CTAs to cover a 148-SM part,
+// each split a whole number of 64-wide K stages, at most 16 splits and 4 Mi partial floats.
+int router_tc_splits(int T, int H, int E);
 // x bf16 [T][H] and W_hi / W_lo bf16 [E][H] as 128-byte-swizzled TMA maps (box 64 x 128).
+// Split s of the K range writes its partial logits to logits + s * T * E; top-k adds the
+// k_splits parts in split order.
 cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
                              const RouterArgs& args, cudaStream_t s);
 // W fp32 [n] -> hi = bf16(W), lo = bf16(W - hi)
@@ -75,7 +83,11 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
                                  cudaStream_t s);
 // mode 0: select from logits (+bias), write ids/gates, then rank.  mode 1: rank given ids.
 // mode 1 validates the given ids (range, distinct per token) and records MOE_ERR_DEBUG_BOUNDS in `status`.
-cudaError_t launch_topk_rank(int mode, const float* logits, const float* bias, int32_t* topk_ids, float* gates,
+// logits holds n_parts partial [T][E] arrays (consecutive); a score is their sum in part order
+// (n_parts > 1 needs E <= kTopkMaxSplitE).
+constexpr int kTopkMaxSplitE = 256;
+cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const float* bias, int32_t* topk_ids,
+                             float* gates,
                              int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
                              cudaStream_t s);
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,

@@ -27,6 +27,9 @@ struct moe_plan_s {
   int inject_fault = 0;
   int static_weights = 0;
   int router_tc = 1;
+  int swap_rows = 0;
+  int prefetch = 0;
+  int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
@@ -121,6 +124,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
   a.mtile_start = at<int32_t>(p, p->off_mtile);
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
+  a.swap_rows = p->swap_rows;
+  a.prefetch = p->prefetch;
   if (mode == 1) {
     a.K = p->H;
     a.N = p->I;
@@ -175,10 +180,13 @@ int run_router(moe_plan_t p, const uint16_t* x, const float* W_router, cudaStrea
     if (rc != MOE_OK) return rc;
     p->x_cached = x;
   }
-  RouterArgs ra{p->T, p->H, p->E, at<float>(p, p->off_logits), region<uint32_t>(p, MOE_REGION_STATUS),
-                p->timeout_ns};
+  RouterArgs ra{p->T, p->H, p->E, p->router_splits, at<float>(p, p->off_logits),
+                region<uint32_t>(p, MOE_REGION_STATUS), p->timeout_ns};
   return cuda_rc(launch_router_tc(p->tmX, p->tmWhi, p->tmWlo, ra, s));
 }
+
+// partial logit arrays the router leaves for top-k
+int logit_parts(moe_plan_t p) { return use_tc_router(p) ? p->router_splits : 1; }
 
 // routing + dispatch + quantisation into the workspace
 int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias, cudaStream_t s) {
@@ -189,9 +197,9 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
   int rc = run_router(p, x, W_router, s);
   if (rc != MOE_OK) return rc;
   mark(p, 1 + MOE_PHASE_ROUTER, s);
-  if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, ids, gates, at<int32_t>(p, p->off_rank),
-                            at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E,
-                            p->k, s)) != cudaSuccess)
+  if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
+                            at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
+                            region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s)) != cudaSuccess)
     return cuda_rc(e);
   mark(p, 1 + MOE_PHASE_TOPK, s);
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
@@ -333,7 +341,10 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   reg(MOE_REGION_HQ, (size_t)rows * I);
   reg(MOE_REGION_HSF, (size_t)p->mt_cap * (I / 128) * 512);
   reg(MOE_REGION_Y, (size_t)rows * H * 2);
-  p->off_logits = add((size_t)T * E * 4);
+  // the tensor-core router's split count depends on the shape only, so results do not
+  // depend on the device or on options
+  p->router_splits = (E >= 16 && E % 16 == 0) ? router_tc_splits(T, H, E) : 1;
+  p->off_logits = add((size_t)p->router_splits * T * E * 4);
   p->off_rank = add(Tk * 4);
   p->off_gcounts = add((size_t)p->G * E * 4);
   p->off_gbase = add((size_t)p->G * E * 4);
@@ -378,6 +389,14 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
     case MOE_OPT_PHASE_EVENTS:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->phase_events = (int)value;
+      return MOE_OK;
+    case MOE_OPT_PREFETCH:
+      if (value < 0 || value > 64) return MOE_ERR_INVALID_ARG;
+      p->prefetch = (int)value;
+      return MOE_OK;
+    case MOE_OPT_SWAP_ROWS:
+      if (value != 0 && value != 32 && value != 64) return MOE_ERR_INVALID_ARG;
+      p->swap_rows = (int)value;
       return MOE_OK;
     default:
       return MOE_ERR_INVALID_ARG;
@@ -487,8 +506,9 @@ int moe_debug_routing(moe_plan_t p, const void* x, const float* W_router, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   rc = run_router(p, static_cast<const uint16_t*>(x), W_router, s);
   if (rc != MOE_OK) return rc;
-  cudaError_t e = launch_topk_rank(0, at<float>(p, p->off_logits), bias, topk_ids, gates, at<int32_t>(p, p->off_rank),
-                       at<int32_t>(p, p->off_gcounts), region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
+  cudaError_t e = launch_topk_rank(0, at<float>(p, p->off_logits), logit_parts(p), bias, topk_ids, gates,
+                                   at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
+                                   region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   return cuda_rc(e);
 }
 
@@ -500,7 +520,7 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
       !aligned(slot_pos, 4))
     return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_topk_rank(1, nullptr, nullptr, const_cast<int32_t*>(topk_ids), nullptr,
+  cudaError_t e = launch_topk_rank(1, nullptr, 1, nullptr, const_cast<int32_t*>(topk_ids), nullptr,
                                    at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
                                    region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;

@@ -77,7 +77,7 @@ extern "C" int moe_route_noalloc(int T, int H, int E, int k, const void* x_bf16,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (moe::launch_router_logits(static_cast<const uint16_t*>(x_bf16), W_router, logits, T, H, E, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe::launch_topk_rank(0, logits, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k, s) !=
+  if (moe::launch_topk_rank(0, logits, 1, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k, s) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;

@@ -126,6 +126,57 @@ __global__ void __launch_bounds__(256) router_logits_warp_kernel(const uint16_t*
 // once per block, then each warp takes 4 tokens at a time so every W value read
 // from shared memory feeds 4 FMAs.
 constexpr int kSmemRouterMaxBytes = 200 * 1024;
+
+// Few tokens: one block per (expert, token) so that all SMs stream W_router.  Thread i covers
+// channels [8i, 8i + 8) of every 2048-channel pass; four passes are loaded before any is
+// used.  The eight warps' partial sums are added in warp order (deterministic).
+__global__ void __launch_bounds__(256) router_logits_split_kernel(const uint16_t* __restrict__ x,
+                                                                  const float* __restrict__ W,
+                                                                  float* __restrict__ logits, int T, int H, int E) {
+  __shared__ float part[8];
+  const int e = blockIdx.x, t = blockIdx.y;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  const uint16_t* xr = x + (long)t * H;
+  const float* wr = W + (long)e * H;
+  float acc = 0.f;
+  for (int base = threadIdx.x * 8; base < H; base += 4 * 2048) {
+    uint4 xv[4];
+    float4 w0[4], w1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = base + u * 2048;
+      if (c < H) {
+        xv[u] = __ldg(reinterpret_cast<const uint4*>(xr + c));
+        w0[u] = __ldg(reinterpret_cast<const float4*>(wr + c));
+        w1[u] = __ldg(reinterpret_cast<const float4*>(wr + c) + 1);
+      } else {
+        xv[u] = make_uint4(0, 0, 0, 0);
+        w0[u] = w1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc = fmaf(__uint_as_float(xv[u].x << 16), w0[u].x, acc);
+      acc = fmaf(__uint_as_float(xv[u].x & 0xFFFF0000u), w0[u].y, acc);
+      acc = fmaf(__uint_as_float(xv[u].y << 16), w0[u].z, acc);
+      acc = fmaf(__uint_as_float(xv[u].y & 0xFFFF0000u), w0[u].w, acc);
+      acc = fmaf(__uint_as_float(xv[u].z << 16), w1[u].x, acc);
+      acc = fmaf(__uint_as_float(xv[u].z & 0xFFFF0000u), w1[u].y, acc);
+      acc = fmaf(__uint_as_float(xv[u].w << 16), w1[u].z, acc);
+      acc = fmaf(__uint_as_float(xv[u].w & 0xFFFF0000u), w1[u].w, acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) part[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = part[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) v += part[w];
+    logits[(long)t * E + e] = v;
+  }
+}
 __global__ void __launch_bounds__(256) router_logits_smem_kernel(const uint16_t* __restrict__ x,
                                                                  const float* __restrict__ W,
                                                                  float* __restrict__ logits, int T, int H, int E) {
@@ -189,31 +240,59 @@ __global__ void __launch_bounds__(256) router_logits_smem_kernel(const uint16_t*
 // Then warp 0 ranks the group's copies: lane = token, and each expert keeps a
 // 32-bit mask of the group's tokens that chose it.  A copy's rank inside its
 // expert is the number of lower lanes in that mask (ascending token order).
-__global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* __restrict__ logits,
+__global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* __restrict__ logits, int n_parts,
                                                          const float* __restrict__ bias, int32_t* topk_ids,
                                                          float* gates, int32_t* __restrict__ local_rank,
                                                          int32_t* __restrict__ group_counts, uint32_t* status,
                                                          int T, int E, int k) {
   __shared__ int32_t ids_s[32][16];
   __shared__ uint32_t mask_s[1024];
+  __shared__ float sum_s[32 * kTopkMaxSplitE];     // the group's summed logits when n_parts > 1
   const int g = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   for (int e = threadIdx.x; e < E; e += blockDim.x) mask_s[e] = 0u;
+  if (mode == 0 && n_parts > 1) {
+    // the whole block adds the parts of the group's 32 x E logits, each in part order
+    // (E % 4 == 0 here: the parts come from the tensor-core router, E % 16 == 0)
+    const long stride4 = (long)T * E / 4;
+    const int n4 = min(32, T - g * 32) * E / 4;
+    const float4* base = reinterpret_cast<const float4*>(logits + (long)g * 32 * E);
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s0 = 0; s0 < n_parts; s0 += 8) {
+        float4 part[8];                // eight parts in flight, then added in part order
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          if (s0 + s < n_parts) part[s] = __ldg(base + (s0 + s) * stride4 + i);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          if (s0 + s < n_parts) {
+            if (s0 + s == 0) v = part[s];
+            else { v.x += part[s].x; v.y += part[s].y; v.z += part[s].z; v.w += part[s].w; }
+          }
+      }
+      reinterpret_cast<float4*>(sum_s)[i] = v;
+    }
+    __syncthreads();
+  }
   const int t = g * 32 + warp;
   if (t < T) {
     if (mode == 0) {
-      const float* row = logits + (long)t * E;
+      const float* row = n_parts > 1 ? sum_s + warp * E : logits + (long)t * E;
+      auto score = [&](int e) { return row[e]; };
       // k rounds of a warp arg-max over (score + bias), lower id on ties
       float chosen_score = 0.f;   // unbiased score of this lane's slot (lane < k)
       int chosen_id = -1;
       uint32_t taken = 0u;        // bit i: expert lane + 32*i already selected (E <= 1024)
       float cached[8];            // E <= 256: this lane's biased scores, read once
+      float raw[8];               // ... and the unbiased ones
       const bool use_cache = E <= 256;
       if (use_cache) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int e = lane + 32 * i;
-          cached[i] = (e < E) ? row[e] + bias[e] : 0.f;
+          raw[i] = (e < E) ? score(e) : 0.f;
+          cached[i] = (e < E) ? raw[i] + bias[e] : 0.f;
         }
       }
       for (int j = 0; j < k; ++j) {
@@ -233,7 +312,7 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
           for (int i = 0, e = lane; e < E; ++i, e += 32) {
             if (taken & (1u << i)) continue;
             if (free_id == 0x7FFFFFFF) free_id = e;
-            const float b = row[e] + bias[e];
+            const float b = score(e) + bias[e];
             if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
           }
         }
@@ -246,7 +325,17 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
         }
         if (best_id == 0x7FFFFFFF) best_id = free_id;   // k <= E guarantees free_id < E
         if ((best_id & 31) == lane) taken |= 1u << (best_id >> 5);
-        if (lane == j) { chosen_id = best_id; chosen_score = row[best_id]; }
+        float s_best;
+        if (use_cache) {               // the owner lane holds the unbiased score in registers
+          float mine = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (i == (best_id >> 5)) mine = raw[i];
+          s_best = __shfl_sync(0xffffffffu, mine, best_id & 31);
+        } else {
+          s_best = score(best_id);
+        }
+        if (lane == j) { chosen_id = best_id; chosen_score = s_best; }
       }
       // softmax over the unbiased scores of the selected experts
       float m = (lane < k) ? chosen_score : -INFINITY;
@@ -545,15 +634,16 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
     int grid = (groups + 7) / 8;
     if (grid > 148) grid = 148;
     router_logits_smem_kernel<<<grid, 256, (size_t)E * H * 4, s>>>(x, W_r, logits, T, H, E);
+  } else if ((long)T * E <= 4096) {
+    router_logits_split_kernel<<<dim3(E, T), 256, 0, s>>>(x, W_r, logits, T, H, E);
   } else if (E <= 32 || (long)T * E <= 16384) {
-    // warp per (token, expert chunk); one expert per warp when few tokens must cover many experts
-    const int ec = (E <= 32) ? 8 : ((long)T * E <= 4096 ? 1 : 2);
+    // warp per (token, expert chunk)
+    const int ec = (E <= 32) ? 8 : 2;
     const long items = (long)T * ((E + ec - 1) / ec);
     const long blocks = (items + 7) / 8;
     const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
     if (ec == 8) router_logits_warp_kernel<8><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
-    else if (ec == 2) router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
-    else router_logits_warp_kernel<1><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
+    else router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
   } else if (E <= 16) {
     dim3 grid((T + 63) / 64, (E + 15) / 16);
     router_logits_kernel<16><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
@@ -564,12 +654,13 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk_rank(int mode, const float* logits, const float* bias, int32_t* topk_ids, float* gates,
-                             int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
-                             cudaStream_t s) {
+cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const float* bias, int32_t* topk_ids,
+                             float* gates, int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E,
+                             int k, cudaStream_t s) {
+  if (n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
   const int G = (T + 31) / 32;
-  topk_rank_kernel<<<G, 1024, 0, s>>>(mode, logits, bias, topk_ids, gates, local_rank, group_counts, status, T, E,
-                                      k);
+  topk_rank_kernel<<<G, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status,
+                                      T, E, k);
   return cudaGetLastError();
 }
 

@@ -75,6 +75,9 @@ class Workload:
     def with_tokens(self, T: int) -> "Workload":
         return dataclasses.replace(self, T=T, name=f"{self.name}@T{T}")
 
+    def with_experts(self, E: int) -> "Workload":
+        return dataclasses.replace(self, E=E, k=min(self.k, E), name=f"{self.name}@E{E}")
+
 
 WORKLOADS = {
     "tiny": Workload("tiny", T=64, H=256, I=512, E=8, k=2, shared=0, router_std=0.02,

@@ -84,13 +84,21 @@ enum moe_option {
                                   and the split router weights built by the last
                                   moe_prepare_weights (or forward) from those pointers.
                                   0 (default): every forward rebuilds them.              */
-  MOE_OPT_GRAPH = 7            /* 1 = moe_forward records its launch sequence as a CUDA
+  MOE_OPT_GRAPH = 7,           /* 1 = moe_forward records its launch sequence as a CUDA
                                   graph the first time it sees a set of argument pointers
                                   (up to 4 sets per plan) and replays it on later calls,
                                   removing per-kernel launch overhead.  Not used while the
                                   caller's stream is capturing or MOE_OPT_PHASE_EVENTS is
                                   1.  The CUDA runtime may reserve memory for the recorded
                                   graphs; changing any option drops them.  Default 0.    */
+  MOE_OPT_SWAP_ROWS = 8,       /* grouped GEMM row tiles holding at most this many rows of
+                                  their expert (0, 32 or 64; default 0) are computed
+                                  transposed: 128 weight rows as the MMA's M side and the
+                                  tile's tokens as N = 32 or 64, so few-token experts do
+                                  not pay for 128-row MMAs.  0 = always 128 token rows.   */
+  MOE_OPT_PREFETCH = 9         /* grouped GEMM: how many K stages of weight tiles the TMA
+                                  producer requests into L2 ahead of its shared-memory
+                                  loads (0..64, default 0 = off)                          */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -86,6 +86,10 @@ def test_options_and_unbound_plan(L):
     assert L.moe_plan_set_option(h, binding.MOE_OPT_TIMEOUT_NS, 0) == binding.MOE_ERR_INVALID_ARG
     assert L.moe_plan_set_option(h, binding.MOE_OPT_INJECT_FAULT, 2) == binding.MOE_ERR_INVALID_ARG
     assert L.moe_plan_set_option(h, 12345, 1) == binding.MOE_ERR_INVALID_ARG
+    for v in (0, 32, 64):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, v) == 0
+    for v in (-1, 16, 65, 128):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, v) == binding.MOE_ERR_INVALID_ARG
     # no workspace bound yet: every compute entry point refuses before touching a device
     null = [None] * 9
     assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE

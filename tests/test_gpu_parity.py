@@ -34,8 +34,11 @@ SMALL = {
 }
 
 
-def plan_for(w):
-    return binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+def plan_for(w, swap_rows=None):
+    p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+    if swap_rows is not None:
+        p.set_option(binding.MOE_OPT_SWAP_ROWS, swap_rows)
+    return p
 
 
 # --------------------------------------------------------------------------- quantisation
@@ -138,12 +141,15 @@ def test_dispatch_flags_invalid_ids(cuda_lib):
 
 # --------------------------------------------------------------------------- whole layer
 
+# swap_rows 64: row tiles with <= 64 rows of their expert run transposed (weights as the
+# MMA's M side); 0: every tile has 128 token rows
+@pytest.mark.parametrize("swap_rows", [64, 0])
 @pytest.mark.parametrize("name", list(SMALL))
-def test_forward_matches_oracle(cuda_lib, name):
+def test_forward_matches_oracle(cuda_lib, name, swap_rows):
     w = SMALL[name]
     case = make_case(w, seed=7)
     d = to_device(case)
-    p = plan_for(w)
+    p = plan_for(w, swap_rows)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
     ref = oracle_forward(case, w)
@@ -165,11 +171,12 @@ def test_forward_matches_oracle(cuda_lib, name):
     assert_output_close(bits(out), ref["y"], name)
 
 
-def test_forward_intermediates_match_oracle(cuda_lib):
-    w = SMALL["ragged_shared"]
+@pytest.mark.parametrize("name,swap_rows", [("ragged_shared", 64), ("ragged_shared", 0), ("dsv3_like", 64)])
+def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows):
+    w = SMALL[name]
     case = make_case(w, seed=8)
     d = to_device(case)
-    p = plan_for(w)
+    p = plan_for(w, swap_rows)
     p.forward(**d)
     ref = oracle_forward(case, w, keep_rows=True)
     hq = p.region("hq").cpu().numpy()
@@ -214,6 +221,43 @@ def test_forward_all_tokens_on_one_expert(cuda_lib):
     assert ref["counts"].tolist() == [0, 0, 700, 0, 0, 0, 0, 0, 700]
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
     assert_output_close(bits(out), ref["y"], "skew")
+
+
+def _count_mix_case(counts, H=256, I_=384, seed=3):
+    """k = 1 routing with prescribed expert loads: token t carries a +10 spike at channel
+    target(t) < E over N(0, 0.1) noise and W_router is the identity on the first E channels,
+    so the top-1 logit of token t is expert target(t) by a margin of about 10."""
+    E = len(counts)
+    target = np.repeat(np.arange(E), counts)
+    T = len(target)
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(T, generator=g)
+    target = torch.from_numpy(target)[perm]
+    w = W("count_mix", T=T, H=H, I_=I_, E=E, k=1, shared=1)
+    case = make_case(w, seed=seed, screened=False)
+    x = 0.1 * torch.randn(T, H, generator=g)
+    x[torch.arange(T), target] += 10.0
+    case["x"] = x.to(torch.bfloat16)
+    Wr = torch.zeros(E, H)
+    Wr[torch.arange(E), torch.arange(E)] = 1.0
+    case["W_router"] = Wr
+    case["bias"] = torch.zeros(E)
+    return w, case
+
+
+@pytest.mark.parametrize("swap_rows", [64, 32, 0])
+def test_forward_tile_row_boundaries(cuda_lib, swap_rows):
+    # expert loads on both sides of 32, 64 and 128 rows, plus an empty expert
+    counts = [1, 17, 32, 33, 64, 65, 128, 129, 0, 200]
+    w, case = _count_mix_case(counts)
+    d = to_device(case)
+    p = plan_for(w, swap_rows)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref = oracle_forward(case, w)
+    assert ref["counts"].tolist() == counts + [w.T]
+    assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
+    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows}")
 
 
 def test_token_permutation_permutes_output(cuda_lib):
