@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch kernels one by one (no CUDA graph replay)")
     ap.add_argument("--opt", action="append", default=[], metavar="NAME=VALUE",
-                    help="plan option, e.g. SWAP_ROWS=0 or PREFETCH=4 (MOE_OPT_<NAME>); repeatable")
+                    help="plan option, e.g. SWAP_ROWS=64 or MAX_SMS=74 (MOE_OPT_<NAME>); repeatable")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for ncu captures)")
     ap.add_argument("--experts", type=int, default=None,

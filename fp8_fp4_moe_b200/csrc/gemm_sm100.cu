@@ -396,28 +396,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       bool withhold = p.inject_fault != 0 && blockIdx.x == 0;
-      // L2 prefetch cursor: walks this CTA's (tile, K stage) sequence p.prefetch stages ahead of
-      // the loads, so weight tiles stream from HBM into L2 while the shared-memory ring is full
-      int pf_tile = blockIdx.x, pf_kt = 0;
-      TileCoord pc{};
-      if (pf_tile < total_tiles) pc = decode_tile(p, pf_tile);
-      auto prefetch_next = [&]() {
-        if (pf_tile >= total_tiles) return;
-        if constexpr (MODE == 1) {
-          const int brow = pc.e * p.rows_b + pc.nt * 128;
-          tma_prefetch_l2_2d(&tmB, pf_kt * BK, brow);
-          tma_prefetch_l2_2d(&tmB, pf_kt * BK, brow + p.N);
-        } else {
-          tma_prefetch_l2_2d(&tmB, pf_kt * BK, pc.e * p.rows_b + pc.nt * BN);
-        }
-        bulk_prefetch_l2(p.sfb + (((long)pc.e * p.n_tiles_n + pc.nt) * KT + pf_kt) * kSfbBytes, kSfbBytes);
-        if (++pf_kt == KT) {
-          pf_kt = 0;
-          pf_tile += gridDim.x;
-          if (pf_tile < total_tiles) pc = decode_tile(p, pf_tile);
-        }
-      };
-      for (int i = 0; i < p.prefetch; ++i) prefetch_next();
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         const TileCoord c = decode_tile(p, tile);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
@@ -446,7 +424,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bulk_load(sfb_s + stage * kSfbBytes, sfb_tile + kt * kSfbBytes, kSfbBytes, &full[stage]);
             fills[stage] += 1;
           }
-          if (p.prefetch > 0) prefetch_next();
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }

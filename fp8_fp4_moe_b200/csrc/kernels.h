@@ -28,7 +28,6 @@ struct GemmArgs {
   int rows_total;      // R + shared * T
   int n_tiles_n;       // linear1: I/128; linear2: ceil(H/256)
   int swap_rows;       // tiles with at most this many expert rows run transposed (0, 32 or 64)
-  int prefetch;        // weight K stages the producer prefetches into L2 ahead of its loads
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
   const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)

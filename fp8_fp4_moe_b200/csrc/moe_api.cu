@@ -28,7 +28,6 @@ struct moe_plan_s {
   int static_weights = 0;
   int router_tc = 1;
   int swap_rows = 0;
-  int prefetch = 0;
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
@@ -125,7 +124,6 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
   a.swap_rows = p->swap_rows;
-  a.prefetch = p->prefetch;
   if (mode == 1) {
     a.K = p->H;
     a.N = p->I;
@@ -389,10 +387,6 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
     case MOE_OPT_PHASE_EVENTS:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->phase_events = (int)value;
-      return MOE_OK;
-    case MOE_OPT_PREFETCH:
-      if (value < 0 || value > 64) return MOE_ERR_INVALID_ARG;
-      p->prefetch = (int)value;
       return MOE_OK;
     case MOE_OPT_SWAP_ROWS:
       if (value != 0 && value != 32 && value != 64) return MOE_ERR_INVALID_ARG;

@@ -91,14 +91,11 @@ enum moe_option {
                                   caller's stream is capturing or MOE_OPT_PHASE_EVENTS is
                                   1.  The CUDA runtime may reserve memory for the recorded
                                   graphs; changing any option drops them.  Default 0.    */
-  MOE_OPT_SWAP_ROWS = 8,       /* grouped GEMM row tiles holding at most this many rows of
+  MOE_OPT_SWAP_ROWS = 8        /* grouped GEMM row tiles holding at most this many rows of
                                   their expert (0, 32 or 64; default 0) are computed
                                   transposed: 128 weight rows as the MMA's M side and the
                                   tile's tokens as N = 32 or 64, so few-token experts do
                                   not pay for 128-row MMAs.  0 = always 128 token rows.   */
-  MOE_OPT_PREFETCH = 9         /* grouped GEMM: how many K stages of weight tiles the TMA
-                                  producer requests into L2 ahead of its shared-memory
-                                  loads (0..64, default 0 = off)                          */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */
