@@ -31,6 +31,7 @@ MOE_OPT_ROUTER_TC = 4
 MOE_OPT_STATIC_WEIGHTS = 6
 MOE_OPT_GRAPH = 7
 MOE_OPT_SWAP_ROWS = 8
+MOE_OPT_PAIR_TILES = 9
 
 PHASES = ["router", "topk_rank", "scan", "scatter_quant", "prepare", "linear1", "linear2", "combine"]
 

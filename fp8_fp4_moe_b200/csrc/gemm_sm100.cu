@@ -127,6 +127,20 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
 __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
 }
+// Epilogue-wide AND of `ok` (a barrier too): every epilogue warp takes the same branch, so a
+// wait that timed out in one warp cannot leave the others blocked in a later epi_bar.
+__device__ __forceinline__ bool epi_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "n"(kEpiWarps * 32)
+      : "memory");
+  return r != 0;
+}
 
 // Store 64 bytes of each of the warp's 32 rows (lane l holds row l's bytes in v[0..3]) so that
 // every global store instruction writes whole 32-byte sectors: the chunk goes through a
@@ -150,10 +164,21 @@ __device__ __forceinline__ void store_rows_64b(uint8_t* buf, const uint4 (&v)[4]
   __syncwarp();
 }
 
+// Release the accumulator: both slots of this CTA, or (CTA pairs) the rank-0 CTA's barrier
+// through its cluster-window address.
+__device__ __forceinline__ void release_acc(uint64_t* acce, uint32_t acce_remote) {
+  if (acce_remote != 0) {
+    mbar_arrive_cluster(acce_remote);
+  } else {
+    mbar_arrive(&acce[0]);
+    mbar_arrive(&acce[1]);
+  }
+}
+
 template <int MODE>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t tmem_base, int q,
-                                              int half, int lane, uint64_t* acce, float* amax_s, int buf,
-                                              uint8_t* obuf) {
+                                              int half, int lane, uint64_t* acce, uint32_t acce_remote,
+                                              float* amax_s, int buf, uint8_t* obuf) {
   const int m = q * 32 + lane;                         // accumulator row = TMEM lane
   const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
   const bool valid = c.mt * BM + m < c.count;
@@ -167,10 +192,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {                                   // accumulator may be overwritten now
-      mbar_arrive(&acce[0]);
-      mbar_arrive(&acce[1]);
-    }
+    if (lane == 0) release_acc(acce, acce_remote);     // accumulator may be overwritten now
     float h[64];
     float amax = 0.f;
 #pragma unroll
@@ -219,10 +241,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&acce[0]);
-      mbar_arrive(&acce[1]);
-    }
+    if (lane == 0) release_acc(acce, acce_remote);
     const int col0 = c.nt * BN + half * 128;
     uint8_t* dst0 = reinterpret_cast<uint8_t*>(p.y + (long)(c.row0 + q * 32) * p.N + col0);
 #pragma unroll
@@ -508,8 +527,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
         ok = mbar_wait(&accf[sl], (sl ? uses1 : uses0) & 1, ctl, kWhereGemmEpilogue);
-      // warp-uniform decision: tcgen05.ld below is .sync.aligned
-      if (!__all_sync(0xffffffffu, ok)) break;
+      // epilogue-uniform decision: tcgen05.ld below is .sync.aligned and the epilogue syncs
+      if (!epi_all(ok)) break;
       tc_fence_after();
       if (sp.swap) {
         const uint32_t acc = tmem_base + kAccCol + sp.lo * 128;
@@ -518,7 +537,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         else
           epilogue_swap<MODE, 64>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
       } else {
-        epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, amax_s, buf, obuf);
+        epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, 0u, amax_s, buf, obuf);
       }
       uses0 += sp.lo == 0;
       uses1 += sp.hi == 1;
@@ -530,6 +549,218 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ CTA-pair grouped GEMM
+// Same tiles as above with two row tiles per CTA pair: rank r of a 2-CTA cluster holds row
+// tile 2*pm + r of its expert (A, 128 rows) and half of the 256 B rows (linear1: rank 0 the
+// gate rows, rank 1 the up rows; linear2: rows 128*r.. of the 256-row tile), and one
+// tcgen05.mma.cta_group::2 (M = 256, N = 256) per 32-deep K step, issued by rank 0, writes
+// each CTA's 128 x 256 accumulator into its own TMEM.  Each CTA loads its own scale atom and
+// the full 256-row weight scale unit (both 2-D TMA), every copy completing on rank 0's stage
+// barrier; rank 0's MMA commits multicast to both CTAs' empty / accumulator barriers; the
+// epilogue warps of both CTAs release the accumulator on rank 0's barrier.  Half the B bytes
+// per CTA leave room for 6 stages.
+constexpr int SP = 6;
+constexpr uint32_t kBHalfBytes = 128 * BK;               // 16 KB of shared memory (unpacked E2M1)
+constexpr uint32_t kPairTxBytesNoA = 128 * BK / 2 + kSfaBytes + kSfbBytes;   // per CTA, without A
+
+struct PairSmem {
+  static constexpr uint32_t a = 0;
+  static constexpr uint32_t b = a + SP * kATileBytes;
+  static constexpr uint32_t sfa = b + SP * kBHalfBytes;
+  static constexpr uint32_t sfb = sfa + SP * kSfaBytes;
+  static constexpr uint32_t amax = sfb + SP * kSfbBytes;
+  static constexpr uint32_t stage_out = amax + 2 * 2 * 128 * 4;
+  static constexpr uint32_t bars = stage_out + 8 * 2048;
+  // full[SP], empty[SP], accf, acce, drain
+  static constexpr uint32_t n_bars = 2 * SP + 3;
+  static constexpr uint32_t misc = bars + n_bars * 8;
+  static constexpr uint32_t total = misc + 16;
+};
+
+// Tile `tile` of the pair grid as seen by CTA `rank`: row tile 2*pm + rank of the expert (its
+// rows can be 0 for rank 1 on an expert with an odd number of row tiles).
+__device__ __forceinline__ TileCoord decode_pair_tile(const GemmArgs& p, int tile, int rank) {
+  int lo = 0, hi = p.n_experts;
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(p.ptile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
+  }
+  TileCoord c;
+  c.e = lo;
+  c.count = __ldg(p.counts + lo);
+  const int mtiles = (c.count + BM - 1) / BM;
+  const int ptiles = (mtiles + 1) / 2;
+  const int local = tile - __ldg(p.ptile_start + lo) * p.n_tiles_n;
+  c.nt = local / ptiles;
+  c.mt = 2 * (local - c.nt * ptiles) + rank;
+  c.row0 = __ldg(p.offsets + lo) + c.mt * BM;
+  c.gmt = __ldg(p.mtile_start + lo) + c.mt;
+  c.rows = max(0, min(BM, c.count - c.mt * BM));
+  return c;
+}
+
+__device__ __forceinline__ int a_box_sel(int rows) { return rows <= 16 ? 0 : rows <= 32 ? 1 : rows <= 64 ? 2 : 3; }
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmSfa, const __grid_constant__ CUtensorMap tmSfb,
+                             const GemmArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_s = smem + PairSmem::a;
+  uint8_t* b_s = smem + PairSmem::b;
+  uint8_t* sfa_s = smem + PairSmem::sfa;
+  uint8_t* sfb_s = smem + PairSmem::sfb;
+  float* amax_s = reinterpret_cast<float*>(smem + PairSmem::amax);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PairSmem::bars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + SP;
+  uint64_t* accf = bars + 2 * SP;
+  uint64_t* acce = accf + 1;
+  uint64_t* drain = accf + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PairSmem::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PairSmem::misc + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int rank = (int)cluster_ctarank();
+  const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&full[s], 1);          // rank 0's: its producer's arrive + both CTAs' bytes
+      mbar_init(&empty[s], 1);         // each CTA's: rank 0's multicast commit
+    }
+    mbar_init(accf, 1);                // each CTA's: rank 0's multicast commit
+    mbar_init(acce, 2 * kEpiWarps);    // rank 0's: the epilogue warps of both CTAs
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(&tmA.m[i]);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmSfa);
+    tma_prefetch_desc(&tmSfb);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  __syncthreads();
+  cluster_sync();                      // the peer's barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  const int total_tiles = __ldg(p.ptile_start + p.n_experts) * p.n_tiles_n;
+  const int KT = p.K / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t fills[SP];
+#pragma unroll
+      for (int s = 0; s < SP; ++s) fills[s] = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        const TileCoord c = decode_pair_tile(p, tile, rank);
+        const int a_sel = a_box_sel(c.rows);
+        // rank 0 expects the bytes of both CTAs: the peer's A box follows from its rows
+        const int peer_rows = max(0, min(BM, c.count - (c.mt + 1) * BM));
+        const uint32_t tx = 2 * kPairTxBytesNoA + ((16u << a_sel) + (16u << a_box_sel(peer_rows))) * BK;
+        const int brow = MODE == 1 ? c.e * p.rows_b + rank * p.N + c.nt * 128 : c.e * p.rows_b + c.nt * BN + rank * 128;
+        const int sfa_row = (c.gmt * KT) * 2;
+        const int sfb_row = ((c.e * p.n_tiles_n + c.nt) * KT) * 4;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(&full[stage], 0);
+          if (rank == 0) {
+            mbar_arrive_expect_tx(&full[stage], tx);
+            fills[stage] += 1;
+          }
+          tma_load_2d_pair(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, fb);
+          tma_load_2d_pair(b_s + stage * kBHalfBytes, &tmB, kt * BK, brow, fb);
+          tma_load_2d_pair(sfa_s + stage * kSfaBytes, &tmSfa, 0, sfa_row + kt * 2, fb);
+          tma_load_2d_pair(sfb_s + stage * kSfbBytes, &tmSfb, 0, sfb_row + kt * 4, fb);
+          if (++stage == SP) { stage = 0; phase ^= 1; }
+        }
+      }
+      // rank 0's stage barriers count both CTAs' copies: waiting for them covers the peer too
+#pragma unroll
+      for (int s = 0; s < SP; ++s) {
+        if (fills[s] > 0 && !mbar_wait_drain(&full[s], (fills[s] - 1) & 1, p.timeout_ns)) {
+          report_status(p.status, kStatusTimeout, kWhereGemmDrain, s);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (rank 0)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        if (!mbar_wait(acce, acc_phase ^ 1, ctl, kWhereGemmMma)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, ctl, kWhereGemmMma + 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_addr = smem_u32(sfa_s + stage * kSfaBytes);
+          const uint32_t sfb_addr = smem_u32(sfb_s + stage * kSfbBytes);
+          tc_cp_32x128b_warpx4_pair(tmem_base + kSfaCol, sf_desc(sfa_addr));
+          tc_cp_32x128b_warpx4_pair(tmem_base + kSfbCol, sf_desc(sfb_addr));
+          tc_cp_32x128b_warpx4_pair(tmem_base + kSfbCol + 4, sf_desc(sfb_addr + 512));
+          const uint32_t a_addr = smem_u32(a_s + stage * kATileBytes);
+          const uint32_t b_addr = smem_u32(b_s + stage * kBHalfBytes);
+#pragma unroll
+          for (int kb = 0; kb < BK / 32; ++kb) {
+            tc_mma_mxf8f6f4_pair(tmem_base + kAccCol, sw128_desc(a_addr + kb * 32), sw128_desc(b_addr + kb * 32),
+                                 idesc_mxf8f6f4(2 * BM, BN, kb, kb), tmem_base + kSfaCol, tmem_base + kSfbCol,
+                                 (kt | kb) != 0);
+          }
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == SP) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit_pair(accf, 0x3);
+        acc_phase ^= 1;
+      }
+      tc_commit_pair(drain, 0x1);
+      if (!mbar_wait_drain(drain, 0, p.timeout_ns)) report_status(p.status, kStatusTimeout, kWhereGemmDrain, 9);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 2) / 4;
+    uint8_t* obuf = smem + PairSmem::stage_out + (warp - 2) * 2048;
+    const uint32_t acce0 = mapa_shared(acce, 0);
+    uint32_t acc_phase = 0;
+    int buf = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const TileCoord c = decode_pair_tile(p, tile, rank);
+      const bool ok = mbar_wait(accf, acc_phase, ctl, kWhereGemmEpilogue);
+      if (!epi_all(ok)) break;
+      tc_fence_after();
+      epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, acce0, amax_s, buf, obuf);
+      acc_phase ^= 1;
+      buf ^= 1;
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();                      // no CTA leaves while its peer may still touch its memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -759,6 +990,8 @@ cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* 
 }
 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
+size_t gemm_pair_smem_bytes() { return PairSmem::total + 1024; }
+int g_pair_clusters[64] = {};
 
 cudaError_t gemm_prepare_device() {
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -769,8 +1002,51 @@ cudaError_t gemm_prepare_device() {
   e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)router_tc_smem_bytes());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_smem_bytes());
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes());
+  if (e != cudaSuccess) return e;
+  for (int mode = 1; mode <= 2; ++mode) {
+    const void* fn = mode == 1 ? (const void*)grouped_gemm_pair_kernel<1> : (const void*)grouped_gemm_pair_kernel<2>;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_pair_smem_bytes());
+    if (e != cudaSuccess) return e;
+  }
+  // co-resident pairs: a persistent grid of more clusters than fit would run in two waves
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 148, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = gemm_pair_smem_bytes();
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, (const void*)grouped_gemm_pair_kernel<1>, &cfg);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) g_pair_clusters[dev] = clusters;
+  return cudaSuccess;
+}
+
+int gemm_pair_max_clusters() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  return g_pair_clusters[dev];
+}
+
+cudaError_t launch_gemm_pair_linear1(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                                     const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
+  grouped_gemm_pair_kernel<1><<<2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s>>>(a, b, sfa, sfb, args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_pair_linear2(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                                     const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
+  grouped_gemm_pair_kernel<2><<<2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s>>>(a, b, sfa, sfb, args);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,

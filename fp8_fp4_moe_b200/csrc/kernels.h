@@ -31,6 +31,7 @@ struct GemmArgs {
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
   const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
+  const int32_t* ptile_start;  // [n_experts + 1] prefix sum of ceil(ceil(count/128)/2) (CTA pairs)
   const uint8_t* sfa;          // activation scale atoms
   const uint8_t* sfb;          // weight scale units
   uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
@@ -55,6 +56,14 @@ cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const Gemm
                                 cudaStream_t s);
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s);
+// CTA-pair variants: b with 128-row boxes (each CTA loads half of the 256 B rows), scale atoms
+// and weight scale units as 2-D uint8 maps of 256-byte rows (boxes of 2 and 4 rows); grid =
+// 2 x pairs.
+cudaError_t launch_gemm_pair_linear1(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                                     const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s);
+cudaError_t launch_gemm_pair_linear2(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
+                                     const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s);
+int gemm_pair_max_clusters();        // co-resident CTA pairs on this device (after gemm_prepare_device)
 
 // ---- router on tensor cores (gemm_sm100.cu) -------------------------------------
 constexpr int kRouterThreads = 192;   // 6 warps: TMA, MMA, 4 x epilogue
@@ -90,8 +99,8 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
                              int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
                              cudaStream_t s);
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
-                                 int32_t* group_base, int32_t* mtile_start, int T, int E, int k, int shared,
-                                 cudaStream_t s);
+                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
+                                 int k, int shared, cudaStream_t s);
 // Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms.
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,

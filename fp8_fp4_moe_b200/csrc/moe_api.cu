@@ -28,11 +28,12 @@ struct moe_plan_s {
   int static_weights = 0;
   int router_tc = 1;
   int swap_rows = 0;
+  int pair_mode = 0;                // MOE_OPT_PAIR_TILES
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
-  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_w1sf, off_w2sf, off_whi, off_wlo;
+  size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_ptile, off_w1sf, off_w2sf, off_whi, off_wlo;
   long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
   // bound state
@@ -42,6 +43,7 @@ struct moe_plan_s {
   int num_sms = 0;
   alignas(64) AMaps amA1, amA2;
   alignas(64) CUtensorMap tmB1, tmB2, tmX, tmWhi, tmWlo;
+  alignas(64) CUtensorMap tmB2p, tmSfa1, tmSfa2, tmSfb1, tmSfb2;   // CTA-pair GEMM operands
   const void* x_cached = nullptr;        // tmX encodes this x pointer
   const void* wr_prepared = nullptr;     // W_router the hi/lo split was made from
   const void* w1_cached = nullptr;
@@ -80,15 +82,15 @@ int get_encode() {
 }
 
 int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (get_encode() != MOE_OK) return MOE_ERR_CUDA;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -121,6 +123,7 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
   a.counts = region<int32_t>(p, MOE_REGION_COUNTS);
   a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
   a.mtile_start = at<int32_t>(p, p->off_mtile);
+  a.ptile_start = at<int32_t>(p, p->off_ptile);
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
   a.swap_rows = p->swap_rows;
@@ -153,6 +156,20 @@ int gemm_grid(moe_plan_t p, int n_tiles_n) {
   int sms = p->num_sms;
   if (p->max_sms > 0 && p->max_sms < sms) sms = p->max_sms;
   return (int)(tiles < sms ? tiles : sms);
+}
+
+// CTA-pair GEMMs (M = 256 per pair) when experts average at least 256 rows, or when forced.
+bool use_pairs(moe_plan_t p) {
+  if (p->pair_mode == 0 || gemm_pair_max_clusters() < 1) return false;
+  return p->pair_mode == 2 || (long long)p->T * p->k >= 256ll * p->E;
+}
+
+int pair_grid(moe_plan_t p, int n_tiles_n) {
+  const long long pt_bound = (p->rows + 2 * kGemmBM - 1) / (2 * kGemmBM) + p->n;
+  long long tiles = pt_bound * n_tiles_n;
+  int pairs = gemm_pair_max_clusters();
+  if (p->max_sms > 0 && p->max_sms / 2 < pairs) pairs = p->max_sms / 2 > 0 ? p->max_sms / 2 : 1;
+  return (int)(tiles < pairs ? tiles : pairs);
 }
 
 // Record the event that closes phase `i` (event 0 opens the forward).
@@ -202,7 +219,8 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
   mark(p, 1 + MOE_PHASE_TOPK, s);
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
                                 region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
-                                at<int32_t>(p, p->off_mtile), p->T, p->E, p->k, p->shared, s)) != cudaSuccess)
+                                at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                p->shared, s)) != cudaSuccess)
     return cuda_rc(e);
   mark(p, 1 + MOE_PHASE_SCAN, s);
   e = launch_scatter_quant(x, ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
@@ -237,11 +255,24 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
   }
   mark(p, 1 + MOE_PHASE_PREPARE, s);
   GemmArgs a1 = gemm_args(p, 1);
-  if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
-  mark(p, 1 + MOE_PHASE_LINEAR1, s);
   GemmArgs a2 = gemm_args(p, 2);
-  if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess) return MOE_ERR_CUDA;
-  mark(p, 1 + MOE_PHASE_LINEAR2, s);
+  if (use_pairs(p)) {
+    if (launch_gemm_pair_linear1(p->amA1, p->tmB1, p->tmSfa1, p->tmSfb1, a1, pair_grid(p, a1.n_tiles_n), s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    mark(p, 1 + MOE_PHASE_LINEAR1, s);
+    if (launch_gemm_pair_linear2(p->amA2, p->tmB2p, p->tmSfa2, p->tmSfb2, a2, pair_grid(p, a2.n_tiles_n), s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    mark(p, 1 + MOE_PHASE_LINEAR2, s);
+  } else {
+    if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    mark(p, 1 + MOE_PHASE_LINEAR1, s);
+    if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    mark(p, 1 + MOE_PHASE_LINEAR2, s);
+  }
   cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
                                  region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
                                  p->shared, s);
@@ -347,6 +378,7 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_gcounts = add((size_t)p->G * E * 4);
   p->off_gbase = add((size_t)p->G * E * 4);
   p->off_mtile = add((size_t)(p->n + 1) * 4);
+  p->off_ptile = add((size_t)(p->n + 1) * 4);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
   p->off_whi = add((size_t)E * H * 2);
@@ -387,6 +419,10 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
     case MOE_OPT_PHASE_EVENTS:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->phase_events = (int)value;
+      return MOE_OK;
+    case MOE_OPT_PAIR_TILES:
+      if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+      p->pair_mode = (int)value;
       return MOE_OK;
     case MOE_OPT_SWAP_ROWS:
       if (value != 0 && value != 32 && value != 64) return MOE_ERR_INVALID_ARG;
@@ -440,6 +476,20 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   if (rc == MOE_OK)
     rc = encode_2d(&p->tmWlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, at<uint16_t>(p, p->off_wlo), p->H, p->E,
                    2ull * p->H, 64, 128);
+  // scale atoms (512 B) and weight scale units (1024 B) as rows of 256 bytes, no swizzle
+  struct SfMap {
+    CUtensorMap* m;
+    const void* base;
+    size_t bytes;
+    uint32_t box_rows;
+  } sf[4] = {{&p->tmSfa1, region<uint8_t>(p, MOE_REGION_XSF), p->region_len[MOE_REGION_XSF], 2},
+             {&p->tmSfa2, region<uint8_t>(p, MOE_REGION_HSF), p->region_len[MOE_REGION_HSF], 2},
+             {&p->tmSfb1, at<uint8_t>(p, p->off_w1sf), (size_t)p->n * (p->I / 128) * (p->H / 128) * 1024, 4},
+             {&p->tmSfb2, at<uint8_t>(p, p->off_w2sf),
+              (size_t)p->n * ((p->H + kGemmBN - 1) / kGemmBN) * (p->I / 128) * 1024, 4}};
+  for (int i = 0; i < 4 && rc == MOE_OK; ++i)
+    rc = encode_2d(sf[i].m, CU_TENSOR_MAP_DATA_TYPE_UINT8, sf[i].base, 256, sf[i].bytes / 256, 256, 256,
+                   sf[i].box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != MOE_OK) {
     p->ws = nullptr;
     return rc;
@@ -465,6 +515,9 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
   if (W2 != p->w2_cached) {
     rc = encode_2d(&p->tmB2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
                    128, 256);
+    if (rc == MOE_OK)
+      rc = encode_2d(&p->tmB2p, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
+                     128, 128);
     if (rc != MOE_OK) return rc;
     p->w2_cached = W2;
   }
@@ -519,7 +572,8 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
                                    region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), counts, offsets, at<int32_t>(p, p->off_gbase),
-                                at<int32_t>(p, p->off_mtile), p->T, p->E, p->k, p->shared, s)) != cudaSuccess)
+                                at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                p->shared, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
                            region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile), slot_pos,

@@ -381,12 +381,14 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
 // --------------------------------------------------------------------------- scan
 // One block.  counts[e] = sum over groups; offsets = exclusive scan over experts
 // (shared expert last, T rows); group_base[g][e] = offsets[e] + rows of e in
-// groups < g; mtile_start = exclusive scan of ceil(count/128).
+// groups < g; mtile_start = exclusive scan of ceil(count/128); ptile_start = exclusive scan of
+// ceil(ceil(count/128)/2) (row-tile pairs of the CTA-pair GEMM).
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __restrict__ group_counts,
                                                              int32_t* counts, int32_t* offsets,
-                                                             int32_t* group_base, int32_t* mtile_start, int T,
-                                                             int E, int k, int shared) {
-  __shared__ int32_t warp_sums[2][32];
+                                                             int32_t* group_base, int32_t* mtile_start,
+                                                             int32_t* ptile_start, int T, int E, int k,
+                                                             int shared) {
+  __shared__ int32_t warp_sums[3][32];
   const int G = (T + 31) / 32;
   const int n = E + shared;
   const int e = threadIdx.x;           // n <= 1025: thread 1024 never needed (E <= 1024, shared expert handled below)
@@ -398,38 +400,45 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
   }
   // block-wide exclusive scans of c and of ceil(c/128)
   int mt = (c + kGemmBM - 1) / kGemmBM;
+  int pt = (mt + 1) / 2;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-  int ic = c, im = mt;
+  int ic = c, im = mt, ip = pt;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int a = __shfl_up_sync(0xffffffffu, ic, off);
     const int b = __shfl_up_sync(0xffffffffu, im, off);
-    if (lane >= off) { ic += a; im += b; }
+    const int d = __shfl_up_sync(0xffffffffu, ip, off);
+    if (lane >= off) { ic += a; im += b; ip += d; }
   }
-  if (lane == 31) { warp_sums[0][warp] = ic; warp_sums[1][warp] = im; }
+  if (lane == 31) { warp_sums[0][warp] = ic; warp_sums[1][warp] = im; warp_sums[2][warp] = ip; }
   __syncthreads();
   if (warp == 0) {
-    int a = warp_sums[0][lane], b = warp_sums[1][lane];
+    int a = warp_sums[0][lane], b = warp_sums[1][lane], d = warp_sums[2][lane];
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int a2 = __shfl_up_sync(0xffffffffu, a, off);
       const int b2 = __shfl_up_sync(0xffffffffu, b, off);
-      if (lane >= off) { a += a2; b += b2; }
+      const int d2 = __shfl_up_sync(0xffffffffu, d, off);
+      if (lane >= off) { a += a2; b += b2; d += d2; }
     }
     warp_sums[0][lane] = a;
     warp_sums[1][lane] = b;
+    warp_sums[2][lane] = d;
   }
   __syncthreads();
   const int base_c = (warp > 0 ? warp_sums[0][warp - 1] : 0) + ic - c;
   const int base_m = (warp > 0 ? warp_sums[1][warp - 1] : 0) + im - mt;
+  const int base_p = (warp > 0 ? warp_sums[2][warp - 1] : 0) + ip - pt;
   if (e < n) {
     counts[e] = c;
     offsets[e] = base_c;
     mtile_start[e] = base_m;
+    ptile_start[e] = base_p;
   }
   if (e == n - 1) {
     offsets[n] = base_c + c;
     mtile_start[n] = base_m + mt;
+    ptile_start[n] = base_p + pt;
   }
   if (e < E) {
     int run = base_c;
@@ -665,9 +674,10 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
 }
 
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
-                                 int32_t* group_base, int32_t* mtile_start, int T, int E, int k, int shared,
-                                 cudaStream_t s) {
-  dispatch_scan_kernel<<<1, 1024, 0, s>>>(group_counts, counts, offsets, group_base, mtile_start, T, E, k, shared);
+                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
+                                 int k, int shared, cudaStream_t s) {
+  dispatch_scan_kernel<<<1, 1024, 0, s>>>(group_counts, counts, offsets, group_base, mtile_start, ptile_start, T,
+                                          E, k, shared);
   return cudaGetLastError();
 }
 

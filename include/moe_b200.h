@@ -91,11 +91,16 @@ enum moe_option {
                                   caller's stream is capturing or MOE_OPT_PHASE_EVENTS is
                                   1.  The CUDA runtime may reserve memory for the recorded
                                   graphs; changing any option drops them.  Default 0.    */
-  MOE_OPT_SWAP_ROWS = 8        /* grouped GEMM row tiles holding at most this many rows of
+  MOE_OPT_SWAP_ROWS = 8,       /* grouped GEMM row tiles holding at most this many rows of
                                   their expert (0, 32 or 64; default 0) are computed
                                   transposed: 128 weight rows as the MMA's M side and the
                                   tile's tokens as N = 32 or 64, so few-token experts do
-                                  not pay for 128-row MMAs.  0 = always 128 token rows.   */
+                                  not pay for 128-row MMAs.  0 = always 128 token rows.
+                                  Single-CTA grouped GEMM only.                           */
+  MOE_OPT_PAIR_TILES = 9       /* grouped GEMMs on CTA pairs (2-CTA clusters, one
+                                  M = 256 MMA across the pair, each CTA loading half of
+                                  the weight tile): 0 (default) = never, 1 = when the
+                                  experts average >= 256 rows (T*k >= 256*E), 2 = always */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -90,6 +90,10 @@ def test_options_and_unbound_plan(L):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, v) == 0
     for v in (-1, 16, 65, 128):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, v) == binding.MOE_ERR_INVALID_ARG
+    for v in (0, 1, 2):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_PAIR_TILES, v) == 0
+    for v in (-1, 3):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_PAIR_TILES, v) == binding.MOE_ERR_INVALID_ARG
     # no workspace bound yet: every compute entry point refuses before touching a device
     null = [None] * 9
     assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE

@@ -34,10 +34,12 @@ SMALL = {
 }
 
 
-def plan_for(w, swap_rows=None):
+def plan_for(w, swap_rows=None, pair_tiles=None):
     p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
     if swap_rows is not None:
         p.set_option(binding.MOE_OPT_SWAP_ROWS, swap_rows)
+    if pair_tiles is not None:
+        p.set_option(binding.MOE_OPT_PAIR_TILES, pair_tiles)
     return p
 
 
@@ -209,13 +211,14 @@ def test_forward_is_deterministic(cuda_lib):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_forward_all_tokens_on_one_expert(cuda_lib):
+@pytest.mark.parametrize("pair_tiles", [0, 2])
+def test_forward_all_tokens_on_one_expert(cuda_lib, pair_tiles):
     # the bias forces every token onto expert 2 (many row tiles for one expert, others empty)
     w = W("skew", T=700, H=256, I_=384, E=8, k=1, shared=1)
     case = make_case(w, seed=2, screened=False)
     case["bias"] = torch.tensor([0, 0, 50, 0, 0, 0, 0, 0], dtype=torch.float32)
     d = to_device(case)
-    p = plan_for(w)
+    p = plan_for(w, pair_tiles=pair_tiles)
     out = p.forward(**d)
     ref = oracle_forward(case, w)
     assert ref["counts"].tolist() == [0, 0, 700, 0, 0, 0, 0, 0, 700]
@@ -245,19 +248,39 @@ def _count_mix_case(counts, H=256, I_=384, seed=3):
     return w, case
 
 
-@pytest.mark.parametrize("swap_rows", [64, 32, 0])
-def test_forward_tile_row_boundaries(cuda_lib, swap_rows):
-    # expert loads on both sides of 32, 64 and 128 rows, plus an empty expert
-    counts = [1, 17, 32, 33, 64, 65, 128, 129, 0, 200]
+@pytest.mark.parametrize("swap_rows,pair_tiles", [(64, 0), (32, 0), (0, 0), (0, 2)])
+def test_forward_tile_row_boundaries(cuda_lib, swap_rows, pair_tiles):
+    # expert loads on both sides of 32, 64, 128 and 256 rows (odd and even row-tile counts for
+    # the CTA-pair GEMM), plus an empty expert
+    counts = [1, 17, 32, 33, 64, 65, 128, 129, 0, 200, 256, 257, 384]
     w, case = _count_mix_case(counts)
     d = to_device(case)
-    p = plan_for(w, swap_rows)
+    p = plan_for(w, swap_rows, pair_tiles)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
     ref = oracle_forward(case, w)
     assert ref["counts"].tolist() == counts + [w.T]
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
-    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows}")
+    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows} pair_tiles={pair_tiles}")
+
+
+# CTA-pair GEMMs forced on the small shapes (auto mode uses them from 256 rows per expert on)
+@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "k_eq_E", "tc_router"])
+def test_forward_pair_tiles_match_oracle(cuda_lib, name):
+    w = SMALL[name]
+    case = make_case(w, seed=11)
+    d = to_device(case)
+    p = plan_for(w, pair_tiles=2)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref = oracle_forward(case, w)
+    assert_output_close(bits(out), ref["y"], name + " pairs")
+    # the single-CTA kernel forms the same products; only the fp32 summation may differ
+    p1 = plan_for(w, pair_tiles=0)
+    out1 = p1.forward(**d)
+    a = F.bf16_to_f64(bits(out))
+    b = F.bf16_to_f64(bits(out1))
+    assert np.linalg.norm(a - b) <= 1e-3 * np.linalg.norm(b)
 
 
 def test_token_permutation_permutes_output(cuda_lib):
