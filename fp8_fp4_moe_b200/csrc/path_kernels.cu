@@ -300,14 +300,25 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
         int best_id = 0x7FFFFFFF;
         int free_id = 0x7FFFFFFF;   // lowest unselected id (fallback when every score is NaN)
         if (use_cache) {
+          // lane-local best (ids ascend with i, so a strict > keeps the lowest id), then two
+          // warp reductions: the largest order-preserving key of (score + 0), then the lowest
+          // id holding it.  Key 0 = no selectable score in this lane (NaN, -inf or taken).
+          int bi = -1;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int e = lane + 32 * i;
             if (e >= E || (taken & (1u << i))) continue;
             if (free_id == 0x7FFFFFFF) free_id = e;
-            const float b = cached[i];
-            if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
+            if (cached[i] > best) { best = cached[i]; bi = i; }
           }
+          uint32_t key = 0u;
+          if (bi >= 0) {
+            const uint32_t u = __float_as_uint(best + 0.0f);       // -0 and +0 compare equal
+            key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+          }
+          const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+          best_id = __reduce_min_sync(0xffffffffu, (key == kmax && bi >= 0) ? lane + 32 * bi : 0x7FFFFFFF);
+          if (kmax == 0u) best_id = __reduce_min_sync(0xffffffffu, free_id);
         } else {
           for (int i = 0, e = lane; e < E; ++i, e += 32) {
             if (taken & (1u << i)) continue;
@@ -316,14 +327,16 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
             if (b > best || (b == best && e < best_id)) { best = b; best_id = e; }
           }
         }
+        if (!use_cache) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-          const int oid = __shfl_xor_sync(0xffffffffu, best_id, off);
-          if (ob > best || (ob == best && oid < best_id)) { best = ob; best_id = oid; }
-          free_id = min(free_id, __shfl_xor_sync(0xffffffffu, free_id, off));
+          for (int off = 16; off > 0; off >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oid = __shfl_xor_sync(0xffffffffu, best_id, off);
+            if (ob > best || (ob == best && oid < best_id)) { best = ob; best_id = oid; }
+            free_id = min(free_id, __shfl_xor_sync(0xffffffffu, free_id, off));
+          }
+          if (best_id == 0x7FFFFFFF) best_id = free_id;   // k <= E guarantees free_id < E
         }
-        if (best_id == 0x7FFFFFFF) best_id = free_id;   // k <= E guarantees free_id < E
         if ((best_id & 31) == lane) taken |= 1u << (best_id >> 5);
         float s_best;
         if (use_cache) {               // the owner lane holds the unbiased score in registers
@@ -565,7 +578,9 @@ __global__ void __launch_bounds__(256) quant_tokens_kernel(const uint16_t* __res
 
 // --------------------------------------------------------------------------- combine
 // out[t] = bf16( sum_{j<k} gate[t][j] * row[slot_pos[t][j]] + shared * row[R + t] ),
-// fp32 accumulation in exactly that order (deterministic, no atomics).
+// fp32 accumulation in exactly that order (deterministic, no atomics).  KMAX >= k bounds
+// the rows a lane holds in registers (all loaded before the first is used).
+template <int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y,
                                                       const int32_t* __restrict__ slot_pos,
                                                       const float* __restrict__ gates, uint16_t* __restrict__ out,
@@ -590,21 +605,31 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const long r = __shfl_sync(0xffffffffu, my_row, j);
-      const float gj = __shfl_sync(0xffffffffu, my_gate, j);
-      if (!active) continue;
-      const uint4 raw = *reinterpret_cast<const uint4*>(y + r * H + c0);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    // all k (+1) rows are loaded before the first use; the sum keeps slot order
+    uint4 raw_j[KMAX];
+    float g_j[KMAX];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(gj, __uint_as_float(w[i] << 16), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(gj, __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+    for (int j = 0; j < KMAX; ++j) {
+      const long r = __shfl_sync(0xffffffffu, my_row, j);
+      g_j[j] = __shfl_sync(0xffffffffu, my_gate, j);
+      if (j < k && active) raw_j[j] = *reinterpret_cast<const uint4*>(y + r * H + c0);
+    }
+    uint4 raw_s = make_uint4(0, 0, 0, 0);
+    if (shared && active) raw_s = *reinterpret_cast<const uint4*>(y + (R + t) * H + c0);
+    if (!active) return;                 // no shuffles below
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        const uint32_t w[4] = {raw_j[j].x, raw_j[j].y, raw_j[j].z, raw_j[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(g_j[j], __uint_as_float(w[i] << 16), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(g_j[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+        }
       }
     }
-    if (!active) return;                 // no shuffles below
     if (shared) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(y + (R + t) * H + c0);
+      const uint4 raw = raw_s;
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -700,7 +725,11 @@ cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T
 cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,
                            int H, int k, int shared, cudaStream_t s) {
   const long items = (long)T * ((H + 255) / 256);
-  combine_kernel<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  const unsigned grid = (unsigned)((items + 7) / 8);
+  if (k <= 2) combine_kernel<2><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  else if (k <= 4) combine_kernel<4><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  else if (k <= 8) combine_kernel<8><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
+  else combine_kernel<16><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
   return cudaGetLastError();
 }
 

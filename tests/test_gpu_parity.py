@@ -94,6 +94,30 @@ def test_routing_exact_ties_lower_id(cuda_lib):
     assert r_ids[0].tolist() == [6, 0, 1]          # 0.75 > 0.5 == 0.5 (lower id first)
 
 
+def test_routing_nan_scores_are_never_preferred(cuda_lib):
+    # experts 0 and 3 score NaN for every token; tokens 0..4 score NaN everywhere and take the
+    # lowest ids (the oracle's stable sort places NaN last); other logits are exact dyadics
+    w = W("nan", T=40, H=256, I_=256, E=8, k=3)
+    x = torch.zeros(w.T, w.H, dtype=torch.bfloat16)
+    x[:, 0] = 1.0
+    x[:, 1] = torch.arange(w.T, dtype=torch.float32).remainder(4).to(torch.bfloat16)
+    x[:5, 2] = float("nan")
+    Wr = torch.zeros(w.E, w.H)
+    Wr[:, 0] = torch.tensor([0.0, 0.5, 0.25, 0.0, 0.125, 0.375, 0.0625, 0.75])
+    Wr[:, 1] = torch.tensor([0.0, 0.0, 0.125, 0.0, 0.25, 0.0, 0.5, 0.0])
+    Wr[:, 2] = 1.0
+    Wr[[0, 3], 3] = float("nan")
+    bias = torch.zeros(w.E)
+    p = plan_for(w)
+    ids, gates = p.debug_routing(x.cuda(), Wr.cuda(), bias.cuda())
+    r_ids, r_gates, _ = M.route(bits(x), Wr.numpy(), bias.numpy(), w.k)
+    ids = ids.cpu().numpy()
+    assert np.array_equal(ids, r_ids)
+    assert (ids[:5] == [0, 1, 2]).all()
+    assert not np.isin(ids[5:], [0, 3]).any()
+    np.testing.assert_allclose(gates.cpu().numpy()[5:], r_gates[5:], rtol=1e-6, atol=1e-7)
+
+
 # --------------------------------------------------------------------------- dispatch
 
 def _ids_case(T, E, k, kind, seed=0):
