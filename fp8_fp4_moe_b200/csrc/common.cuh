@@ -18,7 +18,7 @@ enum : int { kStatusTimeout = -4, kStatusBounds = -6 };
 enum : uint32_t {
   kWhereGemmProducer = 0x100, kWhereGemmSfLoader = 0x200, kWhereGemmMma = 0x300,
   kWhereGemmEpilogue = 0x400, kWhereGemmDrain = 0x500, kWhereRouterProducer = 0x600, kWhereRouterMma = 0x700,
-  kWhereRouterEpilogue = 0x800
+  kWhereRouterEpilogue = 0x800, kWhereGridBarrier = 0x900
 };
 
 __device__ __forceinline__ void report_status(uint32_t* status, int code, uint32_t where, uint32_t detail) {
@@ -36,6 +36,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Load through L2 only: for scheduling data that an earlier phase of the same kernel may
+// have written (the read-only path must not be used for it).
+__device__ __forceinline__ int ld_cg(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -43,6 +51,10 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Retire a barrier whose phases are all complete so its memory may be initialised again.
+__device__ __forceinline__ void mbar_inval(uint64_t* bar) {
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void fence_mbarrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

@@ -34,6 +34,7 @@
 // MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM, returns.
 #include "common.cuh"
 #include "kernels.h"
+#include "path_phases.cuh"
 
 namespace moe {
 
@@ -73,17 +74,17 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
   int lo = 0, hi = p.n_experts;
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
-    if (__ldg(p.mtile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
+    if (ld_cg(p.mtile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
   }
   TileCoord c;
   c.e = lo;
-  c.count = __ldg(p.counts + lo);
+  c.count = ld_cg(p.counts + lo);
   const int mtiles = (c.count + BM - 1) / BM;
-  const int mstart = __ldg(p.mtile_start + lo);
+  const int mstart = ld_cg(p.mtile_start + lo);
   const int local = tile - mstart * p.n_tiles_n;
   c.nt = local / mtiles;             // tiles of one expert: n-major, m fastest
   c.mt = local - c.nt * mtiles;
-  c.row0 = __ldg(p.offsets + lo) + c.mt * BM;
+  c.row0 = ld_cg(p.offsets + lo) + c.mt * BM;
   c.gmt = mstart + c.mt;
   c.rows = min(BM, c.count - c.mt * BM);
   return c;
@@ -350,13 +351,13 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord
   }
 }
 
+// One grouped GEMM over tiles cta, cta + n_ctas, ... by all kGemmThreads threads of the CTA,
+// with `tmem_base` holding 512 allocated TMEM columns and `smem` the 1024-aligned dynamic
+// shared memory.  Initialises its barriers on entry and invalidates them on exit, so the
+// same CTA may run it again (the single persistent forward runs linear1, then linear2).
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-byte alignment for the 128-byte-swizzled tiles
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& tmB, const GemmArgs& p,
+                                          uint8_t* smem, uint32_t tmem_base, int cta, int n_ctas) {
   uint8_t* a_s = smem + SmemLayout::a;
   uint8_t* b_s = smem + SmemLayout::b;
   uint8_t* sfa_s = smem + SmemLayout::sfa;
@@ -368,7 +369,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* accf = bars + 2 * S;      // [2] accumulator slot full
   uint64_t* acce = accf + 2;          // [2] accumulator slot empty
   uint64_t* drain = accf + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 4);
 
   const int warp = threadIdx.x / 32;
@@ -392,17 +392,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int i = 0; i < 4; ++i) tma_prefetch_desc(&tmA.m[i]);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
 
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-  const int total_tiles = __ldg(p.mtile_start + p.n_experts) * p.n_tiles_n;
+  const int total_tiles = ld_cg(p.mtile_start + p.n_experts) * p.n_tiles_n;
   const int KT = p.K / BK;
 
   if (warp == 0) {
@@ -414,8 +408,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      bool withhold = p.inject_fault != 0 && blockIdx.x == 0;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      bool withhold = p.inject_fault != 0 && cta == 0;
+      for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
         const TileCoord c = decode_tile(p, tile);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
@@ -462,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t uses0 = 0, uses1 = 0;      // completed uses of each accumulator slot
       int next_slot = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
         const TileCoord c = decode_tile(p, tile);
         const SlotPlan sp = plan_slots(p, c, next_slot);
         for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
@@ -521,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t uses0 = 0, uses1 = 0;
     int next_slot = 0;
     int buf = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = cta; tile < total_tiles; tile += n_ctas) {
       const TileCoord c = decode_tile(p, tile);
       const SlotPlan sp = plan_slots(p, c, next_slot);
       bool ok = true;
@@ -546,6 +540,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < (int)SmemLayout::n_bars; ++i) mbar_inval(bars + i);
+  }
+  __syncthreads();
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte-swizzled tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
+  const int warp = threadIdx.x / 32;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  gemm_body<MODE>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -586,18 +604,18 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const GemmArgs& p, int til
   int lo = 0, hi = p.n_experts;
   while (hi - lo > 1) {
     int mid = (lo + hi) >> 1;
-    if (__ldg(p.ptile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
+    if (ld_cg(p.ptile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
   }
   TileCoord c;
   c.e = lo;
-  c.count = __ldg(p.counts + lo);
+  c.count = ld_cg(p.counts + lo);
   const int mtiles = (c.count + BM - 1) / BM;
   const int ptiles = (mtiles + 1) / 2;
-  const int local = tile - __ldg(p.ptile_start + lo) * p.n_tiles_n;
+  const int local = tile - ld_cg(p.ptile_start + lo) * p.n_tiles_n;
   c.nt = local / ptiles;
   c.mt = 2 * (local - c.nt * ptiles) + rank;
-  c.row0 = __ldg(p.offsets + lo) + c.mt * BM;
-  c.gmt = __ldg(p.mtile_start + lo) + c.mt;
+  c.row0 = ld_cg(p.offsets + lo) + c.mt * BM;
+  c.gmt = ld_cg(p.mtile_start + lo) + c.mt;
   c.rows = max(0, min(BM, c.count - c.mt * BM));
   return c;
 }
@@ -659,7 +677,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
-  const int total_tiles = __ldg(p.ptile_start + p.n_experts) * p.n_tiles_n;
+  const int total_tiles = ld_cg(p.ptile_start + p.n_experts) * p.n_tiles_n;
   const int KT = p.K / BK;
 
   if (warp == 0) {
@@ -826,11 +844,13 @@ struct RouterSmem {
   static constexpr uint32_t total = misc + 16;
 };
 
-__global__ void __launch_bounds__(kRouterThreads, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
-                     const __grid_constant__ CUtensorMap tmWlo, const RouterArgs p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// One router tile (128 tokens from m0, 128 experts from n0, K split `split` of `n_splits`)
+// by all threads of the CTA; warps 0..5 work (TMA, MMA, 4 x epilogue), any others only join
+// the CTA barriers.  TMEM columns [tmem_base, tmem_base + 128) are the accumulator.
+// Initialises its barriers on entry and invalidates them on exit.
+__device__ __forceinline__ void router_tc_item(const CUtensorMap& tmX, const CUtensorMap& tmWhi,
+                                               const CUtensorMap& tmWlo, const RouterArgs& p, uint8_t* smem,
+                                               uint32_t tmem_base, int m0, int n0, int split, int n_splits) {
   uint8_t* a_s = smem + RouterSmem::a;
   uint8_t* bh_s = smem + RouterSmem::bh;
   uint8_t* bl_s = smem + RouterSmem::bl;
@@ -838,14 +858,12 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   uint64_t* empty = full + RS;
   uint64_t* accf = full + 2 * RS;
   uint64_t* drain = accf + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RouterSmem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + RouterSmem::misc + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * RBN;
-  // K split blockIdx.z of gridDim.z: stages [kt0, kt0 + KT), partial logits in slice blockIdx.z
-  const int KT = p.H / RBK / (int)gridDim.z;
-  const int kt0 = (int)blockIdx.z * KT;
-  float* const logits = p.logits + (long)blockIdx.z * p.T * p.E;
+  // stages [kt0, kt0 + KT) of this split; partial logits in slice `split`
+  const int KT = p.H / RBK / n_splits;
+  const int kt0 = split * KT;
+  float* const logits = p.logits + (long)split * p.T * p.E;
   if (threadIdx.x == 0) {
     for (int s = 0; s < RS; ++s) {
       mbar_init(&full[s], 1);
@@ -856,14 +874,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
-    tmem_relinquish();
-    tc_fence_before();
-  }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (warp == 0) {
     if (lane == 0) {
@@ -912,7 +924,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       tc_commit(drain);
       if (!mbar_wait_drain(drain, 0, p.timeout_ns)) report_status(p.status, kStatusTimeout, kWhereGemmDrain, 0x29);
     }
-  } else {
+  } else if (warp < kRouterThreads / 32) {
     const int q = warp & 3;
     const bool ok = mbar_wait(accf, 0, ctl, kWhereRouterEpilogue);
     if (__all_sync(0xffffffffu, ok)) {
@@ -944,6 +956,28 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * RS + 2; ++i) mbar_inval(full + i);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
+                     const __grid_constant__ CUtensorMap tmWlo, const RouterArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RouterSmem::misc);
+  const int warp = threadIdx.x / 32;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  router_tc_item(tmX, tmWhi, tmWlo, p, smem, tmem_base, blockIdx.y * 128, blockIdx.x * RBN, blockIdx.z, gridDim.z);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 128);
@@ -958,6 +992,140 @@ __global__ void split_router_weights_kernel(const float* __restrict__ W, __nv_bf
     const __nv_bfloat16 h = __float2bfloat16_rn(w);
     hi[i] = h;
     lo[i] = __float2bfloat16_rn(w - __bfloat162float(h));
+  }
+}
+
+// ------------------------------------------------------------------ the single persistent forward
+// Shared memory of the fused kernel: the largest step layout, then the kernel-lifetime words.
+constexpr uint32_t kFusedMiscOffset = (SmemLayout::total + 15) & ~15u;
+static_assert(kFusedMiscOffset >= RouterSmem::total && kFusedMiscOffset >= sizeof(TopkSmem),
+              "every step's shared memory must fit below the fused kernel's own words");
+// Grid-wide barrier for a cooperative launch: bar[0] counts arrivals, bar[1] is the
+// generation the last arrival advances.  The wait is bounded; on expiry the CTA records
+// MOE_ERR_DEVICE_TIMEOUT and the barrier reports false.  All threads call it.
+__device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32_t* status, uint64_t timeout_ns,
+                                          volatile int* ok_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    __threadfence();
+    const uint32_t gen = atomicAdd(&bar[1], 0u);
+    if (atomicAdd(&bar[0], 1u) == n_ctas - 1) {
+      atomicExch(&bar[0], 0u);
+      __threadfence();
+      atomicAdd(&bar[1], 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (atomicAdd(&bar[1], 0u) == gen) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
+          report_status(status, kStatusTimeout, kWhereGridBarrier, gen);
+          ok = false;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    *ok_smem = ok && *reinterpret_cast<volatile uint32_t*>(status) == 0u;
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
+// Generic-proxy stores made visible to later TMA (async-proxy) reads of the same data.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    fused_forward_kernel(const __grid_constant__ AMaps amA1, const __grid_constant__ AMaps amA2,
+                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                         const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
+                         const __grid_constant__ CUtensorMap tmWlo, const FusedArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // kernel-lifetime words past every step's own layout
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kFusedMiscOffset);
+  volatile int* ok_smem = reinterpret_cast<volatile int*>(smem + kFusedMiscOffset + 8);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  (void)lane;
+  constexpr int NW = kGemmThreads / 32;
+  const int cta = blockIdx.x, n_ctas = gridDim.x;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long wstride = (long)n_ctas * NW, wfirst = (long)cta * NW + warp;
+  const int G = (a.T + 31) / 32;
+
+  bool ok = true;
+  // S1 router
+  if (a.router_kind == kRouterTensor) {
+    const int mt = (a.T + 127) / 128, nt = (a.E + RBN - 1) / RBN;
+    for (int it = cta; it < mt * nt * a.router_parts; it += n_ctas) {
+      const int split = it % a.router_parts, tile = it / a.router_parts;
+      router_tc_item(tmX, tmWhi, tmWlo, a.ra, smem, tmem_base, (tile / nt) * 128, (tile % nt) * RBN, split,
+                     a.router_parts);
+    }
+  } else if (a.router_kind == kRouterSplitBlock) {
+    float* part = reinterpret_cast<float*>(smem);
+    for (int it = cta; it < a.E * a.T; it += n_ctas)
+      router_split_block<kGemmThreads>(a.x, a.W_router, a.logits, a.T, a.H, a.E, it % a.E, it / a.E, part);
+  } else if (a.router_kind == kRouterWarp8) {
+    router_warp_items<8>(a.x, a.W_router, a.logits, a.T, a.H, a.E, wfirst, wstride);
+  } else {
+    router_warp_items<2>(a.x, a.W_router, a.logits, a.T, a.H, a.E, wfirst, wstride);
+  }
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem);
+  // S2 top-k, gates, ranks inside each group of 32 tokens
+  if (ok) {
+    TopkSmem& tsm = *reinterpret_cast<TopkSmem*>(smem);
+    for (int g = cta; g < G; g += n_ctas)
+      topk_rank_group<kGemmThreads>(g, 0, a.logits, a.router_parts, a.bias, a.topk_ids, a.gates, a.local_rank,
+                                    a.group_counts, a.status, a.T, a.E, a.k, tsm);
+  }
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  // S3 dispatch: per-expert group scan, expert scan, then scatter + quantisation
+  if (ok)
+    for (long e = wfirst; e < a.E; e += wstride) column_scan_warp((int)e, a.group_counts, a.group_base, a.counts, G, a.E);
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  if (ok && cta == 0)
+    expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.T, a.E, a.shared,
+                                    reinterpret_cast<int32_t(*)[32]>(smem));
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  if (ok) {
+    const long items = (long)a.T * ((a.H + 255) / 256);
+    for (long it = wfirst; it < items; it += wstride)
+      scatter_item(it, a.x, a.topk_ids, a.local_rank, a.group_base, a.offsets, a.mtile_start, a.slot_pos, a.perm,
+                   a.xq, a.xsf, a.T, a.H, a.E, a.k, a.shared);
+  }
+  fence_proxy_async_global();
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  // S4 linear1 + SwiGLU + requantisation
+  if (ok) gemm_body<1>(amA1, tmB1, a.g1, smem, tmem_base, cta, n_ctas);
+  fence_proxy_async_global();
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  // S5 linear2
+  if (ok) gemm_body<2>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
+  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  // S6 combine
+  if (ok) {
+    const long items = (long)a.T * ((a.H + 255) / 256);
+    for (long it = wfirst; it < items; it += wstride) {
+      if (a.k <= 2) combine_item<2>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
+      else if (a.k <= 4) combine_item<4>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
+      else if (a.k <= 8) combine_item<8>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
+      else combine_item<16>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -991,6 +1159,8 @@ cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* 
 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
 size_t gemm_pair_smem_bytes() { return PairSmem::total + 1024; }
+size_t fused_smem_bytes() { return kFusedMiscOffset + 16 + 1024; }
+int g_fused_ctas[64] = {};
 int g_pair_clusters[64] = {};
 
 cudaError_t gemm_prepare_device() {
@@ -1028,7 +1198,34 @@ cudaError_t gemm_prepare_device() {
   e = cudaOccupancyMaxActiveClusters(&clusters, (const void*)grouped_gemm_pair_kernel<1>, &cfg);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64) g_pair_clusters[dev] = clusters;
+  // the fused forward: one CTA per SM, all co-resident (cooperative launch)
+  e = cudaFuncSetAttribute(fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes());
+  if (e != cudaSuccess) return e;
+  int per_sm = 0, sms = 0, coop = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_forward_kernel, kGemmThreads,
+                                                         fused_smem_bytes())) != cudaSuccess)
+    return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) g_fused_ctas[dev] = coop ? per_sm * sms : 0;
   return cudaSuccess;
+}
+
+int fused_max_ctas() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  return g_fused_ctas[dev];
+}
+
+cudaError_t launch_fused_forward(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
+                                 const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
+                                 const FusedArgs& args, int ctas, cudaStream_t s) {
+  if (ctas < 1 || ctas > fused_max_ctas()) return cudaErrorInvalidValue;
+  void* params[] = {const_cast<AMaps*>(&a1), const_cast<AMaps*>(&a2), const_cast<CUtensorMap*>(&b1),
+                    const_cast<CUtensorMap*>(&b2), const_cast<CUtensorMap*>(&x), const_cast<CUtensorMap*>(&whi),
+                    const_cast<CUtensorMap*>(&wlo), const_cast<FusedArgs*>(&args)};
+  return cudaLaunchCooperativeKernel((const void*)fused_forward_kernel, dim3(ctas), dim3(kGemmThreads), params,
+                                    fused_smem_bytes(), s);
 }
 
 int gemm_pair_max_clusters() {

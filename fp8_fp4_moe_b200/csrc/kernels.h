@@ -86,6 +86,45 @@ cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const
 // W fp32 [n] -> hi = bf16(W), lo = bf16(W - hi)
 cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* lo, long n, cudaStream_t s);
 
+// ---- the single persistent forward (gemm_sm100.cu) -------------------------------
+// Every step of the forward in one cooperative launch of one CTA per SM (kGemmThreads
+// threads), the steps separated by grid-wide barriers: router, top-k + rank, per-expert
+// group scan, expert scan, dispatch + quantisation, linear1, linear2, combine.
+enum : int { kRouterSplitBlock = 0, kRouterWarp8 = 1, kRouterWarp2 = 2, kRouterTensor = 3 };
+struct FusedArgs {
+  int T, H, E, k, shared;
+  int router_kind;                 // kRouter*
+  int router_parts;                // partial logit arrays (tensor-core router K splits)
+  const uint16_t* x;
+  const float* W_router;
+  const float* bias;
+  float* logits;
+  int32_t* topk_ids;
+  float* gates;
+  int32_t* local_rank;
+  int32_t* group_counts;
+  int32_t* group_base;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile_start;
+  int32_t* ptile_start;
+  int32_t* slot_pos;
+  int32_t* perm;
+  uint8_t* xq;
+  uint8_t* xsf;
+  const uint16_t* y;
+  uint16_t* out;
+  uint32_t* status;
+  uint32_t* gridbar;               // [2] arrival count, generation (zeroed once per workspace)
+  uint64_t timeout_ns;
+  RouterArgs ra;
+  GemmArgs g1, g2;
+};
+cudaError_t launch_fused_forward(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
+                                 const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
+                                 const FusedArgs& args, int ctas, cudaStream_t s);
+int fused_max_ctas();                // co-resident CTAs of the fused kernel (after gemm_prepare_device)
+
 // ---- routing / dispatch / combine (path_kernels.cu) -----------------------------
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
                                  cudaStream_t s);
@@ -98,6 +137,8 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
                              float* gates,
                              int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
                              cudaStream_t s);
+// counts, offsets, mtile_start, ptile_start (n + 1 entries) and group_base[g][e] = rows of
+// expert e in token groups < g (relative to offsets[e]).
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
                                  int k, int shared, cudaStream_t s);

@@ -29,11 +29,13 @@ struct moe_plan_s {
   int router_tc = 1;
   int swap_rows = 0;
   int pair_mode = 0;                // MOE_OPT_PAIR_TILES
+  int fused = 0;                    // MOE_OPT_FUSED
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
   size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_ptile, off_w1sf, off_w2sf, off_whi, off_wlo;
+  size_t off_gridbar;               // grid barrier words of the fused forward
   long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
   // bound state
@@ -245,9 +247,75 @@ int prepare_weights(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_sc
   return MOE_OK;
 }
 
+// MOE_OPT_FUSED: weight preparation when needed, then every step in one cooperative launch.
+int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias,
+                 const uint8_t* W1_scales, const uint8_t* W2_scales, void* out, cudaStream_t s) {
+  const bool tc = use_tc_router(p);
+  mark(p, 0, s);
+  if (tc) {
+    if (!p->static_weights || W_router != p->wr_prepared) {
+      if (launch_split_router_weights(W_router, at<uint16_t>(p, p->off_whi), at<uint16_t>(p, p->off_wlo),
+                                      (long)p->E * p->H, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      p->wr_prepared = W_router;
+    }
+    if (x != p->x_cached) {
+      int rc = encode_2d(&p->tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, p->H, p->T, 2ull * p->H, 64, 128);
+      if (rc != MOE_OK) return rc;
+      p->x_cached = x;
+    }
+  }
+  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
+    int rc = prepare_weights(p, W1_scales, W2_scales, s);
+    if (rc != MOE_OK) return rc;
+  }
+  FusedArgs a{};
+  a.T = p->T; a.H = p->H; a.E = p->E; a.k = p->k; a.shared = p->shared;
+  a.router_kind = tc ? kRouterTensor
+                     : (long long)p->T * p->E <= 4096 ? kRouterSplitBlock : p->E <= 32 ? kRouterWarp8 : kRouterWarp2;
+  a.router_parts = tc ? p->router_splits : 1;
+  a.x = x;
+  a.W_router = W_router;
+  a.bias = bias;
+  a.logits = at<float>(p, p->off_logits);
+  a.topk_ids = region<int32_t>(p, MOE_REGION_TOPK_IDS);
+  a.gates = region<float>(p, MOE_REGION_GATES);
+  a.local_rank = at<int32_t>(p, p->off_rank);
+  a.group_counts = at<int32_t>(p, p->off_gcounts);
+  a.group_base = at<int32_t>(p, p->off_gbase);
+  a.counts = region<int32_t>(p, MOE_REGION_COUNTS);
+  a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
+  a.mtile_start = at<int32_t>(p, p->off_mtile);
+  a.ptile_start = at<int32_t>(p, p->off_ptile);
+  a.slot_pos = region<int32_t>(p, MOE_REGION_SLOT_POS);
+  a.perm = region<int32_t>(p, MOE_REGION_PERM);
+  a.xq = region<uint8_t>(p, MOE_REGION_XQ);
+  a.xsf = region<uint8_t>(p, MOE_REGION_XSF);
+  a.y = region<uint16_t>(p, MOE_REGION_Y);
+  a.out = static_cast<uint16_t*>(out);
+  a.status = region<uint32_t>(p, MOE_REGION_STATUS);
+  a.gridbar = at<uint32_t>(p, p->off_gridbar);
+  a.timeout_ns = p->timeout_ns;
+  a.ra = RouterArgs{p->T, p->H, p->E, a.router_parts, a.logits, a.status, p->timeout_ns};
+  a.g1 = gemm_args(p, 1);
+  a.g2 = gemm_args(p, 2);
+  int ctas = fused_max_ctas();
+  if (p->max_sms > 0 && p->max_sms < ctas) ctas = p->max_sms;
+  // a launch that ran out of time may have left arrivals behind
+  if (cudaMemsetAsync(a.gridbar, 0, 8, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, p->tmB2, p->tmX, p->tmWhi, p->tmWlo, a, ctas, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  // one kernel: its whole time is reported under the first phase
+  for (int i = 1; i <= MOE_PHASE_COUNT_; ++i) mark(p, i, s);
+  if (p->phase_events && p->events_ready) p->events_recorded = true;
+  return MOE_OK;
+}
+
 // The forward's launch sequence on stream s (TMA maps already current).
 int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias,
                    const uint8_t* W1_scales, const uint8_t* W2_scales, void* out, cudaStream_t s) {
+  if (p->fused) return launch_fused(p, x, W_router, bias, W1_scales, W2_scales, out, s);
   int rc = run_front(p, x, W_router, bias, s);
   if (rc != MOE_OK) return rc;
   if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
@@ -379,6 +447,7 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_gbase = add((size_t)p->G * E * 4);
   p->off_mtile = add((size_t)(p->n + 1) * 4);
   p->off_ptile = add((size_t)(p->n + 1) * 4);
+  p->off_gridbar = add(8);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
   p->off_whi = add((size_t)E * H * 2);
@@ -419,6 +488,11 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
     case MOE_OPT_PHASE_EVENTS:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       p->phase_events = (int)value;
+      return MOE_OK;
+    case MOE_OPT_FUSED:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      if (value == 1 && p->ws && fused_max_ctas() < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+      p->fused = (int)value;
       return MOE_OK;
     case MOE_OPT_PAIR_TILES:
       if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
@@ -495,6 +569,7 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
     return rc;
   }
   if (cudaMemset(region<uint32_t>(p, MOE_REGION_STATUS), 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(at<uint32_t>(p, p->off_gridbar), 0, 8) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -526,7 +601,7 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
       if (cudaEventCreate(&p->ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
     p->events_ready = true;
   }
-  if (p->use_graph && !p->phase_events) {
+  if (p->use_graph && !p->phase_events && !p->fused) {
     cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &st) != cudaSuccess) return MOE_ERR_CUDA;
     if (st == cudaStreamCaptureStatusNone) return forward_graph(p, x, W_router, bias, W1, W1_scales, W2, W2_scales,
@@ -575,9 +650,10 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
                                 at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
                                 p->shared, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
-                           region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile), slot_pos,
-                           perm, nullptr, nullptr, p->T, p->H, p->E, p->k, p->shared, s);
+  // positions = offsets (written just above into the caller's buffer) + group base + rank
+  e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase), offsets,
+                           at<int32_t>(p, p->off_mtile), slot_pos, perm, nullptr, nullptr, p->T, p->H, p->E, p->k,
+                           p->shared, s);
   return cuda_rc(e);
 }
 

@@ -97,10 +97,20 @@ enum moe_option {
                                   tile's tokens as N = 32 or 64, so few-token experts do
                                   not pay for 128-row MMAs.  0 = always 128 token rows.
                                   Single-CTA grouped GEMM only.                           */
-  MOE_OPT_PAIR_TILES = 9       /* grouped GEMMs on CTA pairs (2-CTA clusters, one
+  MOE_OPT_PAIR_TILES = 9,      /* grouped GEMMs on CTA pairs (2-CTA clusters, one
                                   M = 256 MMA across the pair, each CTA loading half of
                                   the weight tile): 0 (default) = never, 1 = when the
                                   experts average >= 256 rows (T*k >= 256*E), 2 = always */
+  MOE_OPT_FUSED = 10           /* 1 = moe_forward runs every step (router, top-k, dispatch
+                                  scans, scatter + quantisation, linear1, linear2, combine)
+                                  in ONE persistent cooperative kernel, one CTA per SM,
+                                  the steps separated by grid-wide barriers (bounded
+                                  waits); weight preparation, when needed, runs before it.
+                                  Router: tensor cores when MOE_OPT_ROUTER_TC applies,
+                                  else CUDA cores (block per expert and token for
+                                  T*E <= 4096, warp per token and expert chunk otherwise).
+                                  moe_phase_times reports the whole kernel under the router
+                                  phase.  No CUDA graph is recorded.  Default 0.          */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -34,12 +34,14 @@ SMALL = {
 }
 
 
-def plan_for(w, swap_rows=None, pair_tiles=None):
+def plan_for(w, swap_rows=None, pair_tiles=None, fused=None):
     p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
     if swap_rows is not None:
         p.set_option(binding.MOE_OPT_SWAP_ROWS, swap_rows)
     if pair_tiles is not None:
         p.set_option(binding.MOE_OPT_PAIR_TILES, pair_tiles)
+    if fused is not None:
+        p.set_option(binding.MOE_OPT_FUSED, fused)
     return p
 
 
@@ -272,20 +274,21 @@ def _count_mix_case(counts, H=256, I_=384, seed=3):
     return w, case
 
 
-@pytest.mark.parametrize("swap_rows,pair_tiles", [(64, 0), (32, 0), (0, 0), (0, 2)])
-def test_forward_tile_row_boundaries(cuda_lib, swap_rows, pair_tiles):
+@pytest.mark.parametrize("swap_rows,pair_tiles,fused", [(64, 0, 0), (32, 0, 0), (0, 0, 0), (0, 2, 0), (0, 0, 1),
+                                                        (64, 0, 1)])
+def test_forward_tile_row_boundaries(cuda_lib, swap_rows, pair_tiles, fused):
     # expert loads on both sides of 32, 64, 128 and 256 rows (odd and even row-tile counts for
     # the CTA-pair GEMM), plus an empty expert
     counts = [1, 17, 32, 33, 64, 65, 128, 129, 0, 200, 256, 257, 384]
     w, case = _count_mix_case(counts)
     d = to_device(case)
-    p = plan_for(w, swap_rows, pair_tiles)
+    p = plan_for(w, swap_rows, pair_tiles, fused)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
     ref = oracle_forward(case, w)
     assert ref["counts"].tolist() == counts + [w.T]
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
-    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows} pair_tiles={pair_tiles}")
+    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows} pair_tiles={pair_tiles} fused={fused}")
 
 
 # CTA-pair GEMMs forced on the small shapes (auto mode uses them from 256 rows per expert on)
@@ -305,6 +308,47 @@ def test_forward_pair_tiles_match_oracle(cuda_lib, name):
     a = F.bf16_to_f64(bits(out))
     b = F.bf16_to_f64(bits(out1))
     assert np.linalg.norm(a - b) <= 1e-3 * np.linalg.norm(b)
+
+
+# every step in one persistent cooperative kernel: each router variant (tensor cores for
+# tc_router, block per expert and token for tiny / t1_k1 / k_eq_E, warp per token and expert
+# chunk for ragged_shared / dsv3_like), routing and dispatch bit-exact, outputs in tolerance
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_fused_matches_oracle(cuda_lib, name):
+    w = SMALL[name]
+    case = make_case(w, seed=13)
+    d = to_device(case)
+    p = plan_for(w, fused=1)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref = oracle_forward(case, w)
+    assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
+    assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
+    assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
+    assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
+    np.testing.assert_allclose(p.region("gates").cpu().numpy(), ref["gates"], rtol=GATE_RTOL, atol=GATE_ATOL)
+    assert_output_close(bits(out), ref["y"], name + " fused")
+    # repeated launches reuse the grid barrier words
+    out2 = p.forward(**d).clone()
+    assert p.check_status()[0] == 0
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+
+
+def test_fused_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    w = SMALL["tiny"]
+    case = make_case(w, seed=1)
+    d = to_device(case)
+    p = plan_for(w, fused=1)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 50_000_000)      # 50 ms
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 1)             # one stage of linear1 never arrives
+    p.forward(**d)
+    code, _ = p.check_status()
+    assert code == binding.MOE_ERR_DEVICE_TIMEOUT
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 0)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 2_000_000_000)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    assert_output_close(bits(out), oracle_forward(case, w)["y"], "fused after timeout")
 
 
 def test_token_permutation_permutes_output(cuda_lib):
