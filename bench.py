@@ -43,6 +43,9 @@ REF_STEP_TOKENS = {"tiny": 64, "mixtral": 1, "dsv3_t1": 1, "dsv3_t512": 1, "dsv3
                    "dsv3_t32768": 1}
 
 
+KERNELS_PER_FORWARD = 8
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -80,7 +83,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("gemm_sm100.cu", "common.cuh", "path_kernels.cu"):
+    for name in ("gemm_sm100.cu", "common.cuh", "path_kernels.cu", "path_phases.cuh"):
         with open(os.path.join(ROOT, "fp8_fp4_moe_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -437,8 +440,9 @@ def run_cuda(args, rank, world, local_rank):
         "config": {"workload": w.description + ("" if not resized else f" (resized to T={w.T}, E={w.E})"),
                    "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
                    "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
-                   "launch": "kernels launched one by one" if args.no_graph else
-                             "CUDA graph replay of the 7 kernels (MOE_OPT_GRAPH)",
+                   "launch": ("one persistent cooperative kernel (MOE_OPT_FUSED)" if fused else
+                              "kernels launched one by one" if args.no_graph else
+                              f"CUDA graph replay of the {KERNELS_PER_FORWARD} kernels (MOE_OPT_GRAPH)"),
                    "phase_times": "separate pass, CUDA events between kernels, 20 steps",
                    "weight_scales": f"re-laid out once before timing ({prepare_ms:.3f} ms), reused "
                                     "(MOE_OPT_STATIC_WEIGHTS)",
@@ -453,7 +457,9 @@ def run_cuda(args, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 7 * args.steps,  # prepare is skipped: weights static
+        # router, top-k, column scan, expert scan, scatter, linear1, linear2, combine (prepare is
+        # skipped: weights static); the fused option is one kernel
+        "gpu_launches": (1 if fused else KERNELS_PER_FORWARD) * args.steps,
         "clocks": clocks,
         "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
     }
