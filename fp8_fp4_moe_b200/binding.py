@@ -45,6 +45,7 @@ EXPORTED = [
     "moe_plan", "moe_plan_set_option", "moe_workspace_bytes", "moe_set_workspace", "moe_workspace_region",
     "moe_forward", "moe_debug_routing", "moe_debug_dispatch", "moe_debug_quant_x", "moe_check_status",
     "moe_plan_destroy", "moe_error_string", "moe_phase_times", "moe_prepare_weights", "moe_route_noalloc",
+    "moe_update_bias", "moe_gemm_workspace_bytes", "moe_gemm_fp8_fp4",
 ]
 
 _lib = None
@@ -91,6 +92,12 @@ def lib() -> ctypes.CDLL:
     L.moe_prepare_weights.restype = i32
     L.moe_phase_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i32]
     L.moe_phase_times.restype = i32
+    L.moe_gemm_workspace_bytes.argtypes = [i32, i32, i32]
+    L.moe_gemm_workspace_bytes.restype = sz
+    L.moe_gemm_fp8_fp4.argtypes = [i32, i32, i32] + [vp] * 6 + [sz, vp]
+    L.moe_gemm_fp8_fp4.restype = i32
+    L.moe_update_bias.argtypes = [vp, vp, ctypes.c_float, vp]
+    L.moe_update_bias.restype = i32
     L.moe_plan_destroy.argtypes = [vp]
     L.moe_plan_destroy.restype = None
     L.moe_error_string.argtypes = [i32]
@@ -125,6 +132,32 @@ def _stream_ptr(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def gemm_fp8_fp4(A, A_scales, B, B_scales, out=None, workspace=None, stream=None):
+    """Dense block-scaled GEMM through moe_gemm_fp8_fp4: out [M, N] bf16 = A . B^T with
+    A E4M3 codes [M, K] (uint8) and UE8M0 scales [M, K/128], B packed E2M1 [N, K/2] and
+    UE8M0 scales [N, K/32].  Returns (out, workspace); the first int32 of the workspace is
+    the device status once the stream has run the call."""
+    M, K = A.shape
+    N = B.shape[0]
+    d = A.device
+    L = lib()
+    need = L.moe_gemm_workspace_bytes(M, N, K)
+    if need == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_gemm_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=d)
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=d)
+    for t, n in ((A_scales, (M, K // 128)), (B, (N, K // 2)), (B_scales, (N, K // 32))):
+        if tuple(t.shape) != n:
+            raise ValueError(f"expected shape {n}, got {tuple(t.shape)}")
+    _check(L.moe_gemm_fp8_fp4(M, N, K, _ptr(A, torch.uint8, d), _ptr(A_scales, torch.uint8, d),
+                              _ptr(B, torch.uint8, d), _ptr(B_scales, torch.uint8, d),
+                              _ptr(out, torch.bfloat16, d), _ptr(workspace, torch.uint8, d), workspace.numel(),
+                              _stream_ptr(stream)), "moe_gemm_fp8_fp4")
+    return out, workspace
 
 
 def route_noalloc(x, W_router, bias, k: int, topk_ids=None, gates=None, stream=None):
@@ -236,6 +269,14 @@ class Plan:
         if n < 0:
             raise MoeError(n, "moe_phase_times")
         return dict(zip(PHASES, list(buf)[:n]))
+
+    def update_bias(self, bias, gamma: float, stream=None):
+        """bias (device fp32 [E]) += gamma * sign(mean load - load), from the last forward's counts."""
+        if bias.numel() != self.E:
+            raise ValueError(f"bias has {bias.numel()} entries, the plan has {self.E} routed experts")
+        _check(lib().moe_update_bias(self._h, _ptr(bias, torch.float32, self.device), ctypes.c_float(gamma),
+                                     _stream_ptr(stream)), "moe_update_bias")
+        return bias
 
     def check_status(self, stream=None):
         detail = (ctypes.c_uint32 * 4)()

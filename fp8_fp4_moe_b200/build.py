@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["gemm_sm100.cu", "path_kernels.cu", "moe_api.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+SOURCES = ["gemm_sm100.cu", "path_kernels.cu", "moe_api.cu", "noalloc.cu", "dense_api.cu"]
+HEADERS = ["common.cuh", "kernels.h", "path_phases.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

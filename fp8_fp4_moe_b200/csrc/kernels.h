@@ -7,6 +7,12 @@
 
 namespace moe {
 
+// 2-D tiled tensor map (cuTensorMapEncodeTiled through the runtime's driver entry point):
+// dims {inner, outer}, row pitch in bytes, box {box_inner, box_outer}.  MOE_OK or MOE_ERR_CUDA.
+int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
+
 // ---- grouped block-scaled GEMMs (gemm_sm100.cu) --------------------------------
 constexpr int kGemmBM = 128;      // rows (tokens) per tile
 constexpr int kGemmBN = 256;      // accumulator columns per tile
@@ -149,6 +155,9 @@ cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, con
                                  int k, int shared, cudaStream_t s);
 // Token-order quantisation (debug entry point).
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s);
+// Auxiliary-loss-free balancing step from the routed experts' loads.
+cudaError_t launch_update_bias(float* bias, const int32_t* counts, int T, int k, int E, float gamma,
+                               cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const float* gates, uint16_t* out, int T,
                            int H, int k, int shared, cudaStream_t s);
 

@@ -6,6 +6,7 @@
 //   -> grouped GEMM linear1 (+SwiGLU +E4M3 requant) -> grouped GEMM linear2 -> combine
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -67,8 +68,9 @@ struct moe_plan_s {
   cudaEvent_t ev[MOE_PHASE_COUNT_ + 1];
 };
 
-namespace {
+namespace moe {
 
+namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -82,10 +84,10 @@ int get_encode() {
   });
   return g_encode ? MOE_OK : MOE_ERR_CUDA;
 }
+}  // namespace
 
 int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
   if (get_encode() != MOE_OK) return MOE_ERR_CUDA;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
@@ -95,6 +97,10 @@ int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
                         swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
+
+}  // namespace moe
+
+namespace {
 
 bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -632,6 +638,14 @@ int moe_debug_routing(moe_plan_t p, const void* x, const float* W_router, const 
                                    at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
                                    region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   return cuda_rc(e);
+}
+
+int moe_update_bias(moe_plan_t p, float* bias, float gamma, void* stream) {
+  int rc = check_bound(p);
+  if (rc != MOE_OK) return rc;
+  if (!aligned(bias, 4) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_update_bias(bias, region<int32_t>(p, MOE_REGION_COUNTS), p->T, p->k, p->E, gamma,
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, int32_t* offsets, int32_t* perm,

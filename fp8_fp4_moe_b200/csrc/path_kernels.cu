@@ -233,7 +233,25 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   combine_item<KMAX>((long)blockIdx.x * 8 + threadIdx.x / 32, y, slot_pos, gates, out, T, H, k, shared);
 }
 
+// --------------------------------------------------------------------------- bias update
+// bias[e] += gamma * sign(T*k - counts[e]*E): an over-used expert (more rows than the mean
+// load T*k/E) loses gamma, an under-used one gains it, one at the mean keeps its bias.
+__global__ void __launch_bounds__(256) update_bias_kernel(float* bias, const int32_t* __restrict__ counts, int T,
+                                                          int k, int E, float gamma) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+    const long long diff = (long long)T * k - (long long)counts[e] * E;
+    const float step = diff > 0 ? gamma : diff < 0 ? -gamma : 0.f;
+    bias[e] = __fadd_rn(bias[e], step);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_update_bias(float* bias, const int32_t* counts, int T, int k, int E, float gamma,
+                               cudaStream_t s) {
+  update_bias_kernel<<<(E + 255) / 256, 256, 0, s>>>(bias, counts, T, k, E, gamma);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* logits, int T, int H, int E,
                                  cudaStream_t s) {

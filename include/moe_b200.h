@@ -234,6 +234,45 @@ int moe_phase_times(moe_plan_t plan, float* ms, int capacity);
  * `detail` (may be NULL) receives the 4 status words. */
 int moe_check_status(moe_plan_t plan, void* stream, uint32_t* detail);
 
+/* One auxiliary-loss-free balancing step on the selection bias ("전문가 혼합(Mixture of
+ * Experts; MoE)" lesson, "부하 분산 문제" item 3 and "Step 2: 100개 토큰 라우팅하기"):
+ * using the routed experts' row counts of the most recent moe_forward on this plan,
+ *   bias[e] += gamma   if counts[e] * E <  T * k   (used less than the mean load),
+ *   bias[e] -= gamma   if counts[e] * E >  T * k   (used more),
+ *   unchanged          otherwise,
+ * one fp32 addition per expert.  bias: device fp32 [E], 4-byte aligned, updated in place;
+ * the call is asynchronous on `stream` and must be ordered after the forward whose counts it
+ * uses.  Returns MOE_OK, MOE_ERR_INVALID_ARG (NULL/misaligned bias, non-finite gamma),
+ * MOE_ERR_WORKSPACE (no workspace bound) or MOE_ERR_CUDA.  The pages' design has this step
+ * in training; it never runs inside moe_forward. */
+int moe_update_bias(moe_plan_t plan, float* bias, float gamma, void* stream);
+
+/* ---- Dense block-scaled GEMM (the grouped GEMM's linear2 kernel with one group) ----------
+ *
+ *   out[m][n] = bf16_rne( sum_k  A(m,k) * 2^(A_scales[m][k/128] - 127)
+ *                               * E2M1(B, n, k) * 2^(B_scales[n][k/32] - 127) )
+ *
+ * The operand formats of the expert FFN ("DeepSeek Mega MoE / DeepGEMM mega kernel", "TL;DR":
+ * FP8 activations x FP4 weights): A = E4M3 codes [M][K] with one UE8M0 (power-of-two) scale
+ * per row per 128 K-channels, B = packed E2M1 [N][K/2] (low nibble = even element) with one
+ * UE8M0 scale per row per 32 K, fp32 accumulation on the tensor cores, bf16 output [M][N],
+ * all row-major.  Constraints: M >= 1, N % 128 == 0, K % 128 == 0, M*K < 2^31 and N*K < 2^32;
+ * A, B and out 16-byte aligned, the scale arrays 4-byte aligned; all device pointers on the
+ * current device.  Codes 0x7F/0xFF (E4M3 NaN) and scale 0xFF give NaN results. */
+
+/* Device workspace moe_gemm_fp8_fp4 needs for an M x N x K product (scale atoms, bookkeeping
+ * and 16 bytes of status). */
+size_t moe_gemm_workspace_bytes(int M, int N, int K);
+
+/* Asynchronous on `stream`; the caller owns every buffer.  `workspace` (256-byte aligned, at
+ * least moe_gemm_workspace_bytes) holds the status words in its first 16 bytes: word 0 is
+ * MOE_OK or MOE_ERR_DEVICE_TIMEOUT once the stream reaches the end of the call (a bounded wait
+ * of the kernel ran out).  Returns MOE_OK, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_INVALID_ARG,
+ * MOE_ERR_WORKSPACE or MOE_ERR_CUDA. */
+int moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* A, const uint8_t* A_scales, const uint8_t* B,
+                     const uint8_t* B_scales, void* out_bf16, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
 /* Release a plan (NULL is a no-op).  Does not free the workspace. */
 void moe_plan_destroy(moe_plan_t plan);
 

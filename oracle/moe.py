@@ -2,7 +2,7 @@
 
 Sources (page title, section):
   [MoE]   "전문가 혼합(Mixture of Experts; MoE)" lesson -- sections "FFN 교체",
-          "부하 분산 문제", "공유 전문가", "Step 1: 라우터".
+          "부하 분산 문제", "공유 전문가", "Step 1: 라우터", "Step 2: 100개 토큰 라우팅하기".
   [Mega]  "Mega MoE" wiki -- sections "한 줄 정의", "어떻게 작동하나".
   [DG]    "DeepSeek Mega MoE / DeepGEMM mega kernel" -- "TL;DR", "Thông số kỹ thuật".
   [Play]  "Mixture-of-Experts 플레이북" -- section "작동 방식".
@@ -248,3 +248,40 @@ def dense_reference(x_bits, W_router, W1, W1_scales, W2, W2_scales, gates_full):
         res = expert_ffn(xq, xexp, W1[e], W1_scales[e], W2[e], W2_scales[e], I)
         y = y + gates_full[:, e][:, None] * F.bf16_to_f64(res["row_bits"])
     return y
+
+
+# ----------------------------------------------------------------------------- bias update
+
+def update_bias(bias, counts, T: int, k: int, gamma: float) -> np.ndarray:
+    """One auxiliary-loss-free balancing step on the per-expert selection bias.
+
+    [MoE] "부하 분산 문제" item 3 and "Step 2: 100개 토큰 라우팅하기": after a step,
+    every expert used more than its target share loses gamma, every expert used
+    less gains gamma.  Readings: the target is the mean load T*k/E (compared
+    exactly as the integers T*k and count*E); an expert exactly at the target
+    keeps its bias; bias is fp32 (the layer's bias input) and each update is one
+    fp32 addition.  `counts` are the E routed experts' loads.
+    """
+    b = np.asarray(bias, dtype=np.float32)
+    c = np.asarray(counts, dtype=np.int64)
+    E = b.shape[0]
+    diff = np.int64(T) * k - c * E                      # > 0: under-used, < 0: over-used
+    step = np.where(diff > 0, np.float32(gamma), np.where(diff < 0, -np.float32(gamma), np.float32(0)))
+    return (b + step.astype(np.float32)).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------- dense GEMM
+
+def dense_gemm(a_codes, a_scale_codes, b_packed, b_scale_codes):
+    """out[m, n] = sum_k deq(A)[m, k] * deq(B)[n, k] in float64, and its bf16 rounding.
+
+    [DG] "TL;DR": the FP8 x FP4 product of the expert FFN, here for one dense operand pair.
+    A: E4M3 codes [M, K] with UE8M0 codes [M, K/128] (one power of two per row per 128
+    channels, the layer's activation format); B: packed E2M1 [N, K/2] with UE8M0 codes
+    [N, K/32].  Returns (out_f64 [M, N], out_bf16_bits [M, N]).
+    """
+    a_exp = np.asarray(a_scale_codes, dtype=np.int64) - 127
+    a = dequantize_blocks(np.asarray(a_codes, dtype=np.uint8), a_exp)
+    b = F.dequant_mxfp4(np.asarray(b_packed, dtype=np.uint8), np.asarray(b_scale_codes, dtype=np.uint8))
+    out = a @ b.T
+    return out, F.f64_to_bf16(out)

@@ -102,9 +102,23 @@ def test_options_and_unbound_plan(L):
     assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE
     assert L.moe_debug_routing(h, *null[:6]) == binding.MOE_ERR_WORKSPACE
     assert L.moe_set_workspace(h, None, 0) == binding.MOE_ERR_WORKSPACE
+    assert L.moe_update_bias(h, None, 0.01, None) == binding.MOE_ERR_WORKSPACE
+    assert L.moe_update_bias(None, None, 0.01, None) == binding.MOE_ERR_INVALID_ARG
     assert L.moe_forward(None, *null) == binding.MOE_ERR_INVALID_ARG
     L.moe_plan_destroy(h)
     L.moe_plan_destroy(None)
+
+
+def test_dense_gemm_validation_without_a_device(L):
+    assert L.moe_gemm_workspace_bytes(0, 128, 128) == 0
+    assert L.moe_gemm_workspace_bytes(4, 100, 128) == 0          # N % 128
+    assert L.moe_gemm_workspace_bytes(4, 128, 96) == 0           # K % 128
+    n = L.moe_gemm_workspace_bytes(300, 256, 512)
+    # status + bookkeeping, 3 row tiles x 4 K-blocks of 512-byte atoms, 1 n-tile x 4 of 1 KB units
+    assert n == 5 * 256 + 3 * 4 * 512 + 4 * 1024
+    null = [None] * 6
+    assert L.moe_gemm_fp8_fp4(4, 100, 128, *null, 0, None) == binding.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_gemm_fp8_fp4(4, 128, 128, *null, 0, None) == binding.MOE_ERR_INVALID_ARG
 
 
 def test_error_strings(L):

@@ -351,6 +351,37 @@ def test_fused_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     assert_output_close(bits(out), oracle_forward(case, w)["y"], "fused after timeout")
 
 
+def test_update_bias_matches_oracle_and_evens_out_loads(cuda_lib):
+    # one step is bit-exact against the oracle's rule on the forward's counts; a loop of
+    # forward + update brings a skewed router's loads close to uniform
+    w = W("bias_loop", T=100, H=256, I_=256, E=8, k=2)
+    case = make_case(w, seed=21, screened=False)
+    Wr = case["W_router"].clone()
+    Wr[:, 0] += torch.linspace(0.6, -0.6, w.E)
+    case["W_router"] = Wr
+    x = case["x"].clone()
+    x[:, 0] = 1.0
+    case["x"] = x
+    d = to_device(case)
+    p = plan_for(w)
+    bias = torch.zeros(w.E, device="cuda")
+    d["bias"] = bias
+    p.forward(**d)
+    counts = p.region("counts").cpu().numpy()[: w.E]
+    before = bias.cpu().numpy().copy()
+    p.update_bias(bias, 0.02)
+    assert np.array_equal(bias.cpu().numpy(), M.update_bias(before, counts, w.T, w.k, 0.02))
+    start = counts.max() / (w.T * w.k / w.E)
+    ratios = []
+    for _ in range(50):
+        p.forward(**d)
+        p.update_bias(bias, 0.02)
+        ratios.append(p.region("counts").cpu().numpy()[: w.E].max() / (w.T * w.k / w.E))
+    assert p.check_status()[0] == 0
+    assert start > 2.0
+    assert min(ratios[-10:]) < 1.3
+
+
 def test_token_permutation_permutes_output(cuda_lib):
     w = SMALL["ragged_shared"]
     case = make_case(w, seed=4, screened=False)
