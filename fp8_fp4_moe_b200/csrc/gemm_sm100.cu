@@ -1008,25 +1008,23 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    __threadfence();
-    const uint32_t gen = atomicAdd(&bar[1], 0u);
-    if (atomicAdd(&bar[0], 1u) == n_ctas - 1) {
-      atomicExch(&bar[0], 0u);
-      __threadfence();
-      atomicAdd(&bar[1], 1u);
+    // the CTA's writes are ordered before its release-add; the last arrival acquires them all
+    // and releases the next generation, which every waiting CTA acquires
+    const uint32_t gen = ld_acquire_gpu(&bar[1]);
+    if (atom_add_acq_rel_gpu(&bar[0], 1u) == n_ctas - 1) {
+      bar[0] = 0u;
+      st_release_gpu(&bar[1], gen + 1);
     } else {
       const uint64_t t0 = globaltimer_ns();
-      while (atomicAdd(&bar[1], 0u) == gen) {
-        if (globaltimer_ns() - t0 > timeout_ns) {
+      for (uint32_t spin = 0; ld_acquire_gpu(&bar[1]) == gen; ++spin) {
+        if ((spin & 63) == 63 && globaltimer_ns() - t0 > timeout_ns) {
           report_status(status, kStatusTimeout, kWhereGridBarrier, gen);
           ok = false;
           break;
         }
-        __nanosleep(64);
       }
     }
-    __threadfence();
-    *ok_smem = ok && *reinterpret_cast<volatile uint32_t*>(status) == 0u;
+    *ok_smem = ok && ld_acquire_gpu(status) == 0u;
   }
   __syncthreads();
   return *ok_smem != 0;
@@ -1035,6 +1033,16 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32
 // Generic-proxy stores made visible to later TMA (async-proxy) reads of the same data.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int KMAX, int U>
+__device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, long first, long stride) {
+  for (long it = first; it < items; it += U * stride) {
+    long its[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) its[u] = it + u * stride;
+    combine_items<KMAX, U>(its, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
+  }
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -1115,12 +1123,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // S6 combine
   if (ok) {
     const long items = (long)a.T * ((a.H + 255) / 256);
-    for (long it = wfirst; it < items; it += wstride) {
-      if (a.k <= 2) combine_item<2>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
-      else if (a.k <= 4) combine_item<4>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
-      else if (a.k <= 8) combine_item<8>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
-      else combine_item<16>(it, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
-    }
+    // several items per warp in flight: one CTA per SM leaves only 10 warps to hide latency
+    if (a.k <= 2) fused_combine<2, 4>(a, items, wfirst, wstride);
+    else if (a.k <= 4) fused_combine<4, 4>(a, items, wfirst, wstride);
+    else if (a.k <= 8) fused_combine<8, 2>(a, items, wfirst, wstride);
+    else fused_combine<16, 1>(a, items, wfirst, wstride);
   }
   __syncthreads();
   if (warp == 1) {

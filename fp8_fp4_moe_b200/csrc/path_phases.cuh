@@ -399,6 +399,10 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
   const int g = t / 32;
   const long R = (long)T * k;
   const int kw = H / 128;
+  // the token's 8 channels of this lane, loaded before the position lookups it does not depend on
+  const int c0 = slice * 256 + lane * 8;
+  const bool active = x != nullptr && c0 < H;     // H % 128 == 0: whole half-warps
+  const uint4 raw = active ? *reinterpret_cast<const uint4*>(x + (long)t * H + c0) : make_uint4(0, 0, 0, 0);
   int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
   int e = -1;
   if (lane < k) {
@@ -421,13 +425,9 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
     sf_off = ((long)(mtile_start[e] + rank / 128) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
   }
   const int ndst = k + shared;
-  const uint16_t* xr = x + (long)t * H;
   {
     // 8 channels per lane; a 128-channel block spans 16 lanes.  Every lane runs
     // the shuffles (full mask); a half-warp past H idles.
-    const int c0 = slice * 256 + lane * 8;
-    const bool active = c0 < H;           // H % 128 == 0: whole half-warps
-    const uint4 raw = active ? *reinterpret_cast<const uint4*>(xr + c0) : make_uint4(0, 0, 0, 0);
     float v[8];
     v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
     v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
@@ -460,55 +460,66 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
 // out[t] = bf16( sum_{j<k} gate[t][j] * row[slot_pos[t][j]] + shared * row[R + t] ),
 // fp32 accumulation in exactly that order (deterministic, no atomics).  KMAX >= k bounds
 // the rows a lane holds in registers (all loaded before the first is used).
-// Called by a whole warp for one (token, 256-channel slice) item.
-template <int KMAX>
-__device__ __forceinline__ void combine_item(long item, const uint16_t* __restrict__ y,
-                                             const int32_t* __restrict__ slot_pos, const float* __restrict__ gates,
-                                             uint16_t* __restrict__ out, int T, int H, int k, int shared) {
+// Called by a whole warp for U (token, 256-channel slice) items (indices past T * slices are
+// skipped).
+template <int KMAX, int U>
+__device__ __forceinline__ void combine_items(const long (&items)[U], const uint16_t* __restrict__ y,
+                                              const int32_t* __restrict__ slot_pos, const float* __restrict__ gates,
+                                              uint16_t* __restrict__ out, int T, int H, int k, int shared) {
   const int lane = threadIdx.x % 32;
   const int n_slices = (H + 255) / 256;
-  if (item >= (long)T * n_slices) return;
-  const int t = (int)(item / n_slices);
-  const int slice = (int)(item % n_slices);
   const long R = (long)T * k;
-  int my_row = 0;
-  float my_gate = 0.f;
-  if (lane < k) {
-    my_row = slot_pos[(long)t * k + lane];
-    my_gate = gates[(long)t * k + lane];
+  // every load of the U items is issued before the first is used; each sum keeps slot order
+  int t[U], c0[U];
+  bool valid[U], active[U];
+  int my_row[U];
+  float my_gate[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    valid[u] = items[u] < (long)T * n_slices;          // warp-uniform
+    t[u] = valid[u] ? (int)(items[u] / n_slices) : 0;
+    c0[u] = (valid[u] ? (int)(items[u] % n_slices) : 0) * 256 + lane * 8;
+    active[u] = valid[u] && c0[u] < H;
+    my_row[u] = 0;
+    my_gate[u] = 0.f;
+    if (valid[u] && lane < k) {
+      my_row[u] = slot_pos[(long)t[u] * k + lane];
+      my_gate[u] = gates[(long)t[u] * k + lane];
+    }
   }
-  {
-    const int c0 = slice * 256 + lane * 8;
-    const bool active = c0 < H;
+  uint4 raw[U][KMAX];
+  float g[U][KMAX];
+  uint4 raw_s[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const long r = __shfl_sync(0xffffffffu, my_row[u], j);
+      g[u][j] = __shfl_sync(0xffffffffu, my_gate[u], j);
+      if (j < k && active[u]) raw[u][j] = *reinterpret_cast<const uint4*>(y + r * H + c0[u]);
+    }
+    raw_s[u] = make_uint4(0, 0, 0, 0);
+    if (shared && active[u]) raw_s[u] = *reinterpret_cast<const uint4*>(y + (R + t[u]) * H + c0[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    if (!active[u]) continue;
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    // all k (+1) rows are loaded before the first use; the sum keeps slot order
-    uint4 raw_j[KMAX];
-    float g_j[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      const long r = __shfl_sync(0xffffffffu, my_row, j);
-      g_j[j] = __shfl_sync(0xffffffffu, my_gate, j);
-      if (j < k && active) raw_j[j] = *reinterpret_cast<const uint4*>(y + r * H + c0);
-    }
-    uint4 raw_s = make_uint4(0, 0, 0, 0);
-    if (shared && active) raw_s = *reinterpret_cast<const uint4*>(y + (R + t) * H + c0);
-    if (!active) return;                 // no shuffles below
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       if (j < k) {
-        const uint32_t w[4] = {raw_j[j].x, raw_j[j].y, raw_j[j].z, raw_j[j].w};
+        const uint32_t w[4] = {raw[u][j].x, raw[u][j].y, raw[u][j].z, raw[u][j].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          acc[2 * i] = fmaf(g_j[j], __uint_as_float(w[i] << 16), acc[2 * i]);
-          acc[2 * i + 1] = fmaf(g_j[j], __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
+          acc[2 * i] = fmaf(g[u][j], __uint_as_float(w[i] << 16), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(g[u][j], __uint_as_float(w[i] & 0xFFFF0000u), acc[2 * i + 1]);
         }
       }
     }
     if (shared) {
-      const uint4 raw = raw_s;
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+      const uint32_t w[4] = {raw_s[u].x, raw_s[u].y, raw_s[u].z, raw_s[u].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         acc[2 * i] += __uint_as_float(w[i] << 16);
@@ -524,8 +535,16 @@ __device__ __forceinline__ void combine_item(long item, const uint16_t* __restri
     o.y = *reinterpret_cast<uint32_t*>(&b1);
     o.z = *reinterpret_cast<uint32_t*>(&b2);
     o.w = *reinterpret_cast<uint32_t*>(&b3);
-    *reinterpret_cast<uint4*>(out + (long)t * H + c0) = o;
+    *reinterpret_cast<uint4*>(out + (long)t[u] * H + c0[u]) = o;
   }
+}
+
+template <int KMAX>
+__device__ __forceinline__ void combine_item(long item, const uint16_t* __restrict__ y,
+                                             const int32_t* __restrict__ slot_pos, const float* __restrict__ gates,
+                                             uint16_t* __restrict__ out, int T, int H, int k, int shared) {
+  const long items[1] = {item};
+  combine_items<KMAX, 1>(items, y, slot_pos, gates, out, T, H, k, shared);
 }
 
 }  // namespace
