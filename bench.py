@@ -43,7 +43,10 @@ REF_STEP_TOKENS = {"tiny": 64, "mixtral": 1, "dsv3_t1": 1, "dsv3_t512": 1, "dsv3
                    "dsv3_t32768": 1}
 
 
-KERNELS_PER_FORWARD = 8
+def kernels_per_forward(w) -> int:
+    """router, top-k, column scan, expert scan, scatter, linear1, linear2, combine; with at
+    most 32 tokens top-k and the two scans are one kernel (prepare is skipped: weights static)."""
+    return 6 if w.T <= 32 else 8
 
 
 def parse():
@@ -442,7 +445,7 @@ def run_cuda(args, rank, world, local_rank):
                    "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
                    "launch": ("one persistent cooperative kernel (MOE_OPT_FUSED)" if fused else
                               "kernels launched one by one" if args.no_graph else
-                              f"CUDA graph replay of the {KERNELS_PER_FORWARD} kernels (MOE_OPT_GRAPH)"),
+                              f"CUDA graph replay of the {kernels_per_forward(w)} kernels (MOE_OPT_GRAPH)"),
                    "phase_times": "separate pass, CUDA events between kernels, 20 steps",
                    "weight_scales": f"re-laid out once before timing ({prepare_ms:.3f} ms), reused "
                                     "(MOE_OPT_STATIC_WEIGHTS)",
@@ -457,9 +460,8 @@ def run_cuda(args, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # router, top-k, column scan, expert scan, scatter, linear1, linear2, combine (prepare is
-        # skipped: weights static); the fused option is one kernel
-        "gpu_launches": (1 if fused else KERNELS_PER_FORWARD) * args.steps,
+        # the fused option is one kernel per forward
+        "gpu_launches": (1 if fused else kernels_per_forward(w)) * args.steps,
         "clocks": clocks,
         "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
     }

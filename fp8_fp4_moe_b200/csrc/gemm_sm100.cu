@@ -50,19 +50,32 @@ constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
 // Transaction bytes per stage: A 16 KB, B counted at 4 bits per element (16 KB), scale atoms.
 constexpr uint32_t kStageTxBytes = BM * BK + BN * BK / 2 + kSfaBytes + kSfbBytes;
 
-struct SmemLayout {
+// Shared memory of the single-CTA grouped GEMM: STAGES pipeline stages with an A region of
+// A_BYTES each, and (STAGING) a 2 KB per-warp buffer the epilogue stores go through.
+template <int STAGES, uint32_t A_BYTES, bool STAGING>
+struct GemmSmem {
+  static constexpr int kStages = STAGES;
+  static constexpr uint32_t kABytes = A_BYTES;
+  static constexpr bool kStaging = STAGING;
   static constexpr uint32_t a = 0;
-  static constexpr uint32_t b = a + S * kATileBytes;
-  static constexpr uint32_t sfa = b + S * kBTileBytes;
-  static constexpr uint32_t sfb = sfa + S * kSfaBytes;
-  static constexpr uint32_t amax = sfb + S * kSfbBytes;           // [2 buffers][2 halves][128 rows] fp32
+  static constexpr uint32_t b = a + STAGES * A_BYTES;
+  static constexpr uint32_t sfa = b + STAGES * kBTileBytes;
+  static constexpr uint32_t sfb = sfa + STAGES * kSfaBytes;
+  static constexpr uint32_t amax = sfb + STAGES * kSfbBytes;      // [2 buffers][2 halves][128 rows] fp32
   static constexpr uint32_t stage_out = amax + 2 * 2 * 128 * 4;   // [8 epilogue warps][32 rows][64 B]
-  static constexpr uint32_t bars = stage_out + 8 * 2048;
-  // full[S], empty[S], accf[2], acce[2], drain
-  static constexpr uint32_t n_bars = 2 * S + 5;
+  static constexpr uint32_t bars = stage_out + (STAGING ? 8 * 2048 : 0);
+  // full[STAGES], empty[STAGES], accf[2], acce[2], drain
+  static constexpr uint32_t n_bars = 2 * STAGES + 5;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t total = misc + 16;
 };
+// Any number of rows per tile: 4 stages with 128-row A regions.
+using SmemLayout = GemmSmem<S, kATileBytes, true>;
+// At most 16 rows per expert (T <= 16): 16-row A regions leave room for 6 stages; the MMA
+// still reads 128 A rows, the ones past the region are other stages' bytes and land in
+// accumulator rows that are never stored.  Epilogue stores go straight to global memory.
+using SmallSmem = GemmSmem<6, 16 * BK, false>;
+static_assert(SmallSmem::total + 1024 <= 232448, "few-token layout exceeds shared memory");
 
 struct TileCoord {
   int e, mt, nt, count, row0, gmt;   // gmt = global row-tile index
@@ -150,6 +163,13 @@ __device__ __forceinline__ bool epi_all(bool ok) {
 // only rows with row_ok set (in the owning lane) are written.
 __device__ __forceinline__ void store_rows_64b(uint8_t* buf, const uint4 (&v)[4], uint8_t* dst0, long row_stride,
                                                bool row_ok, int lane) {
+  if (buf == nullptr) {                // no staging buffer (few rows): each lane writes its row
+    if (row_ok) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(dst0 + lane * row_stride + c * 16) = v[c];
+    }
+    return;
+  }
   const uint32_t okmask = __ballot_sync(0xffffffffu, row_ok);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
@@ -355,21 +375,23 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord
 // with `tmem_base` holding 512 allocated TMEM columns and `smem` the 1024-aligned dynamic
 // shared memory.  Initialises its barriers on entry and invalidates them on exit, so the
 // same CTA may run it again (the single persistent forward runs linear1, then linear2).
-template <int MODE>
+template <int MODE, class L = SmemLayout>
 __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& tmB, const GemmArgs& p,
                                           uint8_t* smem, uint32_t tmem_base, int cta, int n_ctas) {
-  uint8_t* a_s = smem + SmemLayout::a;
-  uint8_t* b_s = smem + SmemLayout::b;
-  uint8_t* sfa_s = smem + SmemLayout::sfa;
-  uint8_t* sfb_s = smem + SmemLayout::sfb;
-  float* amax_s = reinterpret_cast<float*>(smem + SmemLayout::amax);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
+  constexpr int S = L::kStages;
+  constexpr uint32_t kATileBytes = L::kABytes;
+  uint8_t* a_s = smem + L::a;
+  uint8_t* b_s = smem + L::b;
+  uint8_t* sfa_s = smem + L::sfa;
+  uint8_t* sfb_s = smem + L::sfb;
+  float* amax_s = reinterpret_cast<float*>(smem + L::amax);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* accf = bars + 2 * S;      // [2] accumulator slot full
   uint64_t* acce = accf + 2;          // [2] accumulator slot empty
   uint64_t* drain = accf + 4;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SmemLayout::misc + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -414,7 +436,8 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
         const int rows_here = min(BM, c.count - c.mt * BM);
-        const int a_sel = rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
+        // (a 16-row A region only ever gets the 16-row box)
+        const int a_sel = kATileBytes <= 16 * BK || rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
         const uint32_t a_box = 16u << a_sel;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
@@ -423,7 +446,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
           } else {
             // A rows of this tile that belong to the expert decide the box height; the MMA
             // still reads 128 rows, the rest are leftovers whose accumulator rows are dropped
-            mbar_arrive_expect_tx(&full[stage], kStageTxBytes - kATileBytes + a_box * BK);
+            mbar_arrive_expect_tx(&full[stage], kStageTxBytes - BM * BK + a_box * BK);
             tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
             if constexpr (MODE == 1) {
               const int brow = c.e * p.rows_b + c.nt * 128;
@@ -511,7 +534,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
     // ------------------------------------------------------------ epilogue (warps 2..9)
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;      // which half of the accumulator columns
-    uint8_t* obuf = smem + SmemLayout::stage_out + (warp - 2) * 2048;
+    uint8_t* obuf = L::kStaging ? smem + L::stage_out + (warp - 2) * 2048 : nullptr;
     uint32_t uses0 = 0, uses1 = 0;
     int next_slot = 0;
     int buf = 0;
@@ -541,12 +564,12 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
 
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < (int)SmemLayout::n_bars; ++i) mbar_inval(bars + i);
+    for (int i = 0; i < (int)L::n_bars; ++i) mbar_inval(bars + i);
   }
   __syncthreads();
 }
 
-template <int MODE>
+template <int MODE, class L>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs p) {
@@ -563,7 +586,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  gemm_body<MODE>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
+  gemm_body<MODE, L>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -1165,21 +1188,28 @@ cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* 
 }
 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
+size_t gemm_small_smem_bytes() { return SmallSmem::total + 1024; }
 size_t gemm_pair_smem_bytes() { return PairSmem::total + 1024; }
 size_t fused_smem_bytes() { return kFusedMiscOffset + 16 + 1024; }
 int g_fused_ctas[64] = {};
 int g_pair_clusters[64] = {};
 
 cudaError_t gemm_prepare_device() {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)gemm_smem_bytes());
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<1, SmemLayout>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<1, SmallSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_small_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmallSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_small_smem_bytes());
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tile_weight_scales_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)router_tc_smem_bytes());
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmemLayout>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_smem_bytes());
   if (e != cudaSuccess) return e;
   for (int mode = 1; mode <= 2; ++mode) {
@@ -1254,14 +1284,20 @@ cudaError_t launch_gemm_pair_linear2(const AMaps& a, const CUtensorMap& b, const
 }
 
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s) {
-  grouped_gemm_kernel<1><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
+                                cudaStream_t s, bool few_rows) {
+  if (few_rows)
+    grouped_gemm_kernel<1, SmallSmem><<<grid, kGemmThreads, gemm_small_smem_bytes(), s>>>(a, b, args);
+  else
+    grouped_gemm_kernel<1, SmemLayout><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s) {
-  grouped_gemm_kernel<2><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
+                                cudaStream_t s, bool few_rows) {
+  if (few_rows)
+    grouped_gemm_kernel<2, SmallSmem><<<grid, kGemmThreads, gemm_small_smem_bytes(), s>>>(a, b, args);
+  else
+    grouped_gemm_kernel<2, SmemLayout><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
   return cudaGetLastError();
 }
 

@@ -58,10 +58,12 @@ cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_ex
 struct AMaps {
   CUtensorMap m[4];
 };
+// few_rows: every expert has at most 16 rows (T <= 16), so the kernel may use 16-row A regions
+// and 6 pipeline stages.
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s);
+                                cudaStream_t s, bool few_rows = false);
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s);
+                                cudaStream_t s, bool few_rows = false);
 // CTA-pair variants: b with 128-row boxes (each CTA loads half of the 256 B rows), scale atoms
 // and weight scale units as 2-D uint8 maps of 256-byte rows (boxes of 2 and 4 rows); grid =
 // 2 x pairs.
@@ -143,6 +145,12 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
                              float* gates,
                              int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
                              cudaStream_t s);
+// T <= 32: launch_topk_rank followed by launch_dispatch_scan, as one single-block kernel.
+cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
+                                      int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
+                                      uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
+                                      int32_t* mtile_start, int32_t* ptile_start, int T, int E, int k, int shared,
+                                      cudaStream_t s);
 // counts, offsets, mtile_start, ptile_start (n + 1 entries) and group_base[g][e] = rows of
 // expert e in token groups < g (relative to offsets[e]).
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,

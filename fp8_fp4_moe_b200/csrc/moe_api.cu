@@ -220,16 +220,28 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
   int rc = run_router(p, x, W_router, s);
   if (rc != MOE_OK) return rc;
   mark(p, 1 + MOE_PHASE_ROUTER, s);
-  if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
-                            at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
-                            region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s)) != cudaSuccess)
-    return cuda_rc(e);
-  mark(p, 1 + MOE_PHASE_TOPK, s);
-  if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
-                                region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
-                                at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
-                                p->shared, s)) != cudaSuccess)
-    return cuda_rc(e);
+  if (p->T <= 32) {
+    // one token group: top-k, ranks and the scans in one block (reported under top-k)
+    if ((e = launch_topk_scan_one_group(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
+                                        at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
+                                        region<uint32_t>(p, MOE_REGION_STATUS), at<int32_t>(p, p->off_gbase),
+                                        region<int32_t>(p, MOE_REGION_COUNTS), region<int32_t>(p, MOE_REGION_OFFSETS),
+                                        at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                        p->shared, s)) != cudaSuccess)
+      return cuda_rc(e);
+    mark(p, 1 + MOE_PHASE_TOPK, s);
+  } else {
+    if ((e = launch_topk_rank(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
+                              at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
+                              region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s)) != cudaSuccess)
+      return cuda_rc(e);
+    mark(p, 1 + MOE_PHASE_TOPK, s);
+    if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
+                                  region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
+                                  at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                  p->shared, s)) != cudaSuccess)
+      return cuda_rc(e);
+  }
   mark(p, 1 + MOE_PHASE_SCAN, s);
   e = launch_scatter_quant(x, ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase),
                            region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile),
@@ -340,10 +352,12 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR2, s);
   } else {
-    if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess)
+    // an expert never gets more rows than there are tokens
+    const bool few_rows = p->T <= 16;
+    if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, few_rows) != cudaSuccess)
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR1, s);
-    if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s) != cudaSuccess)
+    if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR2, s);
   }

@@ -164,6 +164,25 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
                         T, E, k, sm);
 }
 
+// T <= 32 (a single token group): top-k, ranks and both dispatch scans in one block; the
+// group's counts are the experts' counts and every group base is 0.
+__global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
+    int mode, const float* __restrict__ logits, int n_parts, const float* __restrict__ bias, int32_t* topk_ids,
+    float* gates, int32_t* __restrict__ local_rank, int32_t* __restrict__ group_counts, uint32_t* status,
+    int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
+    int k, int shared) {
+  __shared__ TopkSmem sm;
+  __shared__ int32_t wsum[3][32];
+  topk_rank_group<1024>(0, mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k,
+                        sm);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    counts[e] = group_counts[e];
+    group_base[e] = 0;
+  }
+  __syncthreads();
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, T, E, shared, wsum);
+}
+
 // --------------------------------------------------------------------------- scan
 __global__ void __launch_bounds__(256) column_scan_kernel(const int32_t* __restrict__ group_counts,
                                                           int32_t* __restrict__ group_base, int32_t* counts, int G,
@@ -296,6 +315,18 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
   const int G = (T + 31) / 32;
   topk_rank_kernel<<<G, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status,
                                       T, E, k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
+                                      int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
+                                      uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
+                                      int32_t* mtile_start, int32_t* ptile_start, int T, int E, int k, int shared,
+                                      cudaStream_t s) {
+  if (T > 32 || n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
+  topk_scan_one_group_kernel<<<1, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank,
+                                                 group_counts, status, group_base, counts, offsets, mtile_start,
+                                                 ptile_start, T, E, k, shared);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,8 @@ SMALL = {
     "tiny": I.WORKLOADS["tiny"],
     "ragged_shared": W("ragged_shared", T=333, H=384, I_=256, E=16, k=4, shared=1, router_std=0.05, bias="uniform"),
     "t1_k1": W("t1_k1", T=1, H=256, I_=256, E=4, k=1),
+    # T <= 16: the GEMMs use the few-token shared-memory layout (16-row A regions, 6 stages)
+    "t16_shared": W("t16_shared", T=16, H=512, I_=384, E=4, k=2, shared=1, bias="uniform"),
     "k_eq_E": W("k_eq_E", T=50, H=256, I_=384, E=6, k=6, shared=1),
     "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
     # T >= 256 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
