@@ -43,6 +43,11 @@ __device__ __forceinline__ int ld_cg(const int32_t* p) {
   asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+__device__ __forceinline__ int4 ld_cg_v4(const int4* p) {
+  int4 v;
+  asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
 
 // gpu-scope acquire / release accesses for grid-wide synchronisation
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {

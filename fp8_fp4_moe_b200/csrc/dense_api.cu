@@ -17,7 +17,7 @@ using namespace moe;
 namespace {
 
 struct DenseLayout {
-  size_t status, counts, offsets, mtile, ptile, atoms, units, total;
+  size_t status, counts, offsets, mtile, ptile, tinfo, atoms, units, total;
 };
 
 size_t r256(size_t b) { return (b + 255) & ~size_t(255); }
@@ -31,6 +31,7 @@ DenseLayout dense_layout(int M, int N, int K) {
   L.mtile = off;   off += r256(8);
   L.ptile = off;   off += r256(8);
   const size_t mt = ((size_t)M + 127) / 128, kt = (size_t)K / 128, nt = ((size_t)N + 255) / 256;
+  L.tinfo = off;   off += r256(mt * 16);
   L.atoms = off;   off += r256(mt * kt * 512);
   L.units = off;   off += r256(nt * kt * 1024);
   L.total = off;
@@ -44,13 +45,16 @@ bool shape_ok(int M, int N, int K) {
 
 bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// The single group's bookkeeping and the activation scale atoms: atom (row tile g, K-block kb)
+// The single group's bookkeeping (row-tile table entries {0, 0, M, 0}) and the activation scale
+// atoms: atom (row tile g, K-block kb)
 // holds row 128 g + r's code at bytes (r % 32) * 16 + (r / 32) * 4 .. + 3 (one per 32-K block of
 // the 128).  Rows past M get code 127 (x1); their accumulator rows are never stored.
 __global__ void __launch_bounds__(256) dense_setup_kernel(const uint8_t* __restrict__ A_scales, int M, int K,
                                                           int32_t* counts, int32_t* offsets, int32_t* mtile,
-                                                          int32_t* ptile, uint8_t* atoms) {
+                                                          int32_t* ptile, int4* tinfo, uint8_t* atoms) {
   const int kw = K / 128, mt = (M + 127) / 128;
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < mt; g += gridDim.x * blockDim.x)
+    tinfo[g] = make_int4(0, 0, M, 0);
   const long n = (long)mt * 128 * kw;
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
     const int row = (int)(i / kw), kb = (int)(i % kw);
@@ -115,7 +119,8 @@ int moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* A, const uint8_t* A_sca
   dense_setup_kernel<<<setup_grid, 256, 0, s>>>(A_scales, M, K, reinterpret_cast<int32_t*>(ws + L.counts),
                                                 reinterpret_cast<int32_t*>(ws + L.offsets),
                                                 reinterpret_cast<int32_t*>(ws + L.mtile),
-                                                reinterpret_cast<int32_t*>(ws + L.ptile), ws + L.atoms);
+                                                reinterpret_cast<int32_t*>(ws + L.ptile),
+                                                reinterpret_cast<int4*>(ws + L.tinfo), ws + L.atoms);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_tile_weight_scales(B_scales, ws + L.units, 1, N, K, nt, 2, N, s) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs a{};
@@ -130,6 +135,8 @@ int moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* A, const uint8_t* A_sca
   a.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
   a.mtile_start = reinterpret_cast<const int32_t*>(ws + L.mtile);
   a.ptile_start = reinterpret_cast<const int32_t*>(ws + L.ptile);
+  a.tile_info = reinterpret_cast<const int4*>(ws + L.tinfo);
+  a.ptile_info = nullptr;                // the dense product never runs on CTA pairs
   a.sfa = ws + L.atoms;
   a.sfb = ws + L.units;
   a.y = static_cast<uint16_t*>(out_bf16);

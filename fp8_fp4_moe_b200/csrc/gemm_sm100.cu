@@ -82,22 +82,20 @@ struct TileCoord {
   int rows;                          // rows of the expert in this tile (1..128)
 };
 
+// The tiles of expert e are [mtile_start[e], mtile_start[e + 1]) x n_tiles_n, so tile / n_tiles_n
+// is one of e's row tiles and its table entry names e: one load per tile instead of a search
+// over the experts.
 __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
-  // largest e with mtile_start[e] * n_tiles_n <= tile
-  int lo = 0, hi = p.n_experts;
-  while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
-    if (ld_cg(p.mtile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
-  }
+  const int4 info = ld_cg_v4(p.tile_info + tile / p.n_tiles_n);   // {e, mtile_start, count, offset}
   TileCoord c;
-  c.e = lo;
-  c.count = ld_cg(p.counts + lo);
+  c.e = info.x;
+  c.count = info.z;
   const int mtiles = (c.count + BM - 1) / BM;
-  const int mstart = ld_cg(p.mtile_start + lo);
+  const int mstart = info.y;
   const int local = tile - mstart * p.n_tiles_n;
   c.nt = local / mtiles;             // tiles of one expert: n-major, m fastest
   c.mt = local - c.nt * mtiles;
-  c.row0 = ld_cg(p.offsets + lo) + c.mt * BM;
+  c.row0 = info.w + c.mt * BM;
   c.gmt = mstart + c.mt;
   c.rows = min(BM, c.count - c.mt * BM);
   return c;
@@ -623,22 +621,19 @@ struct PairSmem {
 
 // Tile `tile` of the pair grid as seen by CTA `rank`: row tile 2*pm + rank of the expert (its
 // rows can be 0 for rank 1 on an expert with an odd number of row tiles).
+// The expert comes from the pair-tile table entry tile / n_tiles_n (as in decode_tile).
 __device__ __forceinline__ TileCoord decode_pair_tile(const GemmArgs& p, int tile, int rank) {
-  int lo = 0, hi = p.n_experts;
-  while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
-    if (ld_cg(p.ptile_start + mid) * p.n_tiles_n <= tile) lo = mid; else hi = mid;
-  }
+  const int4 info = ld_cg_v4(p.ptile_info + tile / p.n_tiles_n);   // {e, ptile_start, count, offset}
   TileCoord c;
-  c.e = lo;
-  c.count = ld_cg(p.counts + lo);
+  c.e = info.x;
+  c.count = info.z;
   const int mtiles = (c.count + BM - 1) / BM;
   const int ptiles = (mtiles + 1) / 2;
-  const int local = tile - ld_cg(p.ptile_start + lo) * p.n_tiles_n;
+  const int local = tile - info.y * p.n_tiles_n;
   c.nt = local / ptiles;
   c.mt = 2 * (local - c.nt * ptiles) + rank;
-  c.row0 = ld_cg(p.offsets + lo) + c.mt * BM;
-  c.gmt = ld_cg(p.mtile_start + lo) + c.mt;
+  c.row0 = info.w + c.mt * BM;
+  c.gmt = ld_cg(p.mtile_start + c.e) + c.mt;
   c.rows = max(0, min(BM, c.count - c.mt * BM));
   return c;
 }
@@ -1125,8 +1120,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (long e = wfirst; e < a.E; e += wstride) column_scan_warp((int)e, a.group_counts, a.group_base, a.counts, G, a.E);
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
   if (ok && cta == 0)
-    expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.T, a.E, a.shared,
-                                    reinterpret_cast<int32_t(*)[32]>(smem));
+    expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.tile_info, a.ptile_info,
+                                    a.T, a.E, a.shared, reinterpret_cast<int32_t(*)[32]>(smem));
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
   if (ok) {
     const long items = (long)a.T * ((a.H + 255) / 256);

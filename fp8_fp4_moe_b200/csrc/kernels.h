@@ -38,6 +38,11 @@ struct GemmArgs {
   const int32_t* offsets;      // [n_experts + 1]
   const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
   const int32_t* ptile_start;  // [n_experts + 1] prefix sum of ceil(ceil(count/128)/2) (CTA pairs)
+  // Row-tile table: entry g in [mtile_start[e], mtile_start[e + 1]) holds {e, mtile_start[e],
+  // counts[e], offsets[e]}; the CTA-pair table the same over ptile_start with ptile_start[e]
+  // in .y.  Tile t of the n-major order belongs to the expert of entry t / n_tiles_n.
+  const int4* tile_info;
+  const int4* ptile_info;
   const uint8_t* sfa;          // activation scale atoms
   const uint8_t* sfb;          // weight scale units
   uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
@@ -116,6 +121,8 @@ struct FusedArgs {
   int32_t* offsets;
   int32_t* mtile_start;
   int32_t* ptile_start;
+  int4* tile_info;
+  int4* ptile_info;
   int32_t* slot_pos;
   int32_t* perm;
   uint8_t* xq;
@@ -149,13 +156,13 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
 cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
-                                      int32_t* mtile_start, int32_t* ptile_start, int T, int E, int k, int shared,
-                                      cudaStream_t s);
-// counts, offsets, mtile_start, ptile_start (n + 1 entries) and group_base[g][e] = rows of
-// expert e in token groups < g (relative to offsets[e]).
+                                      int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
+                                      int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s);
+// counts, offsets, mtile_start, ptile_start (n + 1 entries), the row-tile tables (see GemmArgs)
+// and group_base[g][e] = rows of expert e in token groups < g (relative to offsets[e]).
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
-                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
-                                 int k, int shared, cudaStream_t s);
+                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
+                                 int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s);
 // Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms.
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,

@@ -36,6 +36,7 @@ struct moe_plan_s {
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
   size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_ptile, off_w1sf, off_w2sf, off_whi, off_wlo;
+  size_t off_tinfo, off_ptinfo;     // row-tile tables of the grouped GEMMs (mt_cap int4 each)
   size_t off_gridbar;               // grid barrier words of the fused forward
   long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
@@ -132,6 +133,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
   a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
   a.mtile_start = at<int32_t>(p, p->off_mtile);
   a.ptile_start = at<int32_t>(p, p->off_ptile);
+  a.tile_info = at<int4>(p, p->off_tinfo);
+  a.ptile_info = at<int4>(p, p->off_ptinfo);
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
   a.swap_rows = p->swap_rows;
@@ -226,7 +229,8 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
                                         at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gcounts),
                                         region<uint32_t>(p, MOE_REGION_STATUS), at<int32_t>(p, p->off_gbase),
                                         region<int32_t>(p, MOE_REGION_COUNTS), region<int32_t>(p, MOE_REGION_OFFSETS),
-                                        at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                        at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
+                                        at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
                                         p->shared, s)) != cudaSuccess)
       return cuda_rc(e);
     mark(p, 1 + MOE_PHASE_TOPK, s);
@@ -238,7 +242,8 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
     mark(p, 1 + MOE_PHASE_TOPK, s);
     if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), region<int32_t>(p, MOE_REGION_COUNTS),
                                   region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
-                                  at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                  at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
+                                  at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
                                   p->shared, s)) != cudaSuccess)
       return cuda_rc(e);
   }
@@ -305,6 +310,8 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
   a.offsets = region<int32_t>(p, MOE_REGION_OFFSETS);
   a.mtile_start = at<int32_t>(p, p->off_mtile);
   a.ptile_start = at<int32_t>(p, p->off_ptile);
+  a.tile_info = at<int4>(p, p->off_tinfo);
+  a.ptile_info = at<int4>(p, p->off_ptinfo);
   a.slot_pos = region<int32_t>(p, MOE_REGION_SLOT_POS);
   a.perm = region<int32_t>(p, MOE_REGION_PERM);
   a.xq = region<uint8_t>(p, MOE_REGION_XQ);
@@ -467,6 +474,8 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_gbase = add((size_t)p->G * E * 4);
   p->off_mtile = add((size_t)(p->n + 1) * 4);
   p->off_ptile = add((size_t)(p->n + 1) * 4);
+  p->off_tinfo = add((size_t)p->mt_cap * 16);
+  p->off_ptinfo = add((size_t)p->mt_cap * 16);
   p->off_gridbar = add(8);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
@@ -675,7 +684,8 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
                                    region<uint32_t>(p, MOE_REGION_STATUS), p->T, p->E, p->k, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), counts, offsets, at<int32_t>(p, p->off_gbase),
-                                at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile), p->T, p->E, p->k,
+                                at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
+                                at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
                                 p->shared, s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   // positions = offsets (written just above into the caller's buffer) + group base + rank

@@ -169,8 +169,8 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
 __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     int mode, const float* __restrict__ logits, int n_parts, const float* __restrict__ bias, int32_t* topk_ids,
     float* gates, int32_t* __restrict__ local_rank, int32_t* __restrict__ group_counts, uint32_t* status,
-    int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
-    int k, int shared) {
+    int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start,
+    int4* tile_info, int4* ptile_info, int T, int E, int k, int shared) {
   __shared__ TopkSmem sm;
   __shared__ int32_t wsum[3][32];
   topk_rank_group<1024>(0, mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k,
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     group_base[e] = 0;
   }
   __syncthreads();
-  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, T, E, shared, wsum);
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum);
 }
 
 // --------------------------------------------------------------------------- scan
@@ -192,9 +192,10 @@ __global__ void __launch_bounds__(256) column_scan_kernel(const int32_t* __restr
 }
 
 __global__ void __launch_bounds__(1024) expert_scan_kernel(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
-                                                           int32_t* ptile_start, int T, int E, int shared) {
+                                                           int32_t* ptile_start, int4* tile_info, int4* ptile_info,
+                                                           int T, int E, int shared) {
   __shared__ int32_t wsum[3][32];
-  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, T, E, shared, wsum);
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum);
 }
 
 // --------------------------------------------------------------------------- scatter + quant
@@ -321,21 +322,22 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
 cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
-                                      int32_t* mtile_start, int32_t* ptile_start, int T, int E, int k, int shared,
-                                      cudaStream_t s) {
+                                      int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
+                                      int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
   if (T > 32 || n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
   topk_scan_one_group_kernel<<<1, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank,
                                                  group_counts, status, group_base, counts, offsets, mtile_start,
-                                                 ptile_start, T, E, k, shared);
+                                                 ptile_start, tile_info, ptile_info, T, E, k, shared);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
-                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int T, int E,
-                                 int k, int shared, cudaStream_t s) {
+                                 int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
+                                 int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
   const int G = (T + 31) / 32;
   column_scan_kernel<<<(E + 7) / 8, 256, 0, s>>>(group_counts, group_base, counts, G, E);
-  expert_scan_kernel<<<1, 1024, 0, s>>>(counts, offsets, mtile_start, ptile_start, T, E, shared);
+  expert_scan_kernel<<<1, 1024, 0, s>>>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E,
+                                        shared);
   return cudaGetLastError();
 }
 

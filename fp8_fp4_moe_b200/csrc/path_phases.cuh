@@ -309,10 +309,12 @@ __device__ __forceinline__ void column_scan_warp(int e, const int32_t* __restric
 }
 
 // Called by all NT threads of one block (it synchronises them); n = E + shared <= 1024.
+// Also fills the row-tile tables the grouped GEMMs decode their tiles with (one entry per
+// 128-row tile, or per pair of them, of every expert).
 template <int NT>
 __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
-                                                  int32_t* ptile_start, int T, int E, int shared,
-                                                  int32_t (*wsum)[32]) {
+                                                  int32_t* ptile_start, int4* tile_info, int4* ptile_info, int T,
+                                                  int E, int shared, int32_t (*wsum)[32]) {
   constexpr int PER = (1024 + NT - 1) / NT;   // consecutive experts per thread
   constexpr int NW = NT / 32;
   const int n = E + shared;
@@ -362,6 +364,8 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
       offsets[e] = bc;
       mtile_start[e] = bm;
       ptile_start[e] = bp;
+      for (int g = 0; g < mt; ++g) tile_info[bm + g] = make_int4(e, bm, c[j], bc);
+      for (int g = 0; g < (mt + 1) / 2; ++g) ptile_info[bp + g] = make_int4(e, bp, c[j], bc);
     }
     bc += c[j];
     bm += mt;

@@ -114,8 +114,9 @@ def test_dense_gemm_validation_without_a_device(L):
     assert L.moe_gemm_workspace_bytes(4, 100, 128) == 0          # N % 128
     assert L.moe_gemm_workspace_bytes(4, 128, 96) == 0           # K % 128
     n = L.moe_gemm_workspace_bytes(300, 256, 512)
-    # status + bookkeeping, 3 row tiles x 4 K-blocks of 512-byte atoms, 1 n-tile x 4 of 1 KB units
-    assert n == 5 * 256 + 3 * 4 * 512 + 4 * 1024
+    # status + bookkeeping + the 3-entry row-tile table, 3 row tiles x 4 K-blocks of 512-byte
+    # atoms, 1 n-tile x 4 of 1 KB units
+    assert n == 6 * 256 + 3 * 4 * 512 + 4 * 1024
     null = [None] * 6
     assert L.moe_gemm_fp8_fp4(4, 100, 128, *null, 0, None) == binding.MOE_ERR_UNSUPPORTED_SHAPE
     assert L.moe_gemm_fp8_fp4(4, 128, 128, *null, 0, None) == binding.MOE_ERR_INVALID_ARG
