@@ -49,6 +49,17 @@ __device__ __forceinline__ int4 ld_cg_v4(const int4* p) {
   return v;
 }
 
+// Programmatic dependent launch.  wait: block until the previous kernel of the stream has
+// finished and its writes are visible (returns at once when this grid was launched without
+// the attribute).  launch_dependents: this CTA no longer holds back the next kernel's launch.
+// Every kernel of the forward calls wait before it reads anything an earlier kernel wrote and
+// only then launch_dependents, so when a kernel starts, all kernels before its predecessor
+// have finished.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // gpu-scope acquire / release accesses for grid-wide synchronisation
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;

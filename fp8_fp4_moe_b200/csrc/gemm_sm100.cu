@@ -429,31 +429,56 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       uint32_t phase = 0;
       bool ok = true;
       bool withhold = p.inject_fault != 0 && cta == 0;
+      // A rows of a tile that belong to its expert decide the A box height; the MMA still
+      // reads 128 rows, the rest are leftovers whose accumulator rows are dropped.  (A
+      // 16-row A region only ever gets the 16-row box.)
+      auto a_box_of = [&](const TileCoord& c) {
+        const int rows_here = min(BM, c.count - c.mt * BM);
+        return kATileBytes <= 16 * BK || rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
+      };
+      auto load_b = [&](const TileCoord& c, int st, int kt) {
+        if constexpr (MODE == 1) {
+          const int brow = c.e * p.rows_b + c.nt * 128;
+          tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);
+          tma_load_2d(b_s + st * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full[st]);
+        } else {
+          const int brow = c.e * p.rows_b + c.nt * BN;
+          tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);
+        }
+      };
+      // The weights and the tile table were written before the previous kernel started, so
+      // the first tile's first stages request their weight tiles before waiting for it; the
+      // A rows and all scale factors follow the wait.  (Not with the withheld-stage test hook,
+      // whose stage must stay empty.)
+      int npre = 0;
+      if (cta < total_tiles && !withhold) {
+        const TileCoord c0 = decode_tile(p, cta);
+        const uint32_t a_box = 16u << a_box_of(c0);
+        npre = min(S, KT);
+        for (int kt = 0; kt < npre; ++kt) {       // first use of these stages: nothing to wait for
+          mbar_arrive_expect_tx(&full[kt], kStageTxBytes - BM * BK + a_box * BK);
+          load_b(c0, kt, kt);
+        }
+      }
+      griddep_wait();
+      griddep_launch_dependents();
       for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
         const TileCoord c = decode_tile(p, tile);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
-        const int rows_here = min(BM, c.count - c.mt * BM);
-        // (a 16-row A region only ever gets the 16-row box)
-        const int a_sel = kATileBytes <= 16 * BK || rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
+        const int a_sel = a_box_of(c);
         const uint32_t a_box = 16u << a_sel;
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
+          const bool pre = tile == cta && kt < npre;   // weight tile already requested
+          if (!pre && !mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
           if (withhold) {
             withhold = false;            // test hook: this stage never fills
           } else {
-            // A rows of this tile that belong to the expert decide the box height; the MMA
-            // still reads 128 rows, the rest are leftovers whose accumulator rows are dropped
-            mbar_arrive_expect_tx(&full[stage], kStageTxBytes - BM * BK + a_box * BK);
-            tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
-            if constexpr (MODE == 1) {
-              const int brow = c.e * p.rows_b + c.nt * 128;
-              tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full[stage]);
-              tma_load_2d(b_s + stage * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full[stage]);
-            } else {
-              const int brow = c.e * p.rows_b + c.nt * BN;
-              tma_load_2d(b_s + stage * kBTileBytes, &tmB, kt * BK, brow, &full[stage]);
+            if (!pre) {
+              mbar_arrive_expect_tx(&full[stage], kStageTxBytes - BM * BK + a_box * BK);
+              load_b(c, stage, kt);
             }
+            tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
             bulk_load(sfa_s + stage * kSfaBytes, sfa_tile + kt * kSfaBytes, kSfaBytes, &full[stage]);
             bulk_load(sfb_s + stage * kSfbBytes, sfb_tile + kt * kSfbBytes, kSfbBytes, &full[stage]);
             fills[stage] += 1;
@@ -645,6 +670,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmSfa, const __grid_constant__ CUtensorMap tmSfb,
                              const GemmArgs p) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_s = smem + PairSmem::a;
@@ -809,6 +836,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 __global__ void __launch_bounds__(256) tile_weight_scales_kernel(const uint8_t* __restrict__ src,
                                                                  uint8_t* __restrict__ dst, int rows_b, int K,
                                                                  int n_tiles_n, int mode, int N) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ uint32_t sm[];                // [128 rows][K/128 words]
   const int kw = K / 128;
   const int e = blockIdx.y;
@@ -983,6 +1012,8 @@ __device__ __forceinline__ void router_tc_item(const CUtensorMap& tmX, const CUt
 __global__ void __launch_bounds__(kRouterThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
                      const __grid_constant__ CUtensorMap tmWlo, const RouterArgs p) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + RouterSmem::misc);
@@ -1005,6 +1036,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 // W fp32 -> (hi, lo) bf16 with hi = bf16(W), lo = bf16(W - hi) (W - hi is exact in fp32).
 __global__ void split_router_weights_kernel(const float* __restrict__ W, __nv_bfloat16* __restrict__ hi,
                                             __nv_bfloat16* __restrict__ lo, long n) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
     const float w = W[i];
     const __nv_bfloat16 h = __float2bfloat16_rn(w);
@@ -1268,32 +1301,28 @@ int gemm_pair_max_clusters() {
 
 cudaError_t launch_gemm_pair_linear1(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
                                      const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
-  grouped_gemm_pair_kernel<1><<<2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s>>>(a, b, sfa, sfb, args);
-  return cudaGetLastError();
+  return launch_kernel(grouped_gemm_pair_kernel<1>, 2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s, a, b, sfa,
+                       sfb, args);
 }
 
 cudaError_t launch_gemm_pair_linear2(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
                                      const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
-  grouped_gemm_pair_kernel<2><<<2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s>>>(a, b, sfa, sfb, args);
-  return cudaGetLastError();
+  return launch_kernel(grouped_gemm_pair_kernel<2>, 2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s, a, b, sfa,
+                       sfb, args);
 }
 
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s, bool few_rows) {
   if (few_rows)
-    grouped_gemm_kernel<1, SmallSmem><<<grid, kGemmThreads, gemm_small_smem_bytes(), s>>>(a, b, args);
-  else
-    grouped_gemm_kernel<1, SmemLayout><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
-  return cudaGetLastError();
+    return launch_kernel(grouped_gemm_kernel<1, SmallSmem>, grid, kGemmThreads, gemm_small_smem_bytes(), s, a, b, args);
+  return launch_kernel(grouped_gemm_kernel<1, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s, a, b, args);
 }
 
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s, bool few_rows) {
   if (few_rows)
-    grouped_gemm_kernel<2, SmallSmem><<<grid, kGemmThreads, gemm_small_smem_bytes(), s>>>(a, b, args);
-  else
-    grouped_gemm_kernel<2, SmemLayout><<<grid, kGemmThreads, gemm_smem_bytes(), s>>>(a, b, args);
-  return cudaGetLastError();
+    return launch_kernel(grouped_gemm_kernel<2, SmallSmem>, grid, kGemmThreads, gemm_small_smem_bytes(), s, a, b, args);
+  return launch_kernel(grouped_gemm_kernel<2, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s, a, b, args);
 }
 
 cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
@@ -1302,8 +1331,7 @@ cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_ex
   const size_t smem = (size_t)128 * (K / 128) * 4;
   if (smem > 128 * 1024) return cudaErrorInvalidValue;
   dim3 grid(groups, n_experts);
-  tile_weight_scales_kernel<<<grid, 256, smem, s>>>(src, dst, rows_b, K, n_tiles_n, mode, N);
-  return cudaGetLastError();
+  return launch_kernel(tile_weight_scales_kernel, grid, 256, smem, s, src, dst, rows_b, K, n_tiles_n, mode, N);
 }
 
 }  // namespace moe

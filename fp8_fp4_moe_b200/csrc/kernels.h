@@ -5,7 +5,30 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
+
+// Programmatic dependent launch of the forward's kernels: while switched on (per host thread),
+// the launchers below ask for it.  Every kernel they launch waits on the device for its
+// predecessor before reading what earlier kernels wrote (griddep_wait in common.cuh).
+void set_dependent_launch(bool on);
+bool dependent_launch();
+template <class... KArgs, class... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent_launch() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // 2-D tiled tensor map (cuTensorMapEncodeTiled through the runtime's driver entry point):
 // dims {inner, outer}, row pitch in bytes, box {box_inner, box_outer}.  MOE_OK or MOE_ERR_CUDA.

@@ -31,6 +31,7 @@ struct moe_plan_s {
   int swap_rows = 0;
   int pair_mode = 0;                // MOE_OPT_PAIR_TILES
   int fused = 0;                    // MOE_OPT_FUSED
+  int dep_launch = 1;               // MOE_OPT_DEPENDENT_LAUNCH
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
@@ -223,6 +224,9 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
   int rc = run_router(p, x, W_router, s);
   if (rc != MOE_OK) return rc;
   mark(p, 1 + MOE_PHASE_ROUTER, s);
+  // every later kernel of the forward may start before its predecessor ends (it waits for it
+  // on the device); not between the per-phase events
+  set_dependent_launch(p->dep_launch != 0 && !p->phase_events);
   if (p->T <= 32) {
     // one token group: top-k, ranks and the scans in one block (reported under top-k)
     if ((e = launch_topk_scan_one_group(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
@@ -338,9 +342,15 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
 }
 
 // The forward's launch sequence on stream s (TMA maps already current).
+// Plain stream order again when the forward's launch sequence ends, on every return path.
+struct DependentLaunchOff {
+  ~DependentLaunchOff() { set_dependent_launch(false); }
+};
+
 int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const float* bias,
                    const uint8_t* W1_scales, const uint8_t* W2_scales, void* out, cudaStream_t s) {
   if (p->fused) return launch_fused(p, x, W_router, bias, W1_scales, W2_scales, out, s);
+  DependentLaunchOff restore;
   int rc = run_front(p, x, W_router, bias, s);
   if (rc != MOE_OK) return rc;
   if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
@@ -522,6 +532,10 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       if (value == 1 && p->ws && fused_max_ctas() < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
       p->fused = (int)value;
+      return MOE_OK;
+    case MOE_OPT_DEPENDENT_LAUNCH:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->dep_launch = (int)value;
       return MOE_OK;
     case MOE_OPT_PAIR_TILES:
       if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;

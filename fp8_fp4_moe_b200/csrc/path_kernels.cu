@@ -22,6 +22,8 @@ template <int ET>
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ W, float* __restrict__ logits,
                                                             int T, int H, int E) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int TT = 64, KC = 32;
   constexpr int EPT = ET / 16;           // experts per thread
   __shared__ float xs[KC][TT + 1];
@@ -80,12 +82,16 @@ template <int EC>
 __global__ void __launch_bounds__(256) router_logits_warp_kernel(const uint16_t* __restrict__ x,
                                                                  const float* __restrict__ W,
                                                                  float* __restrict__ logits, int T, int H, int E) {
+  griddep_wait();
+  griddep_launch_dependents();
   router_warp_items<EC>(x, W, logits, T, H, E, (long)blockIdx.x * 8 + threadIdx.x / 32, (long)gridDim.x * 8);
 }
 
 __global__ void __launch_bounds__(256) router_logits_split_kernel(const uint16_t* __restrict__ x,
                                                                   const float* __restrict__ W,
                                                                   float* __restrict__ logits, int T, int H, int E) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float part[8];
   router_split_block<256>(x, W, logits, T, H, E, blockIdx.x, blockIdx.y, part);
 }
@@ -98,6 +104,8 @@ constexpr int kSmemRouterMaxBytes = 200 * 1024;
 __global__ void __launch_bounds__(256) router_logits_smem_kernel(const uint16_t* __restrict__ x,
                                                                  const float* __restrict__ W,
                                                                  float* __restrict__ logits, int T, int H, int E) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float4 w_s4[];
   const float* w_s = reinterpret_cast<const float*>(w_s4);
   const int n4 = E * H / 4;
@@ -159,6 +167,8 @@ __global__ void __launch_bounds__(1024) topk_rank_kernel(int mode, const float* 
                                                          float* gates, int32_t* __restrict__ local_rank,
                                                          int32_t* __restrict__ group_counts, uint32_t* status,
                                                          int T, int E, int k) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ TopkSmem sm;
   topk_rank_group<1024>(blockIdx.x, mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status,
                         T, E, k, sm);
@@ -171,6 +181,8 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     float* gates, int32_t* __restrict__ local_rank, int32_t* __restrict__ group_counts, uint32_t* status,
     int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start,
     int4* tile_info, int4* ptile_info, int T, int E, int k, int shared) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ TopkSmem sm;
   __shared__ int32_t wsum[3][32];
   topk_rank_group<1024>(0, mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k,
@@ -187,6 +199,8 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
 __global__ void __launch_bounds__(256) column_scan_kernel(const int32_t* __restrict__ group_counts,
                                                           int32_t* __restrict__ group_base, int32_t* counts, int G,
                                                           int E) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int e = blockIdx.x * 8 + threadIdx.x / 32;
   if (e < E) column_scan_warp(e, group_counts, group_base, counts, G, E);
 }
@@ -194,6 +208,8 @@ __global__ void __launch_bounds__(256) column_scan_kernel(const int32_t* __restr
 __global__ void __launch_bounds__(1024) expert_scan_kernel(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
                                                            int32_t* ptile_start, int4* tile_info, int4* ptile_info,
                                                            int T, int E, int shared) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ int32_t wsum[3][32];
   expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum);
 }
@@ -207,6 +223,8 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
                                                             const int32_t* __restrict__ mtile_start,
                                                             int32_t* slot_pos, int32_t* perm, uint8_t* xq,
                                                             uint8_t* xsf, int T, int H, int E, int k, int shared) {
+  griddep_wait();
+  griddep_launch_dependents();
   scatter_item((long)blockIdx.x * 8 + threadIdx.x / 32, x, topk_ids, local_rank, group_base, offsets, mtile_start,
                slot_pos, perm, xq, xsf, T, H, E, k, shared);
 }
@@ -250,6 +268,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                                                       const int32_t* __restrict__ slot_pos,
                                                       const float* __restrict__ gates, uint16_t* __restrict__ out,
                                                       int T, int H, int k, int shared) {
+  griddep_wait();
+  griddep_launch_dependents();
   combine_item<KMAX>((long)blockIdx.x * 8 + threadIdx.x / 32, y, slot_pos, gates, out, T, H, k, shared);
 }
 
@@ -265,7 +285,12 @@ __global__ void __launch_bounds__(256) update_bias_kernel(float* bias, const int
   }
 }
 
+thread_local bool g_dependent_launch = false;
+
 }  // namespace
+
+void set_dependent_launch(bool on) { g_dependent_launch = on; }
+bool dependent_launch() { return g_dependent_launch; }
 
 cudaError_t launch_update_bias(float* bias, const int32_t* counts, int T, int k, int E, float gamma,
                                cudaStream_t s) {
@@ -314,9 +339,8 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
                              int k, cudaStream_t s) {
   if (n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
   const int G = (T + 31) / 32;
-  topk_rank_kernel<<<G, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status,
-                                      T, E, k);
-  return cudaGetLastError();
+  return launch_kernel(topk_rank_kernel, G, 1024, 0, s, mode, logits, n_parts, bias, topk_ids, gates, local_rank,
+                       group_counts, status, T, E, k);
 }
 
 cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
@@ -325,20 +349,19 @@ cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_part
                                       int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
                                       int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
   if (T > 32 || n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
-  topk_scan_one_group_kernel<<<1, 1024, 0, s>>>(mode, logits, n_parts, bias, topk_ids, gates, local_rank,
-                                                 group_counts, status, group_base, counts, offsets, mtile_start,
-                                                 ptile_start, tile_info, ptile_info, T, E, k, shared);
-  return cudaGetLastError();
+  return launch_kernel(topk_scan_one_group_kernel, 1, 1024, 0, s, mode, logits, n_parts, bias, topk_ids, gates,
+                       local_rank, group_counts, status, group_base, counts, offsets, mtile_start, ptile_start,
+                       tile_info, ptile_info, T, E, k, shared);
 }
 
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
                                  int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
   const int G = (T + 31) / 32;
-  column_scan_kernel<<<(E + 7) / 8, 256, 0, s>>>(group_counts, group_base, counts, G, E);
-  expert_scan_kernel<<<1, 1024, 0, s>>>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E,
-                                        shared);
-  return cudaGetLastError();
+  cudaError_t e = launch_kernel(column_scan_kernel, (E + 7) / 8, 256, 0, s, group_counts, group_base, counts, G, E);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(expert_scan_kernel, 1, 1024, 0, s, counts, offsets, mtile_start, ptile_start, tile_info,
+                       ptile_info, T, E, shared);
 }
 
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
@@ -346,10 +369,8 @@ cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, con
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
                                  int k, int shared, cudaStream_t s) {
   const long items = (long)T * (x == nullptr ? 1 : (H + 255) / 256);
-  scatter_quant_kernel<<<(unsigned)((items + 7) / 8), 256, 0, s>>>(x, topk_ids, local_rank, group_base, offsets,
-                                                                   mtile_start,
-                                                   slot_pos, perm, xq, xsf, T, H, E, k, shared);
-  return cudaGetLastError();
+  return launch_kernel(scatter_quant_kernel, (unsigned)((items + 7) / 8), 256, 0, s, x, topk_ids, local_rank,
+                       group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared);
 }
 
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s) {
@@ -361,11 +382,8 @@ cudaError_t launch_combine(const uint16_t* y, const int32_t* slot_pos, const flo
                            int H, int k, int shared, cudaStream_t s) {
   const long items = (long)T * ((H + 255) / 256);
   const unsigned grid = (unsigned)((items + 7) / 8);
-  if (k <= 2) combine_kernel<2><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
-  else if (k <= 4) combine_kernel<4><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
-  else if (k <= 8) combine_kernel<8><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
-  else combine_kernel<16><<<grid, 256, 0, s>>>(y, slot_pos, gates, out, T, H, k, shared);
-  return cudaGetLastError();
+  auto kern = k <= 2 ? combine_kernel<2> : k <= 4 ? combine_kernel<4> : k <= 8 ? combine_kernel<8> : combine_kernel<16>;
+  return launch_kernel(kern, grid, 256, 0, s, y, slot_pos, gates, out, T, H, k, shared);
 }
 
 }  // namespace moe

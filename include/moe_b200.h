@@ -101,7 +101,7 @@ enum moe_option {
                                   M = 256 MMA across the pair, each CTA loading half of
                                   the weight tile): 0 (default) = never, 1 = when the
                                   experts average >= 256 rows (T*k >= 256*E), 2 = always */
-  MOE_OPT_FUSED = 10           /* 1 = moe_forward runs every step (router, top-k, dispatch
+  MOE_OPT_FUSED = 10,          /* 1 = moe_forward runs every step (router, top-k, dispatch
                                   scans, scatter + quantisation, linear1, linear2, combine)
                                   in ONE persistent cooperative kernel, one CTA per SM,
                                   the steps separated by grid-wide barriers (bounded
@@ -111,6 +111,12 @@ enum moe_option {
                                   T*E <= 4096, warp per token and expert chunk otherwise).
                                   moe_phase_times reports the whole kernel under the router
                                   phase.  No CUDA graph is recorded.  Default 0.          */
+  MOE_OPT_DEPENDENT_LAUNCH = 11 /* 1 (default): the kernels after the first of a
+                                  moe_forward are launched as programmatic dependents
+                                  (each waits on the device for its predecessor; the
+                                  grouped GEMMs request their first weight tiles before
+                                  that wait).  0 = plain stream order.  Off while
+                                  MOE_OPT_PHASE_EVENTS is 1.                              */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -97,6 +97,9 @@ def test_options_and_unbound_plan(L):
     for v in (0, 1):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_FUSED, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_FUSED, 2) == binding.MOE_ERR_INVALID_ARG
+    for v in (0, 1):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, v) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, 2) == binding.MOE_ERR_INVALID_ARG
     # no workspace bound yet: every compute entry point refuses before touching a device
     null = [None] * 9
     assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE

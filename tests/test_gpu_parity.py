@@ -450,6 +450,30 @@ def test_graph_replay_matches_direct_launches(cuda_lib):
     assert p.check_status()[0] == 0
 
 
+@pytest.mark.parametrize("name", ["t16_shared", "dsv3_like", "tc_router", "ragged_shared"])
+def test_dependent_launch_matches_plain_stream_order(cuda_lib, name):
+    # kernels that start early and wait on the device give the same bits as plain stream order,
+    # with and without a recorded graph, with the weight scales re-laid out in the middle of
+    # every forward (the default) and with that step skipped (static weights)
+    w = SMALL[name]
+    d = to_device(make_case(w, seed=21, screened=False))
+    p = plan_for(w)
+    p.set_option(binding.MOE_OPT_DEPENDENT_LAUNCH, 0)
+    ref = p.forward(**d).clone()
+    p.set_option(binding.MOE_OPT_DEPENDENT_LAUNCH, 1)
+    for graph in (0, 1):
+        p.set_option(binding.MOE_OPT_GRAPH, graph)
+        for _ in range(3):
+            out = p.forward(**d)
+            assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), graph
+    p.set_option(binding.MOE_OPT_GRAPH, 0)
+    p.set_option(binding.MOE_OPT_STATIC_WEIGHTS, 1)
+    for _ in range(2):
+        out = p.forward(**d)
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    assert p.check_status()[0] == 0
+
+
 # --------------------------------------------------------------------------- failure detection
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
