@@ -130,6 +130,7 @@ int moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* A, const uint8_t* A_sca
   a.n_experts = 1;
   a.rows_total = M;
   a.n_tiles_n = nt;
+  a.bn = kGemmBN;
   a.swap_rows = 0;
   a.counts = reinterpret_cast<const int32_t*>(ws + L.counts);
   a.offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);

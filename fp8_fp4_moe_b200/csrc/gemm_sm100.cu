@@ -47,8 +47,6 @@ constexpr uint32_t kAccCol = 0, kSfaCol = 256, kSfbCol = 264;
 constexpr uint32_t kATileBytes = BM * BK;            // 16 KB
 constexpr uint32_t kBTileBytes = BN * BK;            // 32 KB in shared memory (unpacked FP4)
 constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
-// Transaction bytes per stage: A 16 KB, B counted at 4 bits per element (16 KB), scale atoms.
-constexpr uint32_t kStageTxBytes = BM * BK + BN * BK / 2 + kSfaBytes + kSfbBytes;
 
 // Shared memory of the single-CTA grouped GEMM: STAGES pipeline stages with an A region of
 // A_BYTES each, and (STAGING) a 2 KB per-warp buffer the epilogue stores go through.
@@ -101,22 +99,27 @@ __device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
   return c;
 }
 
-// Accumulator slots: TMEM columns [0, 128) and [128, 256).  A tile with at most
-// swap_rows rows of its expert is computed transposed (weights as the M = 128
-// operand, the tile's tokens as N = 32 or 64) into one slot, alternating between
-// the two; any other tile takes both slots (M = 128 tokens, N = 256).  The MMA
-// issuer and the epilogue walk the same tile sequence and keep one use counter
-// per slot, so both derive the same mbarrier parities.
+// Accumulator slots.  With 256-row weight tiles (every linear1, linear2 by default) the
+// slots are TMEM columns [0, 128) and [128, 256) and the scale factors sit at 256..271: a
+// tile with at most swap_rows rows of its expert is computed transposed (weights as the
+// M = 128 operand, the tile's tokens as N = 32 or 64) into one slot, alternating between the
+// two, and any other tile takes both slots (M = 128 tokens, N = 256).  With 224-row weight
+// tiles (linear2, DOUBLE) the slots are [0, 224) and [256, 480), the scale factors sit at
+// 224..239, and every tile takes one slot, alternating: the epilogue drains one tile while
+// the MMAs of the next accumulate into the other.  The MMA issuer and the epilogue walk the
+// same tile sequence and keep one use counter per slot, so both derive the same mbarrier
+// parities.
 struct SlotPlan {
   bool swap;
   int lo, hi;        // slots [lo, hi] this tile uses
   int nt_tok;        // swapped tiles: token columns (MMA N)
 };
+template <bool DOUBLE>
 __device__ __forceinline__ SlotPlan plan_slots(const GemmArgs& p, const TileCoord& c, int& next_slot) {
   SlotPlan s;
   s.swap = c.rows <= p.swap_rows;
   s.nt_tok = c.rows <= 32 ? 32 : 64;
-  if (s.swap) {
+  if (s.swap || DOUBLE) {
     s.lo = s.hi = next_slot;
     next_slot ^= 1;
   } else {
@@ -125,6 +128,15 @@ __device__ __forceinline__ SlotPlan plan_slots(const GemmArgs& p, const TileCoor
   }
   return s;
 }
+// TMEM column layout for a weight-tile height NB (256, or 224 for double-buffered linear2).
+template <int NB>
+struct TmemMap {
+  static constexpr bool kDouble = NB < 256;
+  static constexpr uint32_t slot_stride = kDouble ? 256 : 128;
+  static constexpr uint32_t sfa = kDouble ? 224 : 256;
+  static constexpr uint32_t sfb = sfa + 8;              // two atoms: sfb, sfb + 4
+  static_assert(NB % 32 == 0 && NB >= 160 && NB <= 256, "weight tile height");
+};
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart.
@@ -183,35 +195,41 @@ __device__ __forceinline__ void store_rows_64b(uint8_t* buf, const uint4 (&v)[4]
   __syncwarp();
 }
 
-// Release the accumulator: both slots of this CTA, or (CTA pairs) the rank-0 CTA's barrier
-// through its cluster-window address.
+// Release the accumulator: both slots of this CTA (NB = 256), the tile's own slot (acce
+// points at it; NB < 256), or (CTA pairs) the rank-0 CTA's barrier through its cluster-window
+// address.
+template <int NB>
 __device__ __forceinline__ void release_acc(uint64_t* acce, uint32_t acce_remote) {
   if (acce_remote != 0) {
     mbar_arrive_cluster(acce_remote);
+  } else if (NB < 256) {
+    mbar_arrive(acce);
   } else {
     mbar_arrive(&acce[0]);
     mbar_arrive(&acce[1]);
   }
 }
 
-template <int MODE>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t tmem_base, int q,
+// One tile's epilogue; `acc` = TMEM address (lane 0) of the tile's accumulator.
+template <int MODE, int NB = 256>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t acc, int q,
                                               int half, int lane, uint64_t* acce, uint32_t acce_remote,
                                               float* amax_s, int buf, uint8_t* obuf) {
   const int m = q * 32 + lane;                         // accumulator row = TMEM lane
-  const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+  const uint32_t t_row = acc + ((uint32_t)(q * 32) << 16);
   const bool valid = c.mt * BM + m < c.count;
   if constexpr (MODE == 1) {
     // this warp: h channels [64*half, 64*half + 64) of the tile's 128
     uint32_t g[64], u[64];
-    tmem_ld_32x32b_x32(t_row + kAccCol + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-    tmem_ld_32x32b_x32(t_row + kAccCol + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
-    tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-    tmem_ld_32x32b_x32(t_row + kAccCol + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+    static_assert(NB == 256, "linear1 tiles hold 128 gate and 128 up rows");
+    tmem_ld_32x32b_x32(t_row + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+    tmem_ld_32x32b_x32(t_row + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+    tmem_ld_32x32b_x32(t_row + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+    tmem_ld_32x32b_x32(t_row + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) release_acc(acce, acce_remote);     // accumulator may be overwritten now
+    if (lane == 0) release_acc<NB>(acce, acce_remote);     // accumulator may be overwritten now
     float h[64];
     float amax = 0.f;
 #pragma unroll
@@ -245,27 +263,30 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
       }
     }
   } else {
-    // this warp: output columns [128*half, 128*half + 128)
+    // this warp: output columns [128*half, min(128*half + 128, NB)) of the tile
+    const int nch = half == 0 ? 4 : (NB - 128) / 32;   // 32-column chunks (warp-uniform)
     uint32_t packed[64];
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(t_row + kAccCol + half * 128 + ch * 32, r);
-      tmem_ld_wait();
+      if (ch < nch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + half * 128 + ch * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        packed[ch * 16 + i] = *reinterpret_cast<uint32_t*>(&b2);
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          packed[ch * 16 + i] = *reinterpret_cast<uint32_t*>(&b2);
+        }
       }
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) release_acc(acce, acce_remote);
-    const int col0 = c.nt * BN + half * 128;
+    if (lane == 0) release_acc<NB>(acce, acce_remote);
+    const int col0 = c.nt * NB + half * 128;
     uint8_t* dst0 = reinterpret_cast<uint8_t*>(p.y + (long)(c.row0 + q * 32) * p.N + col0);
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
-      if (col0 + ch * 32 < p.N) {                      // warp-uniform column tail
+      if (ch < nch && col0 + ch * 32 < p.N) {          // warp-uniform column tail
         uint4 w[4];
 #pragma unroll
         for (int v = 0; v < 4; ++v)
@@ -302,11 +323,12 @@ __device__ __forceinline__ float warp_transpose_max(float (&a)[TW], int lane) {
 //   linear1: gate accumulator in slot columns [0, NT), up in [64, 64 + NT); warp (q, half)
 //            owns channels q*32 + lane of the tile's 128 and tokens [half*NT/2, half*NT/2 + NT/2);
 //            the per-token amax over the 128 channels goes through shared memory.
-//   linear2: rows 0..127 of the 256-row weight tile in slot columns [0, NT), rows 128..255 in
-//            [64, 64 + NT); warp (q, half) owns output channels half*128 + q*32 + lane, all tokens.
+//   linear2: rows 0..127 of the NB-row weight tile in slot columns [0, NT), rows 128..NB-1 in
+//            [64, 64 + NT) (the MMA also covers rows NB..255 of the stage, which are dropped);
+//            warp (q, half) owns output channels half*128 + q*32 + lane, all tokens.
 // Per token, a warp's 32 channels are consecutive in the output row: one store instruction
 // covers 32 bytes (linear1) or 64 bytes (linear2).
-template <int MODE, int NT>
+template <int MODE, int NT, int NB = 256>
 __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord& c, uint32_t acc, int q, int half,
                                               int lane, uint64_t* acce_slot, float* amax_s, int buf) {
   const uint32_t t_lane = acc + ((uint32_t)(q * 32) << 16);
@@ -359,8 +381,9 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(acce_slot);
-    const int col = c.nt * BN + half * 128 + q * 32 + lane;
-    if (col < p.N) {
+    const int local = half * 128 + q * 32 + lane;     // weight row within the tile
+    const int col = c.nt * NB + local;
+    if (local < NB && col < p.N) {
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.y) + (long)c.row0 * p.N + col;
 #pragma unroll
       for (int j = 0; j < NT; ++j)
@@ -373,11 +396,17 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord
 // with `tmem_base` holding 512 allocated TMEM columns and `smem` the 1024-aligned dynamic
 // shared memory.  Initialises its barriers on entry and invalidates them on exit, so the
 // same CTA may run it again (the single persistent forward runs linear1, then linear2).
-template <int MODE, class L = SmemLayout>
+// NB: weight rows per tile (linear2 may use 224, whose accumulator is double-buffered; tmB's
+// box must then be 224 rows high and the weight scale units laid out for 224-row tiles).
+template <int MODE, class L = SmemLayout, int NB = 256>
 __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& tmB, const GemmArgs& p,
                                           uint8_t* smem, uint32_t tmem_base, int cta, int n_ctas) {
+  static_assert(MODE == 2 || NB == 256, "linear1 tiles are 256 weight rows");
+  using TM = TmemMap<NB>;
   constexpr int S = L::kStages;
   constexpr uint32_t kATileBytes = L::kABytes;
+  // bytes one stage's copies bring: A rows (box height set per tile), weights, scale factors
+  constexpr uint32_t kStageTxNoA = NB * BK / 2 + kSfaBytes + kSfbBytes;
   uint8_t* a_s = smem + L::a;
   uint8_t* b_s = smem + L::b;
   uint8_t* sfa_s = smem + L::sfa;
@@ -442,7 +471,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
           tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);
           tma_load_2d(b_s + st * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full[st]);
         } else {
-          const int brow = c.e * p.rows_b + c.nt * BN;
+          const int brow = c.e * p.rows_b + c.nt * NB;
           tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);
         }
       };
@@ -456,7 +485,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
         const uint32_t a_box = 16u << a_box_of(c0);
         npre = min(S, KT);
         for (int kt = 0; kt < npre; ++kt) {       // first use of these stages: nothing to wait for
-          mbar_arrive_expect_tx(&full[kt], kStageTxBytes - BM * BK + a_box * BK);
+          mbar_arrive_expect_tx(&full[kt], kStageTxNoA + a_box * BK);
           load_b(c0, kt, kt);
         }
       }
@@ -475,7 +504,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
             withhold = false;            // test hook: this stage never fills
           } else {
             if (!pre) {
-              mbar_arrive_expect_tx(&full[stage], kStageTxBytes - BM * BK + a_box * BK);
+              mbar_arrive_expect_tx(&full[stage], kStageTxNoA + a_box * BK);
               load_b(c, stage, kt);
             }
             tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
@@ -504,21 +533,22 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       bool ok = true;
       for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
         const TileCoord c = decode_tile(p, tile);
-        const SlotPlan sp = plan_slots(p, c, next_slot);
+        const SlotPlan sp = plan_slots<TM::kDouble>(p, c, next_slot);
         for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
           ok = mbar_wait(&acce[sl], ((sl ? uses1 : uses0) & 1) ^ 1, ctl, kWhereGemmMma);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t acc = tmem_base + kAccCol + sp.lo * 128;
+        const uint32_t acc = tmem_base + kAccCol + sp.lo * TM::slot_stride;
+        const uint32_t sfa_t = tmem_base + TM::sfa, sfb_t = tmem_base + TM::sfb;
         const uint32_t id_swap0 = idesc_mxf8f6f4(BM, sp.nt_tok, 0, 0, kFmtE2M1, kFmtE4M3);
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&full[stage], phase, ctl, kWhereGemmMma + 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sfa_addr = smem_u32(sfa_s + stage * kSfaBytes);
           const uint32_t sfb_addr = smem_u32(sfb_s + stage * kSfbBytes);
-          tc_cp_32x128b_warpx4(tmem_base + kSfaCol, sf_desc(sfa_addr));
-          tc_cp_32x128b_warpx4(tmem_base + kSfbCol, sf_desc(sfb_addr));
-          tc_cp_32x128b_warpx4(tmem_base + kSfbCol + 4, sf_desc(sfb_addr + 512));
+          tc_cp_32x128b_warpx4(sfa_t, sf_desc(sfa_addr));
+          tc_cp_32x128b_warpx4(sfb_t, sf_desc(sfb_addr));
+          tc_cp_32x128b_warpx4(sfb_t + 4, sf_desc(sfb_addr + 512));
           const uint32_t a_addr = smem_u32(a_s + stage * kATileBytes);
           const uint32_t b_addr = smem_u32(b_s + stage * kBTileBytes);
           if (sp.swap) {
@@ -527,18 +557,16 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
 #pragma unroll
             for (int kb = 0; kb < BK / 32; ++kb) {
               const uint32_t id = id_swap0 | ((uint32_t)kb << 4) | ((uint32_t)kb << 29);
-              tc_mma_mxf8f6f4(acc, sw128_desc(b_addr + kb * 32), sw128_desc(a_addr + kb * 32), id,
-                              tmem_base + kSfbCol, tmem_base + kSfaCol, (kt | kb) != 0);
-              tc_mma_mxf8f6f4(acc + 64, sw128_desc(b_addr + kBTileBytes / 2 + kb * 32),
-                              sw128_desc(a_addr + kb * 32), id, tmem_base + kSfbCol + 4, tmem_base + kSfaCol,
+              tc_mma_mxf8f6f4(acc, sw128_desc(b_addr + kb * 32), sw128_desc(a_addr + kb * 32), id, sfb_t, sfa_t,
                               (kt | kb) != 0);
+              tc_mma_mxf8f6f4(acc + 64, sw128_desc(b_addr + kBTileBytes / 2 + kb * 32),
+                              sw128_desc(a_addr + kb * 32), id, sfb_t + 4, sfa_t, (kt | kb) != 0);
             }
           } else {
 #pragma unroll
             for (int kb = 0; kb < BK / 32; ++kb) {
               tc_mma_mxf8f6f4(acc, sw128_desc(a_addr + kb * 32), sw128_desc(b_addr + kb * 32),
-                              idesc_mxf8f6f4(BM, BN, kb, kb), tmem_base + kSfaCol, tmem_base + kSfbCol,
-                              (kt | kb) != 0);
+                              idesc_mxf8f6f4(BM, NB, kb, kb), sfa_t, sfb_t, (kt | kb) != 0);
             }
           }
           tc_commit(&empty[stage]);
@@ -563,21 +591,22 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
     int buf = 0;
     for (int tile = cta; tile < total_tiles; tile += n_ctas) {
       const TileCoord c = decode_tile(p, tile);
-      const SlotPlan sp = plan_slots(p, c, next_slot);
+      const SlotPlan sp = plan_slots<TM::kDouble>(p, c, next_slot);
       bool ok = true;
       for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
         ok = mbar_wait(&accf[sl], (sl ? uses1 : uses0) & 1, ctl, kWhereGemmEpilogue);
       // epilogue-uniform decision: tcgen05.ld below is .sync.aligned and the epilogue syncs
       if (!epi_all(ok)) break;
       tc_fence_after();
+      const uint32_t acc = tmem_base + kAccCol + sp.lo * TM::slot_stride;
       if (sp.swap) {
-        const uint32_t acc = tmem_base + kAccCol + sp.lo * 128;
         if (sp.nt_tok == 32)
-          epilogue_swap<MODE, 32>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
+          epilogue_swap<MODE, 32, NB>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
         else
-          epilogue_swap<MODE, 64>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
+          epilogue_swap<MODE, 64, NB>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
       } else {
-        epilogue_tile<MODE>(p, c, tmem_base, q, half, lane, acce, 0u, amax_s, buf, obuf);
+        epilogue_tile<MODE, NB>(p, c, acc, q, half, lane, TM::kDouble ? &acce[sp.lo] : acce, 0u, amax_s, buf,
+                                obuf);
       }
       uses0 += sp.lo == 0;
       uses1 += sp.hi == 1;
@@ -592,14 +621,14 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
   __syncthreads();
 }
 
-template <int MODE, class L>
+template <int MODE, class L, int NB = 256>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                         const GemmArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc);
   const int warp = threadIdx.x / 32;
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -609,7 +638,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  gemm_body<MODE, L>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
+  gemm_body<MODE, L, NB>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -835,7 +864,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 // linear2 groups pair row blocks 2t and 2t+1 of a 256-row tile.
 __global__ void __launch_bounds__(256) tile_weight_scales_kernel(const uint8_t* __restrict__ src,
                                                                  uint8_t* __restrict__ dst, int rows_b, int K,
-                                                                 int n_tiles_n, int mode, int N) {
+                                                                 int n_tiles_n, int mode, int N, int tile_rows) {
   griddep_wait();
   griddep_launch_dependents();
   extern __shared__ uint32_t sm[];                // [128 rows][K/128 words]
@@ -849,10 +878,10 @@ __global__ void __launch_bounds__(256) tile_weight_scales_kernel(const uint8_t* 
     hf = grp >= ng;
     nt = grp - hf * ng;
     row_first = grp * 128;
-  } else {                                        // rows_b = H (=N): 256-row tiles, 2 halves
+  } else {                                        // rows_b = H (=N): tile_rows-row tiles, 2 halves
     nt = grp / 2;
     hf = grp % 2;
-    row_first = grp * 128;
+    row_first = nt * tile_rows + hf * 128;
   }
   const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src);
   for (int i = threadIdx.x; i < 128 * kw; i += blockDim.x) {
@@ -1169,7 +1198,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   fence_proxy_async_global();
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
   // S5 linear2
-  if (ok) gemm_body<2>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
+  if (ok) {
+    if (a.g2.bn == kGemmBN2Double)
+      gemm_body<2, SmemLayout, kGemmBN2Double>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
+    else
+      gemm_body<2>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
+  }
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
   // S6 combine
   if (ok) {
@@ -1231,6 +1265,12 @@ cudaError_t gemm_prepare_device() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmallSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_small_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmallSmem, kGemmBN2Double>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_small_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmemLayout, kGemmBN2Double>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes());
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tile_weight_scales_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
   if (e != cudaSuccess) return e;
@@ -1320,18 +1360,27 @@ cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const Gemm
 
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s, bool few_rows) {
+  constexpr int D = kGemmBN2Double;
+  if (args.bn != kGemmBN && args.bn != D) return cudaErrorInvalidValue;
   if (few_rows)
-    return launch_kernel(grouped_gemm_kernel<2, SmallSmem>, grid, kGemmThreads, gemm_small_smem_bytes(), s, a, b, args);
-  return launch_kernel(grouped_gemm_kernel<2, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s, a, b, args);
+    return args.bn == D ? launch_kernel(grouped_gemm_kernel<2, SmallSmem, D>, grid, kGemmThreads,
+                                        gemm_small_smem_bytes(), s, a, b, args)
+                        : launch_kernel(grouped_gemm_kernel<2, SmallSmem>, grid, kGemmThreads,
+                                        gemm_small_smem_bytes(), s, a, b, args);
+  return args.bn == D ? launch_kernel(grouped_gemm_kernel<2, SmemLayout, D>, grid, kGemmThreads, gemm_smem_bytes(),
+                                      s, a, b, args)
+                      : launch_kernel(grouped_gemm_kernel<2, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s,
+                                      a, b, args);
 }
 
 cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
-                                      int n_tiles_n, int mode, int N, cudaStream_t s) {
+                                      int n_tiles_n, int mode, int N, cudaStream_t s, int tile_rows) {
   const int groups = mode == 1 ? rows_b / 128 : n_tiles_n * 2;
   const size_t smem = (size_t)128 * (K / 128) * 4;
   if (smem > 128 * 1024) return cudaErrorInvalidValue;
   dim3 grid(groups, n_experts);
-  return launch_kernel(tile_weight_scales_kernel, grid, 256, smem, s, src, dst, rows_b, K, n_tiles_n, mode, N);
+  return launch_kernel(tile_weight_scales_kernel, grid, 256, smem, s, src, dst, rows_b, K, n_tiles_n, mode, N,
+                       tile_rows);
 }
 
 }  // namespace moe

@@ -41,6 +41,10 @@ constexpr int kGemmBM = 128;      // rows (tokens) per tile
 constexpr int kGemmBN = 256;      // accumulator columns per tile
 constexpr int kGemmBK = 128;      // K per pipeline stage
 constexpr int kGemmStages = 4;
+// linear2 weight tiles of 224 rows (output columns) leave TMEM room for two accumulators, so
+// the epilogue of one tile overlaps the MMAs of the next (single-CTA kernel, H a multiple of
+// 224).  Otherwise 256-row tiles with one accumulator.
+constexpr int kGemmBN2Double = 224;
 constexpr int kGemmThreads = 320; // 10 warps: TMA, MMA, 8 x epilogue
 
 // Scale-factor atoms (the unit the MMA's scale copy reads): 128 rows x 4 K-blocks
@@ -55,7 +59,8 @@ struct GemmArgs {
   int rows_b;          // B rows per expert (2I or H)
   int n_experts;       // E + shared
   int rows_total;      // R + shared * T
-  int n_tiles_n;       // linear1: I/128; linear2: ceil(H/256)
+  int n_tiles_n;       // linear1: I/128; linear2: ceil(H/bn)
+  int bn;              // linear2: weight rows (output columns) per tile, 256 or kGemmBN2Double
   int swap_rows;       // tiles with at most this many expert rows run transposed (0, 32 or 64)
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
@@ -78,9 +83,11 @@ struct GemmArgs {
 
 size_t gemm_smem_bytes();
 cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attributes
-// canonical UE8M0 weight scales [n][rows_b][K/32] -> weight scale units
+// canonical UE8M0 weight scales [n][rows_b][K/32] -> weight scale units.  mode 1: linear1
+// (128 gate + 128 up rows per tile); mode 2: linear2 with tiles of tile_rows weight rows (the
+// unit's second atom covers tile rows 128..255; rows past the tile are never used).
 cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,
-                                      int n_tiles_n, int mode, int N, cudaStream_t s);
+                                      int n_tiles_n, int mode, int N, cudaStream_t s, int tile_rows = kGemmBN);
 // A-operand tensor maps of one activation matrix with box heights 16, 32, 64, 128 rows
 // (the producer picks the smallest box that covers the tile's rows of its expert).
 struct AMaps {

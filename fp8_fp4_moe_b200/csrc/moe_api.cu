@@ -32,6 +32,7 @@ struct moe_plan_s {
   int pair_mode = 0;                // MOE_OPT_PAIR_TILES
   int fused = 0;                    // MOE_OPT_FUSED
   int dep_launch = 1;               // MOE_OPT_DEPENDENT_LAUNCH
+  int l2_tile_rows = 0;             // MOE_OPT_L2_TILE_ROWS
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
@@ -47,7 +48,7 @@ struct moe_plan_s {
   int device = -1;
   int num_sms = 0;
   alignas(64) AMaps amA1, amA2;
-  alignas(64) CUtensorMap tmB1, tmB2, tmX, tmWhi, tmWlo;
+  alignas(64) CUtensorMap tmB1, tmB2, tmB2d, tmX, tmWhi, tmWlo;   // tmB2d: 224-row boxes
   alignas(64) CUtensorMap tmB2p, tmSfa1, tmSfa2, tmSfb1, tmSfb2;   // CTA-pair GEMM operands
   const void* x_cached = nullptr;        // tmX encodes this x pointer
   const void* wr_prepared = nullptr;     // W_router the hi/lo split was made from
@@ -55,6 +56,7 @@ struct moe_plan_s {
   const void* w2_cached = nullptr;
   const void* w1s_prepared = nullptr;   // weight scales the prepared units were built from
   const void* w2s_prepared = nullptr;
+  int w2_tile_rows = 0;                // linear2 tile height the W2 scale units were laid out for
   // MOE_OPT_GRAPH: recorded launch sequences, keyed by the forward's pointers
   int use_graph = 0;
   struct GraphEntry {
@@ -126,6 +128,22 @@ int check_bound(moe_plan_t p) {
   return MOE_OK;
 }
 
+// CTA-pair GEMMs (M = 256 per pair) when experts average at least 256 rows, or when forced.
+bool use_pairs(moe_plan_t p) {
+  if (p->pair_mode == 0 || gemm_pair_max_clusters() < 1) return false;
+  return p->pair_mode == 2 || (long long)p->T * p->k >= 256ll * p->E;
+}
+
+// linear2 weight rows per tile.  224 (double-buffered accumulator) needs H % 224 == 0 and the
+// single-CTA kernel; automatic only for few tokens (T <= 16), where 224-row tiles spread the
+// experts' weight tiles more evenly over the SMs (DSV3 T = 1: 288 tiles instead of 252) --
+// with many tiles per SM the 14 % more tiles cost more than the overlap saves.
+int linear2_bn(moe_plan_t p) {
+  if (use_pairs(p) || p->H % kGemmBN2Double != 0 || p->l2_tile_rows == kGemmBN) return kGemmBN;
+  if (p->l2_tile_rows == kGemmBN2Double) return kGemmBN2Double;
+  return p->T <= 16 ? kGemmBN2Double : kGemmBN;
+}
+
 GemmArgs gemm_args(moe_plan_t p, int mode) {
   GemmArgs a{};
   a.n_experts = p->n;
@@ -144,6 +162,7 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
     a.N = p->I;
     a.rows_b = 2 * p->I;
     a.n_tiles_n = p->I / 128;
+    a.bn = kGemmBN;
     a.sfa = region<uint8_t>(p, MOE_REGION_XSF);
     a.sfb = at<uint8_t>(p, p->off_w1sf);
     a.hq = region<uint8_t>(p, MOE_REGION_HQ);
@@ -153,7 +172,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
     a.K = p->I;
     a.N = p->H;
     a.rows_b = p->H;
-    a.n_tiles_n = (p->H + kGemmBN - 1) / kGemmBN;
+    a.bn = linear2_bn(p);
+    a.n_tiles_n = (p->H + a.bn - 1) / a.bn;
     a.sfa = region<uint8_t>(p, MOE_REGION_HSF);
     a.sfb = at<uint8_t>(p, p->off_w2sf);
     a.y = region<uint16_t>(p, MOE_REGION_Y);
@@ -168,12 +188,6 @@ int gemm_grid(moe_plan_t p, int n_tiles_n) {
   int sms = p->num_sms;
   if (p->max_sms > 0 && p->max_sms < sms) sms = p->max_sms;
   return (int)(tiles < sms ? tiles : sms);
-}
-
-// CTA-pair GEMMs (M = 256 per pair) when experts average at least 256 rows, or when forced.
-bool use_pairs(moe_plan_t p) {
-  if (p->pair_mode == 0 || gemm_pair_max_clusters() < 1) return false;
-  return p->pair_mode == 2 || (long long)p->T * p->k >= 256ll * p->E;
 }
 
 int pair_grid(moe_plan_t p, int n_tiles_n) {
@@ -266,12 +280,21 @@ int prepare_weights(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_sc
   cudaError_t e = launch_tile_weight_scales(W1_scales, at<uint8_t>(p, p->off_w1sf), p->n, 2 * p->I, p->H,
                                             p->I / 128, 1, p->I, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_tile_weight_scales(W2_scales, at<uint8_t>(p, p->off_w2sf), p->n, p->H, p->I,
-                                (p->H + kGemmBN - 1) / kGemmBN, 2, p->H, s);
+  const int bn2 = linear2_bn(p);
+  e = launch_tile_weight_scales(W2_scales, at<uint8_t>(p, p->off_w2sf), p->n, p->H, p->I, (p->H + bn2 - 1) / bn2, 2,
+                                p->H, s, bn2);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   p->w1s_prepared = W1_scales;
   p->w2s_prepared = W2_scales;
+  p->w2_tile_rows = bn2;
   return MOE_OK;
+}
+
+// The prepared weight scale units are stale (new pointers, not promised static, or laid out
+// for another linear2 tile height).
+bool weights_need_prepare(moe_plan_t p, const uint8_t* W1_scales, const uint8_t* W2_scales) {
+  return !p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared ||
+         p->w2_tile_rows != linear2_bn(p);
 }
 
 // MOE_OPT_FUSED: weight preparation when needed, then every step in one cooperative launch.
@@ -292,7 +315,7 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
       p->x_cached = x;
     }
   }
-  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
+  if (weights_need_prepare(p, W1_scales, W2_scales)) {
     int rc = prepare_weights(p, W1_scales, W2_scales, s);
     if (rc != MOE_OK) return rc;
   }
@@ -332,8 +355,8 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
   if (p->max_sms > 0 && p->max_sms < ctas) ctas = p->max_sms;
   // a launch that ran out of time may have left arrivals behind
   if (cudaMemsetAsync(a.gridbar, 0, 8, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, p->tmB2, p->tmX, p->tmWhi, p->tmWlo, a, ctas, s) !=
-      cudaSuccess)
+  const CUtensorMap& b2 = a.g2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
+  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, b2, p->tmX, p->tmWhi, p->tmWlo, a, ctas, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // one kernel: its whole time is reported under the first phase
   for (int i = 1; i <= MOE_PHASE_COUNT_; ++i) mark(p, i, s);
@@ -353,7 +376,7 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
   DependentLaunchOff restore;
   int rc = run_front(p, x, W_router, bias, s);
   if (rc != MOE_OK) return rc;
-  if (!p->static_weights || W1_scales != p->w1s_prepared || W2_scales != p->w2s_prepared) {
+  if (weights_need_prepare(p, W1_scales, W2_scales)) {
     if ((rc = prepare_weights(p, W1_scales, W2_scales, s)) != MOE_OK) return rc;
   }
   mark(p, 1 + MOE_PHASE_PREPARE, s);
@@ -374,7 +397,8 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
     if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, few_rows) != cudaSuccess)
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR1, s);
-    if (launch_gemm_linear2(p->amA2, p->tmB2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
+    const CUtensorMap& b2 = a2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
+    if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR2, s);
   }
@@ -488,7 +512,8 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_ptinfo = add((size_t)p->mt_cap * 16);
   p->off_gridbar = add(8);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
-  p->off_w2sf = add((size_t)p->n * ((H + kGemmBN - 1) / kGemmBN) * (I / 128) * 1024);
+  // linear2 weight scale units for the narrower of the two tile heights (more tiles)
+  p->off_w2sf = add((size_t)p->n * ((H + kGemmBN2Double - 1) / kGemmBN2Double) * (I / 128) * 1024);
   p->off_whi = add((size_t)E * H * 2);
   p->off_wlo = add((size_t)E * H * 2);
   p->total = off;
@@ -532,6 +557,11 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       if (value == 1 && p->ws && fused_max_ctas() < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
       p->fused = (int)value;
+      return MOE_OK;
+    case MOE_OPT_L2_TILE_ROWS:
+      if (value != 0 && value != kGemmBN && value != kGemmBN2Double) return MOE_ERR_INVALID_ARG;
+      if (value == kGemmBN2Double && p->H % kGemmBN2Double != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+      p->l2_tile_rows = (int)value;
       return MOE_OK;
     case MOE_OPT_DEPENDENT_LAUNCH:
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
@@ -633,6 +663,9 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
   if (W2 != p->w2_cached) {
     rc = encode_2d(&p->tmB2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
                    128, 256);
+    if (rc == MOE_OK)
+      rc = encode_2d(&p->tmB2d, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
+                     128, kGemmBN2Double);
     if (rc == MOE_OK)
       rc = encode_2d(&p->tmB2p, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W2, p->I, (uint64_t)p->n * p->H, p->I / 2,
                      128, 128);

@@ -100,6 +100,14 @@ def test_options_and_unbound_plan(L):
     for v in (0, 1):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, 2) == binding.MOE_ERR_INVALID_ARG
+    for v in (0, 256):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, v) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, 128) == binding.MOE_ERR_INVALID_ARG
+    # H = 256 is not a multiple of 224
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, 224) == binding.MOE_ERR_UNSUPPORTED_SHAPE
+    rc, h2 = _plan(L, 64, 896, 512, 8, 2, 0)
+    assert rc == 0 and L.moe_plan_set_option(h2, binding.MOE_OPT_L2_TILE_ROWS, 224) == 0
+    L.moe_plan_destroy(h2)
     # no workspace bound yet: every compute entry point refuses before touching a device
     null = [None] * 9
     assert L.moe_forward(h, *null) == binding.MOE_ERR_WORKSPACE

@@ -12,7 +12,7 @@ import torch
 from fp8_fp4_moe_b200 import binding
 from fp8_fp4_moe_b200 import inputs as I
 
-from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, oracle_forward
+from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, oracle_forward_with_slack
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -37,14 +37,14 @@ def test_full_size_sampled_parity(cuda_lib, name, fused):
         ids = p.region("topk_ids").cpu().numpy()
         busiest = np.bincount(ids.ravel(), minlength=w.E).argmax()
         tokens = np.unique(np.append(tokens, np.nonzero((ids == busiest).any(axis=1))[0][0]))
-    ref = oracle_forward(case, w, tokens=tokens)
+    ref, slack = oracle_forward_with_slack(case, w, tokens=tokens)
     assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
     assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
     assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
     np.testing.assert_allclose(p.region("gates").cpu().numpy(), ref["gates"], rtol=GATE_RTOL, atol=GATE_ATOL)
     got = bits(out)[tokens]
-    assert_output_close(got, ref["y"], name)
+    assert_output_close(got, ref["y"], name, slack)
     assert torch.isfinite(out.float()).all()
     del p, d, out
     torch.cuda.empty_cache()

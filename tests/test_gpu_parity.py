@@ -14,7 +14,8 @@ from fp8_fp4_moe_b200 import inputs as I
 from oracle import formats as F
 from oracle import moe as M
 
-from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, oracle_forward, to_device, untile_scales
+from parity import (GATE_ATOL, GATE_RTOL, assert_output_close, bits, h_decision_range, make_case, oracle_forward,
+                    oracle_forward_with_slack, to_device, untile_scales)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,11 +34,18 @@ SMALL = {
     "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
     # T >= 256 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
     "tc_router": W("tc_router", T=300, H=1024, I_=256, E=48, k=4, shared=1, router_std=0.02, bias="uniform"),
+    # H % 224 == 0: linear2 runs 224-row weight tiles with a double-buffered accumulator
+    "h896": W("h896", T=200, H=896, I_=256, E=8, k=2, shared=1, bias="uniform"),
+    "h1792_t8": W("h1792_t8", T=8, H=1792, I_=256, E=16, k=4, shared=1, router_std=0.01, bias="uniform"),
 }
 
 
 def plan_for(w, swap_rows=None, pair_tiles=None, fused=None):
     p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+    if w.H % 224 == 0:
+        # these shapes run linear2 on 224-row weight tiles (double-buffered accumulator) at any
+        # T; by default only T <= 16 does
+        p.set_option(binding.MOE_OPT_L2_TILE_ROWS, 224)
     if swap_rows is not None:
         p.set_option(binding.MOE_OPT_SWAP_ROWS, swap_rows)
     if pair_tiles is not None:
@@ -182,7 +190,7 @@ def test_forward_matches_oracle(cuda_lib, name, swap_rows):
     p = plan_for(w, swap_rows)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    ref = oracle_forward(case, w)
+    ref, slack = oracle_forward_with_slack(case, w)
     # routing and dispatch inside the forward are bit-exact
     assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
@@ -198,10 +206,11 @@ def test_forward_matches_oracle(cuda_lib, name, swap_rows):
     if w.shared:
         R = w.T * w.k
         assert np.array_equal(xq[R:R + w.T], ref["xq"])
-    assert_output_close(bits(out), ref["y"], name)
+    assert_output_close(bits(out), ref["y"], name, slack)
 
 
-@pytest.mark.parametrize("name,swap_rows", [("ragged_shared", 64), ("ragged_shared", 0), ("dsv3_like", 64)])
+@pytest.mark.parametrize("name,swap_rows", [("ragged_shared", 64), ("ragged_shared", 0), ("dsv3_like", 64),
+                                            ("h896", 0), ("h896", 64)])
 def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows):
     w = SMALL[name]
     case = make_case(w, seed=8)
@@ -213,21 +222,22 @@ def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows):
     hsf = untile_scales(p.region("hsf").cpu().numpy(), ref["counts"], ref["offsets"])
     y = F.bf16_to_f64(bits(p.region("y")))
     offsets = ref["offsets"]
-    agree = total = 0
+    differ = ambiguous = 0
     for e, (lst, res) in ref["rows"].items():
         # oracle rows for expert e are listed in token order == dispatch order
         rows = np.arange(offsets[e], offsets[e + 1])
         assert len(rows) == len(lst)
         g_h = M.dequantize_blocks(hq[rows], hsf[rows] - 127)
-        r_h = M.dequantize_blocks(res["hq"], res["hexp"])
-        # an E4M3 code can flip by one step where fp32 and fp64 h straddle a rounding point
-        assert np.linalg.norm(g_h - r_h) <= 1e-2 * np.linalg.norm(r_h) + 1e-30, e
-        agree += int(np.sum(hq[rows] == res["hq"]))
-        total += hq[rows].size
+        # every requantised value is one a correct decision gives: the oracle's own, or where h
+        # lies on a rounding boundary (within the fp32 accumulation-order spread) its neighbour
+        lo, hi, own = h_decision_range(res["h"], res["hq"], res["hexp"])
+        assert np.all((g_h >= lo) & (g_h <= hi)), e
+        differ += int(np.sum(g_h != own))
+        ambiguous += int(np.sum(lo != hi))
         ry = res["o"]
         err = np.linalg.norm(y[rows] - ry) / max(np.linalg.norm(ry), 1e-300)
         assert err < 5e-3, (e, err)
-    assert agree / total > 0.99         # codes differ only where fp32 and fp64 h straddle a rounding point
+    assert differ <= ambiguous
 
 
 def test_forward_is_deterministic(cuda_lib):
@@ -248,10 +258,10 @@ def test_forward_all_tokens_on_one_expert(cuda_lib, pair_tiles):
     d = to_device(case)
     p = plan_for(w, pair_tiles=pair_tiles)
     out = p.forward(**d)
-    ref = oracle_forward(case, w)
+    ref, slack = oracle_forward_with_slack(case, w)
     assert ref["counts"].tolist() == [0, 0, 700, 0, 0, 0, 0, 0, 700]
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
-    assert_output_close(bits(out), ref["y"], "skew")
+    assert_output_close(bits(out), ref["y"], "skew", slack)
 
 
 def _count_mix_case(counts, H=256, I_=384, seed=3):
@@ -276,21 +286,24 @@ def _count_mix_case(counts, H=256, I_=384, seed=3):
     return w, case
 
 
-@pytest.mark.parametrize("swap_rows,pair_tiles,fused", [(64, 0, 0), (32, 0, 0), (0, 0, 0), (0, 2, 0), (0, 0, 1),
-                                                        (64, 0, 1)])
-def test_forward_tile_row_boundaries(cuda_lib, swap_rows, pair_tiles, fused):
+@pytest.mark.parametrize("swap_rows,pair_tiles,fused,H", [(64, 0, 0, 256), (32, 0, 0, 256), (0, 0, 0, 256),
+                                                          (0, 2, 0, 256), (0, 0, 1, 256), (64, 0, 1, 256),
+                                                          (0, 0, 0, 896), (64, 0, 0, 896), (0, 0, 1, 896),
+                                                          (0, 2, 0, 896)])
+def test_forward_tile_row_boundaries(cuda_lib, swap_rows, pair_tiles, fused, H):
     # expert loads on both sides of 32, 64, 128 and 256 rows (odd and even row-tile counts for
-    # the CTA-pair GEMM), plus an empty expert
+    # the CTA-pair GEMM), plus an empty expert; H = 896 gives linear2 224-row weight tiles
     counts = [1, 17, 32, 33, 64, 65, 128, 129, 0, 200, 256, 257, 384]
-    w, case = _count_mix_case(counts)
+    w, case = _count_mix_case(counts, H=H)
     d = to_device(case)
     p = plan_for(w, swap_rows, pair_tiles, fused)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    ref = oracle_forward(case, w)
+    ref, slack = oracle_forward_with_slack(case, w)
     assert ref["counts"].tolist() == counts + [w.T]
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
-    assert_output_close(bits(out), ref["y"], f"count_mix swap_rows={swap_rows} pair_tiles={pair_tiles} fused={fused}")
+    assert_output_close(bits(out), ref["y"],
+                        f"count_mix H={H} swap_rows={swap_rows} pair_tiles={pair_tiles} fused={fused}", slack)
 
 
 # CTA-pair GEMMs forced on the small shapes (auto mode uses them from 256 rows per expert on)
@@ -302,8 +315,8 @@ def test_forward_pair_tiles_match_oracle(cuda_lib, name):
     p = plan_for(w, pair_tiles=2)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    ref = oracle_forward(case, w)
-    assert_output_close(bits(out), ref["y"], name + " pairs")
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(out), ref["y"], name + " pairs", slack)
     # the single-CTA kernel forms the same products; only the fp32 summation may differ
     p1 = plan_for(w, pair_tiles=0)
     out1 = p1.forward(**d)
@@ -323,13 +336,13 @@ def test_forward_fused_matches_oracle(cuda_lib, name):
     p = plan_for(w, fused=1)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    ref = oracle_forward(case, w)
+    ref, slack = oracle_forward_with_slack(case, w)
     assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
     assert np.array_equal(p.region("counts").cpu().numpy(), ref["counts"])
     assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
     assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
     np.testing.assert_allclose(p.region("gates").cpu().numpy(), ref["gates"], rtol=GATE_RTOL, atol=GATE_ATOL)
-    assert_output_close(bits(out), ref["y"], name + " fused")
+    assert_output_close(bits(out), ref["y"], name + " fused", slack)
     # repeated launches reuse the grid barrier words
     out2 = p.forward(**d).clone()
     assert p.check_status()[0] == 0
@@ -350,7 +363,8 @@ def test_fused_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     p.set_option(binding.MOE_OPT_TIMEOUT_NS, 2_000_000_000)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    assert_output_close(bits(out), oracle_forward(case, w)["y"], "fused after timeout")
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(out), ref["y"], "fused after timeout", slack)
 
 
 def test_update_bias_matches_oracle_and_evens_out_loads(cuda_lib):
@@ -450,7 +464,7 @@ def test_graph_replay_matches_direct_launches(cuda_lib):
     assert p.check_status()[0] == 0
 
 
-@pytest.mark.parametrize("name", ["t16_shared", "dsv3_like", "tc_router", "ragged_shared"])
+@pytest.mark.parametrize("name", ["t16_shared", "dsv3_like", "tc_router", "ragged_shared", "h1792_t8"])
 def test_dependent_launch_matches_plain_stream_order(cuda_lib, name):
     # kernels that start early and wait on the device give the same bits as plain stream order,
     # with and without a recorded graph, with the weight scales re-laid out in the middle of
@@ -491,4 +505,5 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     p.set_option(binding.MOE_OPT_TIMEOUT_NS, 2_000_000_000)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
-    assert_output_close(bits(out), oracle_forward(case, w)["y"], "after timeout")
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(out), ref["y"], "after timeout", slack)
