@@ -187,12 +187,17 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
   __shared__ int32_t wsum[3][32];
   topk_rank_group<1024>(0, mode, logits, n_parts, bias, topk_ids, gates, local_rank, group_counts, status, T, E, k,
                         sm);
+  // the group's per-expert masks are still in shared memory: counts without a global round trip
+  int32_t* cnt_s = reinterpret_cast<int32_t*>(sm.mask);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    counts[e] = group_counts[e];
+    const int c = __popc(sm.mask[e]);
+    cnt_s[e] = c;
+    counts[e] = c;
     group_base[e] = 0;
   }
   __syncthreads();
-  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum);
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum,
+                          cnt_s);
 }
 
 // --------------------------------------------------------------------------- scan

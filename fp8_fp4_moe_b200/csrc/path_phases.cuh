@@ -310,11 +310,14 @@ __device__ __forceinline__ void column_scan_warp(int e, const int32_t* __restric
 
 // Called by all NT threads of one block (it synchronises them); n = E + shared <= 1024.
 // Also fills the row-tile tables the grouped GEMMs decode their tiles with (one entry per
-// 128-row tile, or per pair of them, of every expert).
+// 128-row tile, or per pair of them, of every expert).  The routed experts' counts are read
+// from cnt_src (the counts array itself, or a copy in shared memory).
 template <int NT>
 __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
                                                   int32_t* ptile_start, int4* tile_info, int4* ptile_info, int T,
-                                                  int E, int shared, int32_t (*wsum)[32]) {
+                                                  int E, int shared, int32_t (*wsum)[32],
+                                                  const int32_t* cnt_src = nullptr) {
+  if (cnt_src == nullptr) cnt_src = counts;
   constexpr int PER = (1024 + NT - 1) / NT;   // consecutive experts per thread
   constexpr int NW = NT / 32;
   const int n = E + shared;
@@ -324,7 +327,7 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int e = threadIdx.x * PER + j;
-    c[j] = e < E ? counts[e] : (e == E && shared ? T : 0);
+    c[j] = e < E ? cnt_src[e] : (e == E && shared ? T : 0);
     const int mt = (c[j] + kGemmBM - 1) / kGemmBM;
     tc += c[j];
     tm += mt;

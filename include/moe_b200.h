@@ -94,9 +94,10 @@ enum moe_option {
   MOE_OPT_SWAP_ROWS = 8,       /* grouped GEMM row tiles holding at most this many rows of
                                   their expert (0, 32 or 64; default 0) are computed
                                   transposed: 128 weight rows as the MMA's M side and the
-                                  tile's tokens as N = 32 or 64, so few-token experts do
-                                  not pay for 128-row MMAs.  0 = always 128 token rows.
-                                  Single-CTA grouped GEMM only.                           */
+                                  tile's tokens as N = 32 or 64.  Fewer multiply-adds, but
+                                  twice the MMA instructions, each with a fixed cost, so
+                                  it measured slower on B200; kept as an option.
+                                  0 = always 128 token rows.  Single-CTA kernel only.     */
   MOE_OPT_PAIR_TILES = 9,      /* grouped GEMMs on CTA pairs (2-CTA clusters, one
                                   M = 256 MMA across the pair, each CTA loading half of
                                   the weight tile): 0 (default) = never, 1 = when the
