@@ -35,6 +35,15 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_binding_constants_match_the_header():
+    # every MOE_OPT_ / MOE_ERR_ value the binding defines is the header's
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    header = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(MOE_(?:OPT|ERR)_\w+)\s*=\s*(-?\d+)", text)}
+    assert len([k for k in header if k.startswith("MOE_OPT_")]) >= 12
+    for name, value in header.items():
+        assert getattr(binding, name) == value, name
+
+
 def _plan(L, *shape):
     h = ctypes.c_void_p()
     rc = L.moe_plan(*shape, ctypes.byref(h))
