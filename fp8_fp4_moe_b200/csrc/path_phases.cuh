@@ -389,33 +389,41 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
 // block, smallest 2^p with amax <= 448 * 2^p (p >= -126; p = 0 if all zero),
 // codes = E4M3 round-to-nearest-even of x * 2^-p (exact scaling), written once
 // per destination row together with the block's UE8M0 code word.
-// Called by a whole warp for one item; the slice-0 warp also records the positions.
-__device__ __forceinline__ void scatter_item(long item, const uint16_t* __restrict__ x,
-                                             const int32_t* __restrict__ topk_ids,
-                                             const int32_t* __restrict__ local_rank,
-                                             const int32_t* __restrict__ group_base,
-                                             const int32_t* __restrict__ offsets,
-                                             const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
-                                             int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E, int k,
-                                             int shared) {
+// Called by a whole warp for one item = (token, SL consecutive slices): the destination rows
+// are looked up once for the SL slices, whose x loads are all issued first; the warp of the
+// token's first slices also records the positions.  scatter_item: one slice per item.
+template <int SL>
+__device__ __forceinline__ void scatter_items(long item, const uint16_t* __restrict__ x,
+                                              const int32_t* __restrict__ topk_ids,
+                                              const int32_t* __restrict__ local_rank,
+                                              const int32_t* __restrict__ group_base,
+                                              const int32_t* __restrict__ offsets,
+                                              const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
+                                              int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E, int k,
+                                              int shared) {
   const int lane = threadIdx.x % 32;
   const int n_slices = (x == nullptr) ? 1 : (H + 255) / 256;
-  if (item >= (long)T * n_slices) return;
-  const int t = (int)(item / n_slices);
-  const int slice = (int)(item % n_slices);
+  const int n_grp = (n_slices + SL - 1) / SL;
+  if (item >= (long)T * n_grp) return;
+  const int t = (int)(item / n_grp);
+  const int grp = (int)(item % n_grp);
   const int g = t / 32;
   const long R = (long)T * k;
   const int kw = H / 128;
-  // the token's 8 channels of this lane, loaded before the position lookups it does not depend on
-  const int c0 = slice * 256 + lane * 8;
-  const bool active = x != nullptr && c0 < H;     // H % 128 == 0: whole half-warps
-  const uint4 raw = active ? *reinterpret_cast<const uint4*>(x + (long)t * H + c0) : make_uint4(0, 0, 0, 0);
+  // the token's 8 channels of this lane in each slice, loaded before the position lookups they
+  // do not depend on
+  uint4 raw[SL];
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    raw[s] = x != nullptr && c0 < H ? *reinterpret_cast<const uint4*>(x + (long)t * H + c0) : make_uint4(0, 0, 0, 0);
+  }
   int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
   int e = -1;
   if (lane < k) {
     e = topk_ids[(long)t * k + lane];
     row = offsets[e] + group_base[(long)g * E + e] + local_rank[(long)t * k + lane];
-    if (slice == 0) {
+    if (grp == 0) {
       slot_pos[(long)t * k + lane] = row;
       perm[row] = t * k + lane;
     }
@@ -432,14 +440,19 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
     sf_off = ((long)(mtile_start[e] + rank / 128) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
   }
   const int ndst = k + shared;
-  {
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    if ((grp * SL + s) * 256 >= H) break;        // warp-uniform: the slice starts past H
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    const bool active = c0 < H;                  // H % 128 == 0: whole half-warps
     // 8 channels per lane; a 128-channel block spans 16 lanes.  Every lane runs
     // the shuffles (full mask); a half-warp past H idles.
+    const uint4 rw = raw[s];
     float v[8];
-    v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-    v[4] = __uint_as_float(raw.z << 16); v[5] = __uint_as_float(raw.z & 0xFFFF0000u);
-    v[6] = __uint_as_float(raw.w << 16); v[7] = __uint_as_float(raw.w & 0xFFFF0000u);
+    v[0] = __uint_as_float(rw.x << 16); v[1] = __uint_as_float(rw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(rw.y << 16); v[3] = __uint_as_float(rw.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(rw.z << 16); v[5] = __uint_as_float(rw.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(rw.w << 16); v[7] = __uint_as_float(rw.w & 0xFFFF0000u);
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -461,6 +474,17 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
       }
     }
   }
+}
+__device__ __forceinline__ void scatter_item(long item, const uint16_t* __restrict__ x,
+                                             const int32_t* __restrict__ topk_ids,
+                                             const int32_t* __restrict__ local_rank,
+                                             const int32_t* __restrict__ group_base,
+                                             const int32_t* __restrict__ offsets,
+                                             const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
+                                             int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E, int k,
+                                             int shared) {
+  scatter_items<1>(item, x, topk_ids, local_rank, group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H,
+                   E, k, shared);
 }
 
 // --------------------------------------------------------------------------- combine
