@@ -205,6 +205,36 @@ def cpu_baseline(w: I.Workload, n_tokens: int):
                       f"{len(tokens)} sampled tokens ({len(need)} experts), float64 numpy; {dt:.1f} s"}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def token_seed(rank: int) -> int:
+    """Seed of a rank's token batch: rank 0 times the workload's own tokens, the other replicas
+    distinct batches of the same shape (weights and router are shared)."""
+    return 0 if rank == 0 else 1000 + rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of the ranks' values (every rank calls it, in the same order)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def init_ranks(world: int, local_rank: int, need_gpu: bool) -> None:
+    """One process per GPU over NCCL; without a GPU (the CPU reference arm) over gloo."""
+    if world <= 1:
+        return
+    import datetime
+    timeout = datetime.timedelta(seconds=120)
+    if need_gpu or torch.cuda.is_available():
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local_rank))
+    else:
+        torch.distributed.init_process_group("gloo", timeout=timeout)
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -261,7 +291,7 @@ def run_cuda(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     _, W_r, bias = I.make_routing_inputs(w, 0)
-    x, _, _ = I.make_routing_inputs(w, 1000 + rank) if rank > 0 else I.make_routing_inputs(w, 0)
+    x, _, _ = I.make_routing_inputs(w, token_seed(rank))
     W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device=dev)
     torch.cuda.empty_cache()        # return the quantiser's temporaries: only live tensors stay on the device
     d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
@@ -314,10 +344,7 @@ def run_cuda(args, rank, world, local_rank):
     code, detail = plan.check_status()
     if code != 0:
         raise RuntimeError(f"device status {code} {detail}")
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(total_ms, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
     # Per-kernel times for the roofline: CUDA events recorded on the forward's stream
     # between its kernels (graph replay is off while the events are on).
@@ -373,10 +400,7 @@ def run_cuda(args, rank, world, local_rank):
             out_done[b].record(s_out)
         t_end.record(s_out)
         t_end.synchronize()
-        t = torch.tensor([t_start.elapsed_time(t_end)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_total = float(t.item())
+        e2e_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
         e2e = {"value": world * w.T * args.steps / (e2e_total / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
@@ -475,11 +499,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local_rank))
+    init_ranks(world, local_rank, need_gpu=args.impl != "reference")
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world)
