@@ -347,10 +347,8 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
     const int grid = (int)(blocks < 148 * 16 ? blocks : 148 * 16);
     if (ec == 8) router_logits_warp_kernel<8><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
     else router_logits_warp_kernel<2><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
-  } else if (E <= 16) {
-    dim3 grid((T + 63) / 64, (E + 15) / 16);
-    router_logits_kernel<16><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
   } else {
+    // more than 32 experts and T * E > 16384 (E <= 32 took the warp kernel above)
     dim3 grid((T + 63) / 64, (E + 63) / 64);
     router_logits_kernel<64><<<grid, 256, 0, s>>>(x, W_r, logits, T, H, E);
   }

@@ -34,6 +34,10 @@ SMALL = {
     "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
     # T >= 256 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
     "tc_router": W("tc_router", T=300, H=1024, I_=256, E=48, k=4, shared=1, router_std=0.02, bias="uniform"),
+    # E > 32 with T * E > 16384 and E % 16 != 0: the tiled CUDA-core router
+    "wide_router": W("wide_router", T=500, H=512, I_=256, E=40, k=6, shared=1, router_std=0.02, bias="uniform"),
+    # k > 8: the combine keeps up to 16 rows a lane in registers
+    "k10": W("k10", T=40, H=256, I_=256, E=24, k=10, shared=1, router_std=0.05, bias="uniform"),
     # H % 224 == 0: linear2 runs 224-row weight tiles with a double-buffered accumulator
     "h896": W("h896", T=200, H=896, I_=256, E=8, k=2, shared=1, bias="uniform"),
     "h1792_t8": W("h1792_t8", T=8, H=1792, I_=256, E=16, k=4, shared=1, router_std=0.01, bias="uniform"),
@@ -76,7 +80,8 @@ def test_quant_x_bit_exact(cuda_lib, name):
 
 # --------------------------------------------------------------------------- routing
 
-@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "t1_k1", "k_eq_E", "dsv3_like", "tc_router"])
+@pytest.mark.parametrize("name", ["tiny", "ragged_shared", "t1_k1", "k_eq_E", "dsv3_like", "tc_router", "wide_router",
+                                  "k10"])
 def test_routing_bit_exact(cuda_lib, name):
     w = SMALL[name]
     case = make_case(w, seed=5)
