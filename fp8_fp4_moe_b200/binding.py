@@ -35,6 +35,7 @@ MOE_OPT_PAIR_TILES = 9
 MOE_OPT_FUSED = 10
 MOE_OPT_DEPENDENT_LAUNCH = 11
 MOE_OPT_L2_TILE_ROWS = 12
+MOE_OPT_CHAIN = 13
 
 PHASES = ["router", "topk_rank", "scan", "scatter_quant", "prepare", "linear1", "linear2", "combine"]
 

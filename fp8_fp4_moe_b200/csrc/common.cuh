@@ -18,7 +18,7 @@ enum : int { kStatusTimeout = -4, kStatusBounds = -6 };
 enum : uint32_t {
   kWhereGemmProducer = 0x100, kWhereGemmSfLoader = 0x200, kWhereGemmMma = 0x300,
   kWhereGemmEpilogue = 0x400, kWhereGemmDrain = 0x500, kWhereRouterProducer = 0x600, kWhereRouterMma = 0x700,
-  kWhereRouterEpilogue = 0x800, kWhereGridBarrier = 0x900
+  kWhereRouterEpilogue = 0x800, kWhereGridBarrier = 0x900, kWhereGemmDependency = 0xA00
 };
 
 __device__ __forceinline__ void report_status(uint32_t* status, int code, uint32_t where, uint32_t detail) {
@@ -58,6 +58,11 @@ __device__ __forceinline__ int4 ld_cg_v4(const int4* p) {
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Orders this thread's generic-proxy global accesses with later async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // gpu-scope acquire / release accesses for grid-wide synchronisation

@@ -497,8 +497,27 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
         const int a_sel = a_box_of(c);
         const uint32_t a_box = 16u << a_sel;
+        // chained kernel: this tile's A rows exist once every linear1 tile of its expert is
+        // stored (bounded wait; on expiry the stages already requested are still completed, so
+        // that the drain below finds every copy accounted for, and nothing further is loaded)
+        bool dep_ok = true;
+        if (p.dep_wait != nullptr) {
+          const uint32_t need = (uint32_t)(((c.count + BM - 1) / BM) * p.dep_per_mtile);
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(p.dep_wait + c.e) < need) {
+            if (*ctl.abort_flag) { dep_ok = false; break; }
+            if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+              report_status(ctl.status, kStatusTimeout, kWhereGemmDependency, (uint32_t)c.e);
+              *ctl.abort_flag = 1;
+              dep_ok = false;
+              break;
+            }
+          }
+          fence_proxy_async_global();      // the acquired rows before this thread's TMA reads
+        }
         for (int kt = 0; kt < KT; ++kt) {
           const bool pre = tile == cta && kt < npre;   // weight tile already requested
+          if (!dep_ok && !pre) { ok = false; break; }
           if (!pre && !mbar_wait(&empty[stage], phase ^ 1, ctl, kWhereGemmProducer)) { ok = false; break; }
           if (withhold) {
             withhold = false;            // test hook: this stage never fills
@@ -608,6 +627,16 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
         epilogue_tile<MODE, NB>(p, c, acc, q, half, lane, TM::kDouble ? &acce[sp.lo] : acce, 0u, amax_s, buf,
                                 obuf);
       }
+      if (p.dep_signal != nullptr) {
+        // chained kernel: publish this tile's h rows and scale words to the linear2 producers
+        // (generic stores -> other CTAs' TMA reads: proxy fence, CTA barrier, gpu-scope release)
+        fence_proxy_async_global();
+        epi_bar();
+        if (threadIdx.x == 2 * 32) {
+          __threadfence();
+          atomicAdd(p.dep_signal + c.e, 1u);
+        }
+      }
       uses0 += sp.lo == 0;
       uses1 += sp.hi == 1;
       buf ^= 1;
@@ -639,6 +668,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   gemm_body<MODE, L, NB>(tmA, tmB, p, smem, tmem_base, blockIdx.x, gridDim.x);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// linear1 then linear2 in one cooperative launch for few tokens (the few-row layout): each CTA
+// runs its linear1 tiles, then its linear2 tiles, in one TMEM allocation.  linear2's producer
+// requests its first weight stages as soon as the CTA's linear1 work is done and waits, per
+// tile, only for the linear1 tiles of that tile's expert (g1.dep_signal == g2.dep_wait, zeroed
+// before the launch) -- no grid-wide barrier and no second launch.  Co-residency of all CTAs
+// (cooperative launch) guarantees that every awaited linear1 tile is being worked on.
+template <int NB2>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    chained_gemm_kernel(const __grid_constant__ AMaps tmA1, const __grid_constant__ AMaps tmA2,
+                        const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                        const GemmArgs g1, const GemmArgs g2) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmallSmem::misc);
+  const int warp = threadIdx.x / 32;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  gemm_body<1, SmallSmem>(tmA1, tmB1, g1, smem, tmem_base, blockIdx.x, gridDim.x);
+  gemm_body<2, SmallSmem, NB2>(tmA2, tmB2, g2, smem, tmem_base, blockIdx.x, gridDim.x);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
@@ -1111,9 +1171,6 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32
 }
 
 // Generic-proxy stores made visible to later TMA (async-proxy) reads of the same data.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 template <int KMAX, int U>
 __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, long first, long stride) {
@@ -1272,6 +1329,12 @@ cudaError_t gemm_prepare_device() {
   e = cudaFuncSetAttribute(grouped_gemm_kernel<2, SmemLayout, kGemmBN2Double>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes());
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(chained_gemm_kernel<kGemmBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_small_smem_bytes());
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(chained_gemm_kernel<kGemmBN2Double>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_small_smem_bytes());
+  if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tile_weight_scales_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1371,6 +1434,33 @@ cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const Gemm
                                       s, a, b, args)
                       : launch_kernel(grouped_gemm_kernel<2, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s,
                                       a, b, args);
+}
+
+cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
+                              const GemmArgs& g1, const GemmArgs& g2, int grid, cudaStream_t s) {
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const void* k = g2.bn == kGemmBN2Double ? reinterpret_cast<const void*>(chained_gemm_kernel<kGemmBN2Double>)
+                                          : reinterpret_cast<const void*>(chained_gemm_kernel<kGemmBN>);
+  if (g2.bn != kGemmBN && g2.bn != kGemmBN2Double) return cudaErrorInvalidValue;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemmThreads, gemm_small_smem_bytes())) !=
+      cudaSuccess)
+    return e;
+  if (grid < 1 || grid > per_sm * sms) return cudaErrorInvalidValue;   // every CTA co-resident
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_small_smem_bytes();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;      // co-resident CTAs (also when recorded in a graph)
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (g2.bn == kGemmBN2Double) return cudaLaunchKernelEx(&cfg, chained_gemm_kernel<kGemmBN2Double>, a1, a2, b1, b2, g1, g2);
+  return cudaLaunchKernelEx(&cfg, chained_gemm_kernel<kGemmBN>, a1, a2, b1, b2, g1, g2);
 }
 
 cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_experts, int rows_b, int K,

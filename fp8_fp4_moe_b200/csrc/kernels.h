@@ -71,6 +71,12 @@ struct GemmArgs {
   // in .y.  Tile t of the n-major order belongs to the expert of entry t / n_tiles_n.
   const int4* tile_info;
   const int4* ptile_info;
+  // Chained linear1 -> linear2 in one kernel: linear1's epilogue adds 1 to dep_signal[e] when a
+  // tile of expert e is stored; linear2's producer loads a tile's A rows only once
+  // dep_wait[e] >= ceil(count_e / 128) * dep_per_mtile.  Null outside the chained kernel.
+  uint32_t* dep_signal;
+  const uint32_t* dep_wait;
+  int dep_per_mtile;
   const uint8_t* sfa;          // activation scale atoms
   const uint8_t* sfb;          // weight scale units
   uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
@@ -99,6 +105,11 @@ cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const Gemm
                                 cudaStream_t s, bool few_rows = false);
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s, bool few_rows = false);
+// linear1 + linear2 in one cooperative launch (few-row layout, at most 16 rows per expert):
+// g1.dep_signal == g2.dep_wait (n_experts counters, zero before the launch), g2.dep_per_mtile =
+// g1.n_tiles_n; b2's box height = g2.bn.  grid <= the co-resident CTAs of the device.
+cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
+                              const GemmArgs& g1, const GemmArgs& g2, int grid, cudaStream_t s);
 // CTA-pair variants: b with 128-row boxes (each CTA loads half of the 256 B rows), scale atoms
 // and weight scale units as 2-D uint8 maps of 256-byte rows (boxes of 2 and 4 rows); grid =
 // 2 x pairs.

@@ -33,12 +33,14 @@ struct moe_plan_s {
   int fused = 0;                    // MOE_OPT_FUSED
   int dep_launch = 1;               // MOE_OPT_DEPENDENT_LAUNCH
   int l2_tile_rows = 0;             // MOE_OPT_L2_TILE_ROWS
+  int chain = 0;                    // MOE_OPT_CHAIN
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
   size_t region_len[MOE_REGION_COUNT_];
   size_t off_logits, off_rank, off_gcounts, off_gbase, off_mtile, off_ptile, off_w1sf, off_w2sf, off_whi, off_wlo;
   size_t off_tinfo, off_ptinfo;     // row-tile tables of the grouped GEMMs (mt_cap int4 each)
+  size_t off_dep;                   // per-expert linear1 tile counters of the chained GEMM kernel
   size_t off_gridbar;               // grid barrier words of the fused forward
   long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
   size_t total;
@@ -394,13 +396,27 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
   } else {
     // an expert never gets more rows than there are tokens
     const bool few_rows = p->T <= 16;
-    if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, few_rows) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    mark(p, 1 + MOE_PHASE_LINEAR1, s);
     const CUtensorMap& b2 = a2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
-    if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    mark(p, 1 + MOE_PHASE_LINEAR2, s);
+    if (few_rows && p->chain) {
+      // one cooperative launch: linear2 tiles start as soon as their expert's linear1 tiles are
+      // stored (per-expert counters, zeroed here); reported under linear1
+      uint32_t* dep = at<uint32_t>(p, p->off_dep);
+      if (cudaMemsetAsync(dep, 0, (size_t)p->n * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+      a1.dep_signal = dep;
+      a2.dep_wait = dep;
+      a2.dep_per_mtile = a1.n_tiles_n;
+      if (launch_gemm_chain(p->amA1, p->amA2, p->tmB1, b2, a1, a2, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      mark(p, 1 + MOE_PHASE_LINEAR1, s);
+      mark(p, 1 + MOE_PHASE_LINEAR2, s);
+    } else {
+      if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, few_rows) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      mark(p, 1 + MOE_PHASE_LINEAR1, s);
+      if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      mark(p, 1 + MOE_PHASE_LINEAR2, s);
+    }
   }
   cudaError_t e = launch_combine(region<uint16_t>(p, MOE_REGION_Y), region<int32_t>(p, MOE_REGION_SLOT_POS),
                                  region<float>(p, MOE_REGION_GATES), static_cast<uint16_t*>(out), p->T, p->H, p->k,
@@ -510,6 +526,7 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_ptile = add((size_t)(p->n + 1) * 4);
   p->off_tinfo = add((size_t)p->mt_cap * 16);
   p->off_ptinfo = add((size_t)p->mt_cap * 16);
+  p->off_dep = add((size_t)p->n * 4);
   p->off_gridbar = add(8);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   // linear2 weight scale units for the narrower of the two tile heights (more tiles)
@@ -557,6 +574,10 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
       if (value == 1 && p->ws && fused_max_ctas() < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
       p->fused = (int)value;
+      return MOE_OK;
+    case MOE_OPT_CHAIN:
+      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      p->chain = (int)value;
       return MOE_OK;
     case MOE_OPT_L2_TILE_ROWS:
       if (value != 0 && value != kGemmBN && value != kGemmBN2Double) return MOE_ERR_INVALID_ARG;

@@ -118,12 +118,20 @@ enum moe_option {
                                   grouped GEMMs request their first weight tiles before
                                   that wait).  0 = plain stream order.  Off while
                                   MOE_OPT_PHASE_EVENTS is 1.                              */
-  MOE_OPT_L2_TILE_ROWS = 12    /* linear2 weight rows per tile: 0 (default) = 224 when
+  MOE_OPT_L2_TILE_ROWS = 12,   /* linear2 weight rows per tile: 0 (default) = 224 when
                                   T <= 16 and H % 224 == 0, else 256; 224 = always when
                                   H % 224 == 0 (else MOE_ERR_UNSUPPORTED_SHAPE): the
                                   narrower tile leaves TMEM room for two accumulators, so
                                   one tile's epilogue overlaps the next tile's MMAs;
                                   256 = always.  CTA-pair GEMMs always use 256.            */
+  MOE_OPT_CHAIN = 13           /* 1 = with at most 16 tokens, linear1 and linear2 run as
+                                  one cooperative launch: each linear2 tile's producer
+                                  streams its weights at once and waits (bounded) only
+                                  for the linear1 tiles of its own expert.  moe_phase_times
+                                  reports both under linear1.  Measured slower inside a
+                                  CUDA graph (the cooperative launch cannot start early
+                                  as the dependent launches do).  0 (default) = two
+                                  launches.                                                */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */

@@ -109,6 +109,9 @@ def test_options_and_unbound_plan(L):
     for v in (0, 1):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, 2) == binding.MOE_ERR_INVALID_ARG
+    for v in (0, 1):
+        assert L.moe_plan_set_option(h, binding.MOE_OPT_CHAIN, v) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_CHAIN, 2) == binding.MOE_ERR_INVALID_ARG
     for v in (0, 256):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, 128) == binding.MOE_ERR_INVALID_ARG

@@ -17,17 +17,20 @@ from parity import GATE_ATOL, GATE_RTOL, assert_output_close, bits, make_case, o
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 SAMPLES = {"mixtral": 24, "dsv3_t1": 1, "dsv3_t512": 8, "dsv3_t8192_zipf": 8, "dsv3_t32768": 6}
-# separate launches for every workload; the single persistent kernel for three of them
-CASES = [(n, 0) for n in SAMPLES] + [("dsv3_t1", 1), ("dsv3_t512", 1), ("mixtral", 1)]
+# separate launches for every workload; the single persistent kernel for three of them; the
+# chained linear1 -> linear2 launch for single-token decode
+CASES = [(n, 0, 0) for n in SAMPLES] + [("dsv3_t1", 1, 0), ("dsv3_t512", 1, 0), ("mixtral", 1, 0),
+                                        ("dsv3_t1", 0, 1)]
 
 
-@pytest.mark.parametrize("name,fused", CASES)
-def test_full_size_sampled_parity(cuda_lib, name, fused):
+@pytest.mark.parametrize("name,fused,chain", CASES)
+def test_full_size_sampled_parity(cuda_lib, name, fused, chain):
     w = I.WORKLOADS[name]
     case = make_case(w, seed=0, screened=True, weight_device="cuda")
     d = {k: v.cuda().contiguous() for k, v in case.items()}
     p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
     p.set_option(binding.MOE_OPT_FUSED, fused)
+    p.set_option(binding.MOE_OPT_CHAIN, chain)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
     rng = np.random.default_rng(1)

@@ -493,6 +493,49 @@ def test_dependent_launch_matches_plain_stream_order(cuda_lib, name):
     assert p.check_status()[0] == 0
 
 
+@pytest.mark.parametrize("name", ["t1_k1", "t16_shared", "h1792_t8"])
+def test_chained_gemms_match_two_launches_bitwise(cuda_lib, name):
+    # linear1 and linear2 in one cooperative launch with per-expert counters compute the same
+    # products in the same order as two launches: the same bits, graph or not (h1792_t8 runs
+    # linear2 on 224-row tiles, the others on 256-row tiles)
+    w = SMALL[name]
+    case = make_case(w, seed=23, screened=False)
+    d = to_device(case)
+    p = plan_for(w)
+    ref = p.forward(**d).clone()
+    p.set_option(binding.MOE_OPT_CHAIN, 1)
+    for graph in (0, 1):
+        p.set_option(binding.MOE_OPT_GRAPH, graph)
+        for _ in range(3):
+            out = p.forward(**d)
+            assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), graph
+    assert p.check_status()[0] == 0
+    ref_o, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(out), ref_o["y"], name + " chained", slack)
+
+
+def test_chained_gemms_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    # one linear1 stage never fills: that CTA's MMA wait runs out, its expert's counter never
+    # completes, and every linear2 producer waiting on it runs out too -- all bounded
+    w = SMALL["t16_shared"]
+    case = make_case(w, seed=1)
+    d = to_device(case)
+    p = plan_for(w)
+    p.set_option(binding.MOE_OPT_CHAIN, 1)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 50_000_000)
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 1)
+    p.forward(**d)
+    code, detail = p.check_status()
+    assert code == binding.MOE_ERR_DEVICE_TIMEOUT
+    assert detail[1] & 0xF00 in (0x100, 0x200, 0x300, 0x400, 0xA00)
+    p.set_option(binding.MOE_OPT_INJECT_FAULT, 0)
+    p.set_option(binding.MOE_OPT_TIMEOUT_NS, 2_000_000_000)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(out), ref["y"], "chained after timeout", slack)
+
+
 # --------------------------------------------------------------------------- failure detection
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
