@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -117,7 +118,9 @@ class ClockSampler:
     def __init__(self, gpu_ids):
         self.gpu_ids = gpu_ids
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # raw samples (the JSON line carries their summary); MOE_BENCH_CLOCKS_DIR keeps them
+        out_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"moe_bench_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
