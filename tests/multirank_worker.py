@@ -21,8 +21,10 @@ def main():
         torch.distributed.barrier()
         step_max = bench.max_over_ranks(10.0 * (rank + 1), world, torch.device("cpu"))
         e2e_max = bench.max_over_ranks(-float(rank), world, torch.device("cpu"))
-        print(json.dumps({"rank": rank, "backend": torch.distributed.get_backend(), "step_max": step_max,
-                          "e2e_max": e2e_max, "seed": bench.token_seed(rank)}), flush=True)
+        # one file per rank (the ranks' stdout streams interleave under the launcher)
+        with open(os.path.join(sys.argv[1], f"rank{rank}.json"), "w") as f:
+            json.dump({"rank": rank, "backend": torch.distributed.get_backend(), "step_max": step_max,
+                       "e2e_max": e2e_max, "seed": bench.token_seed(rank)}, f)
     finally:
         torch.distributed.destroy_process_group()
 

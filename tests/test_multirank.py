@@ -26,10 +26,13 @@ def _json_lines(text):
     return [json.loads(line) for line in text.splitlines() if line.startswith("{")]
 
 
-def test_max_over_ranks_and_token_batches_on_two_gloo_ranks():
-    r = _torchrun([os.path.join("tests", "multirank_worker.py")])
+def test_max_over_ranks_and_token_batches_on_two_gloo_ranks(tmp_path):
+    r = _torchrun([os.path.join("tests", "multirank_worker.py"), str(tmp_path)])
     assert r.returncode == 0, r.stderr[-3000:]
-    lines = sorted(_json_lines(r.stdout), key=lambda d: d["rank"])
+    lines = []
+    for rank in range(2):
+        with open(tmp_path / f"rank{rank}.json") as f:
+            lines.append(json.load(f))
     assert [d["rank"] for d in lines] == [0, 1]
     for d in lines:
         assert d["backend"] == "gloo"
