@@ -35,6 +35,22 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as pedantic C99 and C11, not only as C++
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "moe_b200.h"\nint main(void) { moe_plan_t p = 0; (void)p; return 0; }\n')
+    for std in ("c99", "c11"):
+        r = subprocess.run([gcc, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                            os.path.dirname(HEADER), "-c", str(src), "-o", str(tmp_path / f"{std}.o")],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_binding_constants_match_the_header():
     # every MOE_OPT_ / MOE_ERR_ value the binding defines is the header's
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
