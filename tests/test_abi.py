@@ -51,6 +51,35 @@ def test_header_is_plain_c(tmp_path):
         assert r.returncode == 0, r.stderr
 
 
+def test_a_c_program_links_and_plans_without_a_device(L, tmp_path):
+    # a caller in C links the library directly: planning and workspace sizing need no GPU
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.join(ROOT, "fp8_fp4_moe_b200")
+    src = tmp_path / "plan.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "moe_b200.h"\n'
+        "int main(void) {\n"
+        "  moe_plan_t p = 0;\n"
+        "  if (moe_plan(4096, 4096, 14336, 8, 2, 0, &p) != MOE_OK) return 1;\n"
+        "  size_t ws = moe_workspace_bytes(p);\n"
+        "  moe_plan_destroy(p);\n"
+        "  if (moe_plan(4096, 100, 14336, 8, 2, 0, &p) != MOE_ERR_UNSUPPORTED_SHAPE) return 2;\n"
+        '  printf("%zu\\n", ws);\n'
+        "  return ws > 0 ? 0 : 3;\n"
+        "}\n")
+    exe = tmp_path / "plan"
+    r = subprocess.run([gcc, "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-L", lib_dir, "-lmoe_b200",
+                        f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert int(r.stdout) > 0
+
+
 def test_binding_constants_match_the_header():
     # every MOE_OPT_ / MOE_ERR_ value the binding defines is the header's
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
