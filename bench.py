@@ -6,7 +6,10 @@
 A step is one whole layer forward (router, top-k + gates, dispatch + E4M3
 quantisation, grouped linear1 + SwiGLU + requant, grouped linear2, combine) over
 one batch of T synthetic tokens already resident in HBM.  The default workload
-is the Mixtral-shaped layer (T=4096, H=4096, I=14336, E=8, k=2).  With N > 1
+is the DeepSeek-V3-shaped large-batch prefill (T=32768, H=7168, I=2048, E=256
+routed + 1 shared, k=8); the same run also times the metric's other batch points
+(T=1, T=512 and the Zipf-skewed T=8192 layer) on the same expert weights and
+reports them under "per_T".  With N > 1
 (launched by torchrun) every rank runs an independent replica on its own GPU and
 its own token batch: the layer has no exchange step on one device, so there is
 no collective on the data path (weak scaling); ranks only meet for the timing
@@ -55,10 +58,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="dsv3_t32768", choices=sorted(I.WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-t", action="store_true",
+                    help="time only the named workload (by default the T = 32768 headline also times the "
+                         "T = 1 / 512 / 8192 points of the metric on the same weights)")
     ap.add_argument("--no-graph", action="store_true", help="launch kernels one by one (no CUDA graph replay)")
     ap.add_argument("--opt", action="append", default=[], metavar="NAME=VALUE",
                     help="plan option, e.g. SWAP_ROWS=64 or MAX_SMS=74 (MOE_OPT_<NAME>); repeatable")
@@ -288,16 +294,61 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------- CUDA arm
 
-def run_cuda(args, rank, world, local_rank):
-    from fp8_fp4_moe_b200 import binding
-    w = workload(args)
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    _, W_r, bias = I.make_routing_inputs(w, 0)
-    x, _, _ = I.make_routing_inputs(w, token_seed(rank))
+# The metric is quoted at T = 1 / 512 / 8192 / 32768 on the DeepSeek-V3-shaped layer (the "Mega
+# MoE" batch points).  The headline line times the largest of them; the other three share its
+# expert weights (same H, I, E, k, shared expert and weight seed) and are timed in the same run.
+COMPANIONS = {"dsv3_t32768": ["dsv3_t1", "dsv3_t512", "dsv3_t8192_zipf"]}
+# short points run more steps so that the timed region is long enough to read the clocks from
+MIN_TIMED_S = 0.25
+MAX_POINT_STEPS = 2000
+
+
+def make_weights(w: I.Workload, dev):
     W1, W1s, W2, W2s = I.make_expert_weights(w, 0, device=dev)
     torch.cuda.empty_cache()        # return the quantiser's temporaries: only live tensors stay on the device
-    d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
+    return dict(W1=W1, W1_scales=W1s, W2=W2, W2_scales=W2s)
+
+
+def roofline_of(w, alg, avg, fused, peaks, peak_src, bf16_key, workload_key, resized):
+    """Roofline of the dominant kernel from the per-kernel CUDA-event times `avg` (ms)."""
+    fp8 = 2.0 * peaks[bf16_key]
+    hbm = peaks["hbm_gbs"]
+    dominant = max(avg, key=avg.get)
+    dom_ms = avg[dominant]
+    if fused:
+        # one persistent kernel for the whole forward: its time is reported as the first phase
+        dominant, dom_ms = "fused_forward", sum(avg.values())
+    if dominant in ("linear1", "linear2", "fused_forward"):
+        flops = alg[f"{dominant}_flops"] if not fused else w.flops()
+        byts = alg[f"{dominant}_bytes"] if not fused else alg["layer_bytes"]
+        if flops / byts > fp8 * 1e12 / (hbm * 1e9):
+            roof = {"bound": "tensor", "achieved": flops / (dom_ms * 1e-3) / 1e12, "peak": fp8,
+                    "unit": "TFLOP/s", "algorithmic": flops}
+        else:
+            roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                    "algorithmic": byts}
+    else:
+        byts = alg["layer_bytes"]
+        roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                "algorithmic": byts}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dominant
+    roof["kernel_ms"] = dom_ms
+    roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json: 2 x {bf16_key} (FP8 = 2 x BF16 dense)"
+                           if roof["unit"] == "TFLOP/s" else f"{peak_src} MEASURED_PEAKS.json hbm_gbs")
+    roof["traffic"] = ncu_traffic(dominant, workload_key) if not resized else None
+    return roof
+
+
+def measure(w: I.Workload, weights: dict, args, rank, world, dev, steps: int, resized: bool, workload_key: str):
+    """Time `steps` forwards of workload `w` (inputs resident in HBM, L2 flushed between steps),
+    then the per-kernel event pass and the end-to-end pass.  Every rank calls it in the same order
+    (barriers and max-over-ranks reductions).  Returns rank 0's record (None elsewhere)."""
+    from fp8_fp4_moe_b200 import binding
+    _, W_r, bias = I.make_routing_inputs(w, 0)
+    x, _, _ = I.make_routing_inputs(w, token_seed(rank))
+    d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), **weights)
+    del x
     plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared, device=dev)
     # launch the forward's kernels as one recorded CUDA graph (per pointer set)
     plan.set_option(binding.MOE_OPT_GRAPH, 0 if args.no_graph else 1)
@@ -324,23 +375,21 @@ def run_cuda(args, rank, world, local_rank):
         raise RuntimeError(f"device status {code} {detail}")
     counts = plan.region("counts").cpu().numpy()
 
-    sampler = ClockSampler(list(range(world)) if rank == 0 else [local_rank])
+    sampler = ClockSampler(list(range(world)) if rank == 0 else [local_index(dev)])
     if rank == 0:
         sampler.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     step_ms = []
-    for _ in range(args.steps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
         flush.fill_(1)                                   # L2 scrub between timed steps (not timed)
-        ev0 = torch.cuda.Event(enable_timing=True)
-        ev1 = torch.cuda.Event(enable_timing=True)
-        ev0.record(stream)
+        ev[i][0].record(stream)
         plan.forward(**d, out=out)
-        ev1.record(stream)
-        ev1.synchronize()
-        step_ms.append(ev0.elapsed_time(ev1))
+        ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if rank == 0 else None
@@ -353,12 +402,15 @@ def run_cuda(args, rank, world, local_rank):
     # between its kernels (graph replay is off while the events are on).
     plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 1)
     phases = []
-    for _ in range(min(args.steps, 20)):
+    for _ in range(min(steps, 20)):
         flush.fill_(1)
         plan.forward(**d, out=out)
         phases.append(plan.phase_times())
     plan.set_option(binding.MOE_OPT_PHASE_EVENTS, 0)
     plan.set_option(binding.MOE_OPT_GRAPH, 0 if args.no_graph else 1)
+    for kv in args.opt:
+        name, value = kv.split("=", 1)
+        plan.set_option(getattr(binding, "MOE_OPT_" + name.upper()), int(value))
 
     # end to end through the public API: pinned host x -> device, forward, out -> pinned host
     # Every step copies its tokens host -> device, runs the layer and copies the
@@ -366,55 +418,17 @@ def run_cuda(args, rank, world, local_rank):
     # copy out) with double-buffered device tensors, as a serving loop would.
     e2e = None
     if not args.no_e2e:
-        nbuf = 2
-        x_host = d["x"].cpu().pin_memory()
-        out_host = [torch.empty(w.T, w.H, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
-        x_dev = [torch.empty_like(d["x"]) for _ in range(nbuf)]
-        out_dev = [torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        in_done = [torch.cuda.Event() for _ in range(nbuf)]
-        fwd_done = [torch.cuda.Event() for _ in range(nbuf)]
-        out_done = [torch.cuda.Event() for _ in range(nbuf)]
-        d_e2e = dict(d)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(s_in)
-        stream.wait_event(t_start)
-        s_out.wait_event(t_start)
-        for i in range(args.steps):
-            b = i % nbuf
-            if i >= nbuf:
-                s_in.wait_event(fwd_done[b])           # x_dev[b] no longer read
-            with torch.cuda.stream(s_in):
-                x_dev[b].copy_(x_host, non_blocking=True)
-            in_done[b].record(s_in)
-            stream.wait_event(in_done[b])
-            if i >= nbuf:
-                stream.wait_event(out_done[b])         # out_dev[b] already copied out
-            d_e2e["x"] = x_dev[b]
-            plan.forward(**d_e2e, out=out_dev[b], stream=stream)
-            fwd_done[b].record(stream)
-            s_out.wait_event(fwd_done[b])
-            with torch.cuda.stream(s_out):
-                out_host[b].copy_(out_dev[b], non_blocking=True)
-            out_done[b].record(s_out)
-        t_end.record(s_out)
-        t_end.synchronize()
-        e2e_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-        e2e = {"value": world * w.T * args.steps / (e2e_total / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-               "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
-               "ms_per_step": e2e_total / args.steps,
-               "pipelining": "copy-in / compute / copy-out on 3 streams, double-buffered"}
-        code, detail = plan.check_status()
-        if code != 0:
-            raise RuntimeError(f"device status {code} {detail}")
+        e2e = measure_e2e(w, plan, d, args, world, dev, stream, steps)
+    del flush
     if rank != 0:
+        del plan, d, out
+        torch.cuda.empty_cache()
         return None
 
+    alg = algorithmic_counts(w, counts)
+    avg = {k: statistics.mean(p[k] for p in phases) for k in phases[0]}
+    ms = total_ms / steps
+    fused = any(o.replace(" ", "").upper() == "FUSED=1" for o in args.opt)
     peaks, peak_src = load_peaks()
     # Tensor peak: measured bf16 x the nominal FP8:BF16 dense ratio of 2.  The burst
     # figure when the SM clock stayed at its maximum during the timed steps, the
@@ -422,40 +436,130 @@ def run_cuda(args, rank, world, local_rank):
     at_max = bool(clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz")
                   and clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"])
     bf16_key = "bf16_tflops" if at_max else "bf16_tflops_sustained"
-    fp8_sustained = 2.0 * peaks[bf16_key]
+    fp8 = 2.0 * peaks[bf16_key]
     hbm = peaks["hbm_gbs"]
-    alg = algorithmic_counts(w, counts)
-    avg = {k: statistics.mean(p[k] for p in phases) for k in phases[0]}
-    ms = total_ms / args.steps
-    dominant = max(avg, key=avg.get)
-    dom_ms = avg[dominant]
-    fused = any(o.replace(" ", "").upper() == "FUSED=1" for o in args.opt)
-    if fused:
-        # one persistent kernel for the whole forward: its time is reported as the first phase
-        dominant, dom_ms = "fused_forward", sum(avg.values())
-    if dominant in ("linear1", "linear2", "fused_forward"):
-        flops = alg[f"{dominant}_flops"] if not fused else w.flops()
-        byts = alg[f"{dominant}_bytes"] if not fused else alg["layer_bytes"]
-        if flops / byts > fp8_sustained * 1e12 / (hbm * 1e9):
-            roof = {"bound": "tensor", "achieved": flops / (dom_ms * 1e-3) / 1e12, "peak": fp8_sustained,
-                    "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
-    else:
-        byts = alg["layer_bytes"]
-        roof = {"bound": "hbm", "achieved": byts / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = dominant
-    roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json: 2 x {bf16_key} (FP8 = 2 x BF16 dense)"
-                           if roof["unit"] == "TFLOP/s" else f"{peak_src} MEASURED_PEAKS.json hbm_gbs")
+    roof = roofline_of(w, alg, avg, fused, peaks, peak_src, bf16_key, workload_key, resized)
+    rec = {
+        "workload": w.description + ("" if not resized else f" (resized to T={w.T}, E={w.E})"),
+        "T": w.T,
+        "steps": steps,
+        "ms_per_step": ms,
+        "tokens_per_s": world * w.T / (ms * 1e-3),
+        "tflops": w.flops() / (ms * 1e-3) / 1e12,
+        "tflops_frac_fp8": w.flops() / (ms * 1e-3) / 1e12 / fp8,
+        "fp8_peak_tflops": fp8,
+        "hbm_gbs": alg["layer_bytes"] / (ms * 1e-3) / 1e9,
+        "hbm_frac": alg["layer_bytes"] / (ms * 1e-3) / 1e9 / hbm,
+        "layer_flops": alg["layer_flops"],
+        "layer_bytes": alg["layer_bytes"],
+        "phases_ms": avg,
+        "roofline": roof,
+        "e2e": e2e,
+        # the fused option is one kernel per forward
+        "gpu_launches": (1 if fused else kernels_per_forward(w)) * steps,
+        "clocks": clocks,
+        "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
+        "touched_experts": alg["touched_experts"],
+        "weight_scales_prepare_ms": prepare_ms,
+    }
+    del plan, d, out
+    torch.cuda.empty_cache()
+    return rec
+
+
+def local_index(dev) -> int:
+    return dev.index if dev.index is not None else 0
+
+
+def measure_e2e(w, plan, d, args, world, dev, stream, steps):
+    nbuf = 2
+    x_host = d["x"].cpu().pin_memory()
+    out_host = [torch.empty(w.T, w.H, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    x_dev = [torch.empty_like(d["x"]) for _ in range(nbuf)]
+    out_dev = [torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_done = [torch.cuda.Event() for _ in range(nbuf)]
+    fwd_done = [torch.cuda.Event() for _ in range(nbuf)]
+    out_done = [torch.cuda.Event() for _ in range(nbuf)]
+    d_e2e = dict(d)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(s_in)
+    stream.wait_event(t_start)
+    s_out.wait_event(t_start)
+    for i in range(steps):
+        b = i % nbuf
+        if i >= nbuf:
+            s_in.wait_event(fwd_done[b])           # x_dev[b] no longer read
+        with torch.cuda.stream(s_in):
+            x_dev[b].copy_(x_host, non_blocking=True)
+        in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if i >= nbuf:
+            stream.wait_event(out_done[b])         # out_dev[b] already copied out
+        d_e2e["x"] = x_dev[b]
+        plan.forward(**d_e2e, out=out_dev[b], stream=stream)
+        fwd_done[b].record(stream)
+        s_out.wait_event(fwd_done[b])
+        with torch.cuda.stream(s_out):
+            out_host[b].copy_(out_dev[b], non_blocking=True)
+        out_done[b].record(s_out)
+    t_end.record(s_out)
+    t_end.synchronize()
+    e2e_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    code, detail = plan.check_status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} {detail}")
+    return {"value": world * w.T * steps / (e2e_total / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+            "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size()),
+            "ms_per_step": e2e_total / steps, "steps": steps,
+            "pipelining": "copy-in / compute / copy-out on 3 streams, double-buffered"}
+
+
+def point_steps(ms_estimate: float, steps: int) -> int:
+    """Steps of a companion point: at least `steps`, enough for MIN_TIMED_S of timed forwards."""
+    want = int(MIN_TIMED_S * 1e3 / max(ms_estimate, 1e-3)) + 1
+    return max(steps, min(want, MAX_POINT_STEPS))
+
+
+def run_cuda(args, rank, world, local_rank):
+    w = workload(args)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
     resized = args.tokens is not None or args.experts is not None
-    roof["traffic"] = ncu_traffic(dominant, args.workload) if not resized else None
+    weights = make_weights(w, dev)
+    head = measure(w, weights, args, rank, world, dev, args.steps, resized, args.workload)
+    per_t = None
+    companions = [] if (resized or args.no_per_t) else COMPANIONS.get(args.workload, [])
+    if companions:
+        per_t = {}
+        for name in companions:
+            wc = I.WORKLOADS[name]
+            assert (wc.H, wc.I, wc.E, wc.k, wc.shared, wc.weight_std) == (w.H, w.I, w.E, w.k, w.shared, w.weight_std)
+            # a short untimed run sizes the step count so every point's timed region is long enough
+            est = measure_estimate(wc, weights, dev)
+            est = max_over_ranks(est, world, dev)
+            rec = measure(wc, weights, args, rank, world, dev, point_steps(est, args.steps), False, name)
+            if rank == 0:
+                per_t[f"T={wc.T}"] = rec
+        head_key = f"T={w.T}"
+        if rank == 0:
+            per_t = {head_key: {k: v for k, v in head.items()}, **per_t}
+            per_t = dict(sorted(per_t.items(), key=lambda kv: kv[1]["T"]))
+    if rank != 0:
+        return None
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, CPU_SAMPLE_TOKENS[args.workload])
 
-    value = world * w.T * args.steps / (total_ms / 1e3)
+    ms = head["ms_per_step"]
+    value = world * w.T * args.steps / (ms * args.steps / 1e3)
+    fused = any(o.replace(" ", "").upper() == "FUSED=1" for o in args.opt)
     line = {
         "metric": METRIC,
         "value": value,
@@ -469,32 +573,57 @@ def run_cuda(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8e4m3 x fp4e2m1 (fp32 accumulate)",
         "data": "synthetic",
-        "config": {"workload": w.description + ("" if not resized else f" (resized to T={w.T}, E={w.E})"),
+        "config": {"workload": head["workload"],
                    "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
                    "shared": w.shared, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
                    "launch": ("one persistent cooperative kernel (MOE_OPT_FUSED)" if fused else
                               "kernels launched one by one" if args.no_graph else
                               f"CUDA graph replay of the {kernels_per_forward(w)} kernels (MOE_OPT_GRAPH)"),
                    "phase_times": "separate pass, CUDA events between kernels, 20 steps",
-                   "weight_scales": f"re-laid out once before timing ({prepare_ms:.3f} ms), reused "
-                                    "(MOE_OPT_STATIC_WEIGHTS)",
+                   "weight_scales": f"re-laid out once before timing ({head['weight_scales_prepare_ms']:.3f} ms), "
+                                    "reused (MOE_OPT_STATIC_WEIGHTS)",
                    "parallelism": f"replicas x{world} (token-sharded, no collective)",
-                   "options": args.opt},
-        "tflops": w.flops() / (ms * 1e-3) / 1e12,
-        "tflops_frac_fp8": w.flops() / (ms * 1e-3) / 1e12 / fp8_sustained,
-        "fp8_peak_tflops": fp8_sustained,
-        "hbm_gbs": alg["layer_bytes"] / (ms * 1e-3) / 1e9,
-        "hbm_frac": alg["layer_bytes"] / (ms * 1e-3) / 1e9 / hbm,
-        "phases_ms": avg,
-        "roofline": roof,
+                   "options": args.opt,
+                   "per_T": ("the T = 1 / 512 / 8192 (Zipf-skewed) DeepSeek-V3-shaped layers on the same "
+                             "expert weights, each timed in this run with its own steps, clocks, roofline "
+                             "and end-to-end pass" if per_t else None)},
+        "tflops": head["tflops"],
+        "tflops_frac_fp8": head["tflops_frac_fp8"],
+        "fp8_peak_tflops": head["fp8_peak_tflops"],
+        "hbm_gbs": head["hbm_gbs"],
+        "hbm_frac": head["hbm_frac"],
+        "phases_ms": head["phases_ms"],
+        "roofline": head["roofline"],
         "cpu_baseline": cpu,
-        "e2e": e2e,
-        # the fused option is one kernel per forward
-        "gpu_launches": (1 if fused else kernels_per_forward(w)) * args.steps,
-        "clocks": clocks,
-        "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "max_expert_load_ratio": head["max_expert_load_ratio"],
+        "per_T": per_t,
     }
     return line
+
+
+def measure_estimate(w, weights, dev) -> float:
+    """Milliseconds of one forward of `w` (untimed sizing run: 3 forwards, the last one timed)."""
+    from fp8_fp4_moe_b200 import binding
+    x, W_r, bias = I.make_routing_inputs(w, 0)
+    d = dict(x=x.to(dev), W_router=W_r.to(dev), bias=bias.to(dev), **weights)
+    plan = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared, device=dev)
+    plan.set_option(binding.MOE_OPT_STATIC_WEIGHTS, 1)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(2):
+        plan.forward(**d, out=out)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    plan.forward(**d, out=out)
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b)
+    del plan, d, out
+    torch.cuda.empty_cache()
+    return ms
 
 
 def main():

@@ -166,17 +166,34 @@ def gemm_fp8_fp4(A, A_scales, B, B_scales, out=None, workspace=None, stream=None
 def route_noalloc(x, W_router, bias, k: int, topk_ids=None, gates=None, stream=None):
     """Routing through moe_route_noalloc: no plan, no workspace, no device allocation
     inside the library (the outputs are the caller's; pass them to avoid any
-    allocation here too).  Returns (topk_ids int32 [T,k], gates fp32 [T,k])."""
-    d = x.device
+    allocation here too).  Runs on x's device (made current for the call; `stream`, if
+    given, must belong to it).  Returns (topk_ids int32 [T,k], gates fp32 [T,k])."""
+    if x.dim() != 2:
+        raise ValueError(f"x must be [T, H], got shape {tuple(x.shape)}")
     T, H = x.shape
+    if W_router.dim() != 2 or W_router.shape[1] != H:
+        raise ValueError(f"W_router must be [E, {H}], got shape {tuple(W_router.shape)}")
     E = W_router.shape[0]
-    if topk_ids is None:
-        topk_ids = torch.empty(T, k, dtype=torch.int32, device=d)
-    if gates is None:
-        gates = torch.empty(T, k, dtype=torch.float32, device=d)
-    rc = lib().moe_route_noalloc(T, H, E, k, _ptr(x, torch.bfloat16, d), _ptr(W_router, torch.float32, d),
-                                 _ptr(bias, torch.float32, d), _ptr(topk_ids, torch.int32, d),
-                                 _ptr(gates, torch.float32, d), _stream_ptr(stream))
+    if bias.dim() != 1 or bias.numel() != E:
+        raise ValueError(f"bias must be [{E}], got shape {tuple(bias.shape)}")
+    d = x.device
+    if d.type != "cuda":
+        raise ValueError(f"x must be on a CUDA device, got {d}")
+    with torch.cuda.device(d):
+        if topk_ids is None:
+            topk_ids = torch.empty(T, k, dtype=torch.int32, device=d)
+        if gates is None:
+            gates = torch.empty(T, k, dtype=torch.float32, device=d)
+        for name, t in (("topk_ids", topk_ids), ("gates", gates)):
+            if tuple(t.shape) != (T, k):
+                raise ValueError(f"{name} must be [{T}, {k}], got shape {tuple(t.shape)}")
+        if stream is None:
+            stream = torch.cuda.current_stream(d)
+        elif stream.device != d:
+            raise ValueError(f"stream on {stream.device}, x on {d}")
+        rc = lib().moe_route_noalloc(T, H, E, k, _ptr(x, torch.bfloat16, d), _ptr(W_router, torch.float32, d),
+                                     _ptr(bias, torch.float32, d), _ptr(topk_ids, torch.int32, d),
+                                     _ptr(gates, torch.float32, d), stream.cuda_stream)
     _check(rc, "moe_route_noalloc")
     return topk_ids, gates
 
@@ -239,6 +256,10 @@ class Plan:
 
     def debug_routing(self, x, W_router, bias, stream=None):
         d = self.device
+        for name, t, shape in (("x", x, (self.T, self.H)), ("W_router", W_router, (self.E, self.H)),
+                               ("bias", bias, (self.E,))):
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be {list(shape)}, got shape {tuple(t.shape)}")
         ids = torch.empty(self.T, self.k, dtype=torch.int32, device=d)
         gates = torch.empty(self.T, self.k, dtype=torch.float32, device=d)
         _check(lib().moe_debug_routing(self._h, _ptr(x, torch.bfloat16, d), _ptr(W_router, torch.float32, d),

@@ -32,7 +32,9 @@ size_t round_up(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Device address of the scratch array on the current device.  The host-side
 // name g_route_scratch is only a stand-in for the symbol, so the address is
-// looked up once per device (with that device current) and cached.
+// looked up once per device (with that device current) and cached for the
+// life of the process; a reset of the device (cudaDeviceReset) unloads the
+// module that holds the array and leaves the cached address stale.
 int scratch_on_current_device(unsigned char** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
@@ -47,6 +49,18 @@ int scratch_on_current_device(unsigned char** out) {
 }
 
 bool aligned(const void* p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// True when p is device (or managed) memory that the device `dev` owns.  The kernels run on the
+// current device, so a buffer of another device would be read through a foreign address.
+// cudaPointerGetAttributes allocates nothing.
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();                // clear the (non-sticky) error so later calls do not see it
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
 
 }  // namespace
 
@@ -63,6 +77,11 @@ extern "C" int moe_route_noalloc(int T, int H, int E, int k, const void* x_bf16,
   const size_t status_bytes = 256;
   if (logits_bytes + rank_bytes + counts_bytes + status_bytes > kScratchBytes) return MOE_ERR_WORKSPACE;
 
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!on_device(x_bf16, dev) || !on_device(W_router, dev) || !on_device(bias, dev) || !on_device(topk_ids, dev) ||
+      !on_device(gates, dev))
+    return MOE_ERR_INVALID_ARG;
   unsigned char* scratch = nullptr;
   int rc = scratch_on_current_device(&scratch);
   if (rc != MOE_OK) return rc;

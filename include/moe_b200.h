@@ -222,9 +222,16 @@ int moe_debug_routing(moe_plan_t plan, const void* x_bf16, const float* W_router
  * -- about 15,000 tokens at E = 256, k = 8.  Shapes as for moe_plan
  * (MOE_ERR_UNSUPPORTED_SHAPE otherwise).  Calls no allocating routine.
  *
+ * Every pointer must be device memory of the CURRENT device (the kernels run
+ * there); MOE_ERR_INVALID_ARG otherwise (checked with cudaPointerGetAttributes,
+ * before anything is launched).
+ *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and leave their intermediates in it:
+ * device current) and caches it for the life of the process; make that first
+ * call before any stream capture.  The cached address is not valid after the
+ * device is reset (cudaDeviceReset): do not call this entry point again in a
+ * process that reset a device it used.  All calls share the one array and
+ * leave their intermediates in it:
  * calls whose kernels can overlap on the GPU (different streams without
  * ordering between them) race on it, so order them on one stream or by events.
  * Asynchronous on `stream`. */

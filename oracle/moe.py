@@ -170,14 +170,22 @@ def expert_ffn(xq, xexp, W1_e, W1s_e, W2_e, W2s_e, I: int):
 
 # ----------------------------------------------------------------------------- forward
 
+def _expert_job(job):
+    """expert_ffn on one expert's rows; `job` = its argument tuple (a picklable unit of work)."""
+    return expert_ffn(*job)
+
+
 def forward(x_bits, W_router, bias, W1, W1_scales, W2, W2_scales, k: int, shared: int,
-            tokens=None, keep_rows: bool = False):
+            tokens=None, keep_rows: bool = False, ffn_map=None):
     """The whole layer for all tokens, or only for `tokens` (routing is always global).
 
     [MoE] "FFN 교체": y = sum over the top-k experts of gate * Expert_e(x);
     [Play] "작동 방식" step 3 (weighted sum) and the shared expert every token
     passes.  Each output row depends only on its own token, so computing a
     subset of tokens is exact.
+
+    `ffn_map` (default: the builtin map) evaluates the experts' FFNs, which are
+    independent of one another: a process pool's map gives the same numbers.
 
     Returns a dict with ids, gates, scores, counts, offsets, perm, slot_pos,
     the token-order x quantisation (xq, xexp), out_bits [n_tok, H] (bf16 bits),
@@ -210,12 +218,11 @@ def forward(x_bits, W_router, bias, W1, W1_scales, W2, W2_scales, k: int, shared
     n = len(tok)
     row_vals = np.zeros((n, k + shared, H), dtype=np.float64)   # bf16 rows as float64
     extras = {}
-    for e in range(n_tot):
+    used = [e for e in range(n_tot) if rows_by_expert[e]]
+    sels = {e: np.array([i for i, _ in rows_by_expert[e]], dtype=np.int64) for e in used}
+    jobs = ((xq[sels[e]], xexp[sels[e]], W1[e], W1_scales[e], W2[e], W2_scales[e], I) for e in used)
+    for e, res in zip(used, (map if ffn_map is None else ffn_map)(_expert_job, jobs)):
         lst = rows_by_expert[e]
-        if not lst:
-            continue
-        sel = np.array([i for i, _ in lst], dtype=np.int64)
-        res = expert_ffn(xq[sel], xexp[sel], W1[e], W1_scales[e], W2[e], W2_scales[e], I)
         rv = F.bf16_to_f64(res["row_bits"])
         for r, (i, j) in enumerate(lst):
             row_vals[i, j if j >= 0 else k] = rv[r]

@@ -194,3 +194,21 @@ def test_error_strings(L):
     for code in range(-6, 1):
         assert L.moe_error_string(code)
     assert L.moe_error_string(-99) == b"unknown error"
+
+
+def test_route_noalloc_binding_rejects_mismatched_shapes_before_the_library():
+    """The binding validates every shape (and the device) before any pointer reaches the C ABI."""
+    import torch
+
+    from fp8_fp4_moe_b200 import binding
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    W = torch.zeros(8, 256, dtype=torch.float32)
+    b = torch.zeros(8, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        binding.route_noalloc(x[0], W, b, 2)                       # x not [T, H]
+    with pytest.raises(ValueError):
+        binding.route_noalloc(x, W[:, :128], b, 2)                 # W_router too narrow
+    with pytest.raises(ValueError):
+        binding.route_noalloc(x, W, b[:7], 2)                      # bias of the wrong length
+    with pytest.raises(ValueError):
+        binding.route_noalloc(x, W, b, 2)                          # CPU tensors
