@@ -425,6 +425,9 @@ def measure(w: I.Workload, weights: dict, args, rank, world, dev, steps: int, re
         torch.cuda.empty_cache()
         return None
 
+    tile_rows = plan.get_option(binding.MOE_OPT_TILE_ROWS)
+    zero_pad = plan.get_option(binding.MOE_OPT_ZERO_PAD)
+    l2_rows = plan.get_option(binding.MOE_OPT_L2_TILE_ROWS)
     alg = algorithmic_counts(w, counts)
     avg = {k: statistics.mean(p[k] for p in phases) for k in phases[0]}
     ms = total_ms / steps
@@ -461,6 +464,7 @@ def measure(w: I.Workload, weights: dict, args, rank, world, dev, steps: int, re
         "max_expert_load_ratio": float(counts[:w.E].max() / (w.T * w.k / w.E)),
         "touched_experts": alg["touched_experts"],
         "weight_scales_prepare_ms": prepare_ms,
+        "gemm_tiles": {"rows": tile_rows, "zero_padded": zero_pad == 1, "linear2_weight_rows": l2_rows},
     }
     del plan, d, out
     torch.cuda.empty_cache()

@@ -36,16 +36,18 @@ MOE_OPT_FUSED = 10
 MOE_OPT_DEPENDENT_LAUNCH = 11
 MOE_OPT_L2_TILE_ROWS = 12
 MOE_OPT_CHAIN = 13
+MOE_OPT_TILE_ROWS = 14
+MOE_OPT_ZERO_PAD = 15
 
 PHASES = ["router", "topk_rank", "scan", "scatter_quant", "prepare", "linear1", "linear2", "combine"]
 
 REGIONS = {
     "status": 0, "topk_ids": 1, "gates": 2, "counts": 3, "offsets": 4, "perm": 5, "slot_pos": 6,
-    "xq": 7, "xsf": 8, "hq": 9, "hsf": 10, "y": 11,
+    "xq": 7, "xsf": 8, "hq": 9, "hsf": 10, "y": 11, "stamps": 12,
 }
 
 EXPORTED = [
-    "moe_plan", "moe_plan_set_option", "moe_workspace_bytes", "moe_set_workspace", "moe_workspace_region",
+    "moe_plan", "moe_plan_set_option", "moe_plan_get_option", "moe_workspace_bytes", "moe_set_workspace", "moe_workspace_region",
     "moe_forward", "moe_debug_routing", "moe_debug_dispatch", "moe_debug_quant_x", "moe_check_status",
     "moe_plan_destroy", "moe_error_string", "moe_phase_times", "moe_prepare_weights", "moe_route_noalloc",
     "moe_update_bias", "moe_gemm_workspace_bytes", "moe_gemm_fp8_fp4",
@@ -73,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.moe_plan.restype = i32
     L.moe_plan_set_option.argtypes = [vp, i32, ctypes.c_longlong]
     L.moe_plan_set_option.restype = i32
+    L.moe_plan_get_option.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_longlong)]
+    L.moe_plan_get_option.restype = i32
     L.moe_workspace_bytes.argtypes = [vp]
     L.moe_workspace_bytes.restype = sz
     L.moe_set_workspace.argtypes = [vp, vp, sz]
@@ -224,6 +228,12 @@ class Plan:
     def set_option(self, key: int, value: int):
         _check(lib().moe_plan_set_option(self._h, key, value), "moe_plan_set_option")
 
+    def get_option(self, key: int) -> int:
+        """The option's value for this plan (row-tile heights resolved to what the GEMMs use)."""
+        v = ctypes.c_longlong()
+        _check(lib().moe_plan_get_option(self._h, key, ctypes.byref(v)), "moe_plan_get_option")
+        return v.value
+
     def region(self, name: str) -> torch.Tensor:
         """A typed view of a workspace region (for tests and debugging)."""
         off, n = ctypes.c_size_t(), ctypes.c_size_t()
@@ -231,11 +241,12 @@ class Plan:
         raw = self.workspace[off.value:off.value + n.value]
         dt = {"status": torch.int32, "topk_ids": torch.int32, "gates": torch.float32, "counts": torch.int32,
               "offsets": torch.int32, "perm": torch.int32, "slot_pos": torch.int32, "xq": torch.uint8,
-              "xsf": torch.uint8, "hq": torch.uint8, "hsf": torch.uint8, "y": torch.bfloat16}[name]
+              "xsf": torch.uint8, "hq": torch.uint8, "hsf": torch.uint8, "y": torch.bfloat16,
+              "stamps": torch.int64}[name]
         v = raw.view(dt)
         shapes = {"topk_ids": (self.T, self.k), "gates": (self.T, self.k), "slot_pos": (self.T, self.k),
                   "xq": (self.rows, self.H), "xsf": (-1, self.H // 128, 512), "hq": (self.rows, self.I),
-                  "hsf": (-1, self.I // 128, 512), "y": (self.rows, self.H)}
+                  "hsf": (-1, self.I // 128, 512), "y": (self.rows, self.H), "stamps": (-1, 1024)}
         return v.view(shapes[name]) if name in shapes else v
 
     def forward(self, x, W_router, bias, W1, W1_scales, W2, W2_scales, out=None, stream=None):

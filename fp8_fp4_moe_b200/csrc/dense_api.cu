@@ -124,6 +124,7 @@ int moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* A, const uint8_t* A_sca
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_tile_weight_scales(B_scales, ws + L.units, 1, N, K, nt, 2, N, s) != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs a{};
+  a.bm = kGemmBM;
   a.K = K;
   a.N = N;
   a.rows_b = N;

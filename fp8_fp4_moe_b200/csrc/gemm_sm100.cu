@@ -49,18 +49,21 @@ constexpr uint32_t kBTileBytes = BN * BK;            // 32 KB in shared memory (
 constexpr uint32_t kSfaBytes = 512, kSfbBytes = 1024;
 
 // Shared memory of the single-CTA grouped GEMM: STAGES pipeline stages with an A region of
-// A_BYTES each, and (STAGING) a 2 KB per-warp buffer the epilogue stores go through.
-template <int STAGES, uint32_t A_BYTES, bool STAGING>
+// A_BYTES each, and (STAGING) a 2 KB per-warp buffer the epilogue stores go through.  The
+// linear1 epilogue exchanges per-row amax values for AMAX_ROWS accumulator rows (the rows a
+// tile can hold; 128 also leaves room for the transposed-tile exchange).
+template <int STAGES, uint32_t A_BYTES, bool STAGING, int AMAX_ROWS = 128>
 struct GemmSmem {
   static constexpr int kStages = STAGES;
   static constexpr uint32_t kABytes = A_BYTES;
   static constexpr bool kStaging = STAGING;
+  static constexpr int kAmaxRows = AMAX_ROWS;
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + STAGES * A_BYTES;
   static constexpr uint32_t sfa = b + STAGES * kBTileBytes;
   static constexpr uint32_t sfb = sfa + STAGES * kSfaBytes;
-  static constexpr uint32_t amax = sfb + STAGES * kSfbBytes;      // [2 buffers][2 halves][128 rows] fp32
-  static constexpr uint32_t stage_out = amax + 2 * 2 * 128 * 4;   // [8 epilogue warps][32 rows][64 B]
+  static constexpr uint32_t amax = sfb + STAGES * kSfbBytes;      // [2 buffers][2 halves][AMAX_ROWS] fp32
+  static constexpr uint32_t stage_out = amax + 2 * 2 * AMAX_ROWS * 4;   // [8 epilogue warps][32 rows][64 B]
   static constexpr uint32_t bars = stage_out + (STAGING ? 8 * 2048 : 0);
   // full[STAGES], empty[STAGES], accf[2], acce[2], drain
   static constexpr uint32_t n_bars = 2 * STAGES + 5;
@@ -69,11 +72,11 @@ struct GemmSmem {
 };
 // Any number of rows per tile: 4 stages with 128-row A regions.
 using SmemLayout = GemmSmem<S, kATileBytes, true>;
-// At most 16 rows per expert (T <= 16): 16-row A regions leave room for 6 stages; the MMA
+// 32-row row tiles (decode-sized experts): 32-row A regions leave room for 6 stages; the MMA
 // still reads 128 A rows, the ones past the region are other stages' bytes and land in
 // accumulator rows that are never stored.  Epilogue stores go straight to global memory.
-using SmallSmem = GemmSmem<6, 16 * BK, false>;
-static_assert(SmallSmem::total + 1024 <= 232448, "few-token layout exceeds shared memory");
+using SmallSmem = GemmSmem<6, kGemmBMSmall * BK, false, kGemmBMSmall>;
+static_assert(SmallSmem::total + 1024 <= 232448, "small-tile layout exceeds shared memory");
 
 struct TileCoord {
   int e, mt, nt, count, row0, gmt;   // gmt = global row-tile index
@@ -82,22 +85,42 @@ struct TileCoord {
 
 // The tiles of expert e are [mtile_start[e], mtile_start[e + 1]) x n_tiles_n, so tile / n_tiles_n
 // is one of e's row tiles and its table entry names e: one load per tile instead of a search
-// over the experts.
-__device__ __forceinline__ TileCoord decode_tile(const GemmArgs& p, int tile) {
-  const int4 info = ld_cg_v4(p.tile_info + tile / p.n_tiles_n);   // {e, mtile_start, count, offset}
+// over the experts.  Each role loads the entry of its next tile while it works on the current
+// one (tile_entry / TileCursor), so the load's latency is off the tile boundary.
+__device__ __forceinline__ int4 tile_entry(const GemmArgs& p, int tile, int total_tiles) {
+  return tile < total_tiles ? ld_cg_v4(p.tile_info + tile / p.n_tiles_n) : make_int4(0, 0, 0, 0);
+}
+// info = the table entry {e, mtile_start, count, offset} of `tile`
+__device__ __forceinline__ TileCoord decode_tile_entry(const GemmArgs& p, int tile, int4 info) {
+  const int bm = p.bm;
   TileCoord c;
   c.e = info.x;
   c.count = info.z;
-  const int mtiles = (c.count + BM - 1) / BM;
+  const int mtiles = (c.count + bm - 1) / bm;
   const int mstart = info.y;
   const int local = tile - mstart * p.n_tiles_n;
   c.nt = local / mtiles;             // tiles of one expert: n-major, m fastest
   c.mt = local - c.nt * mtiles;
-  c.row0 = info.w + c.mt * BM;
+  c.row0 = info.w + c.mt * bm;
   c.gmt = mstart + c.mt;
-  c.rows = min(BM, c.count - c.mt * BM);
+  c.rows = min(bm, c.count - c.mt * bm);
   return c;
 }
+// Walks tiles first, first + stride, ... with the next tile's table entry already requested.
+struct TileCursor {
+  int tile, stride, total;
+  int4 next;
+  __device__ __forceinline__ TileCursor(const GemmArgs& p, int first, int stride_, int total_)
+      : tile(first), stride(stride_), total(total_), next(tile_entry(p, first, total_)) {}
+  __device__ __forceinline__ bool more() const { return tile < total; }
+  // coordinates of the current tile; requests the entry of the one after it
+  __device__ __forceinline__ TileCoord take(const GemmArgs& p) {
+    const TileCoord c = decode_tile_entry(p, tile, next);
+    next = tile_entry(p, tile + stride, total);
+    return c;
+  }
+  __device__ __forceinline__ void advance() { tile += stride; }
+};
 
 // Accumulator slots.  With 256-row weight tiles (every linear1, linear2 by default) the
 // slots are TMEM columns [0, 128) and [128, 256) and the scale factors sit at 256..271: a
@@ -114,10 +137,10 @@ struct SlotPlan {
   int lo, hi;        // slots [lo, hi] this tile uses
   int nt_tok;        // swapped tiles: token columns (MMA N)
 };
-template <bool DOUBLE>
+template <bool DOUBLE, bool SWAP_OK = true>
 __device__ __forceinline__ SlotPlan plan_slots(const GemmArgs& p, const TileCoord& c, int& next_slot) {
   SlotPlan s;
-  s.swap = c.rows <= p.swap_rows;
+  s.swap = SWAP_OK && c.rows <= p.swap_rows;
   s.nt_tok = c.rows <= 32 ? 32 : 64;
   if (s.swap || DOUBLE) {
     s.lo = s.hi = next_slot;
@@ -210,14 +233,15 @@ __device__ __forceinline__ void release_acc(uint64_t* acce, uint32_t acce_remote
   }
 }
 
-// One tile's epilogue; `acc` = TMEM address (lane 0) of the tile's accumulator.
-template <int MODE, int NB = 256>
+// One tile's epilogue; `acc` = TMEM address (lane 0) of the tile's accumulator.  AR: rows of
+// the amax exchange buffer (>= the tile's rows; accumulator rows past them are never stored).
+template <int MODE, int NB = 256, int AR = 128>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord& c, uint32_t acc, int q,
                                               int half, int lane, uint64_t* acce, uint32_t acce_remote,
                                               float* amax_s, int buf, uint8_t* obuf) {
   const int m = q * 32 + lane;                         // accumulator row = TMEM lane
   const uint32_t t_row = acc + ((uint32_t)(q * 32) << 16);
-  const bool valid = c.mt * BM + m < c.count;
+  const bool valid = m < c.rows;                       // rows of this tile of the expert
   if constexpr (MODE == 1) {
     // this warp: h channels [64*half, 64*half + 64) of the tile's 128
     uint32_t g[64], u[64];
@@ -240,10 +264,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& p, const TileCoord
       amax = fmaxf(amax, fabsf(hv));
     }
     // the 128-channel block's amax spans both halves: exchange through shared memory
-    float* slot = amax_s + buf * 256;
-    slot[half * 128 + m] = amax;
+    float* slot = amax_s + buf * 2 * AR;
+    if (m < AR) slot[half * AR + m] = amax;
     epi_bar();
-    amax = fmaxf(amax, slot[(half ^ 1) * 128 + m]);
+    if (m < AR) amax = fmaxf(amax, slot[(half ^ 1) * AR + m]);
     const int pexp = pow2_exp_e4m3(amax);
     const float sc = exp2_neg(pexp);
     uint4 w[4];
@@ -392,15 +416,48 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& p, const TileCoord
   }
 }
 
+// Bounded wait until *ctr >= need, then a gpu-scope acquire.  Polls with relaxed loads and a
+// growing pause (one thread per waiter: callers elect it).  On expiry records
+// MOE_ERR_DEVICE_TIMEOUT at `where` and returns false; returns false at once when `abort_flag`
+// (if given) is raised.
+__device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t need, uint32_t* status,
+                                             uint64_t timeout_ns, uint32_t where, volatile int* abort_flag) {
+  if (ld_acquire_gpu(ctr) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t pause = 32;
+  while (ld_relaxed_gpu(ctr) < need) {
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      report_status(status, kStatusTimeout, where, need);
+      return false;
+    }
+    poll_pause(pause);
+  }
+  fence_acq_rel_gpu();
+  return true;
+}
+
+// Work an epilogue warp does before its first tile or after its last one (the single-kernel
+// forward's scatter and combine); called with the warp's index among all epilogue warps of the
+// grid, their number, and whether the GEMM ran without a device-side failure.
+struct NoEpilogueWork {
+  __device__ __forceinline__ void operator()(int, int, bool) const {}
+};
+
 // One grouped GEMM over tiles cta, cta + n_ctas, ... by all kGemmThreads threads of the CTA,
 // with `tmem_base` holding 512 allocated TMEM columns and `smem` the 1024-aligned dynamic
 // shared memory.  Initialises its barriers on entry and invalidates them on exit, so the
 // same CTA may run it again (the single persistent forward runs linear1, then linear2).
 // NB: weight rows per tile (linear2 may use 224, whose accumulator is double-buffered; tmB's
 // box must then be 224 rows high and the weight scale units laid out for 224-row tiles).
-template <int MODE, class L = SmemLayout, int NB = 256>
+// Readiness (single-kernel forward): with p.rows_ready set, the producer loads no A rows or
+// activation scales before *p.rows_ready >= p.rows_ready_need (weights stream before that); with
+// p.tiles_done set, the epilogue adds 1 to it after each stored tile.  `pre` / `post`: work of
+// the epilogue warps around their tiles (NoEpilogueWork elsewhere).
+template <int MODE, class L = SmemLayout, int NB = 256, class Pre = NoEpilogueWork, class Post = NoEpilogueWork>
 __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& tmB, const GemmArgs& p,
-                                          uint8_t* smem, uint32_t tmem_base, int cta, int n_ctas) {
+                                          uint8_t* smem, uint32_t tmem_base, int cta, int n_ctas,
+                                          const Pre& pre = Pre(), const Post& post = Post()) {
   static_assert(MODE == 2 || NB == 256, "linear1 tiles are 256 weight rows");
   using TM = TmemMap<NB>;
   constexpr int S = L::kStages;
@@ -447,23 +504,42 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int total_tiles = ld_cg(p.mtile_start + p.n_experts) * p.n_tiles_n;
   const int KT = p.K / BK;
+  // the transposed-tile epilogue needs the full amax exchange buffer
+  constexpr bool kSwapOk = L::kAmaxRows >= 128;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t fills[S];
+      // Rows of each stage's A region that may hold data of an earlier tile (all of them at the
+      // start).  With p.zeros set (128-row regions only) the rows a tile's box does not cover are
+      // zeroed by a bulk copy from that buffer before the MMA reads them: the MMA computes all 128
+      // rows whatever the tile holds, and zero operands draw less power than stale rows.
+      constexpr uint32_t kARows = kATileBytes / BK;
+      const bool zero_pad = p.zeros != nullptr && kARows == BM;
+      uint32_t dirty[S];
 #pragma unroll
-      for (int s = 0; s < S; ++s) fills[s] = 0;
+      for (int s = 0; s < S; ++s) {
+        fills[s] = 0;
+        dirty[s] = kARows;
+      }
+      // bytes of the zero copy stage st needs before a box of a_box rows lands (0 if none)
+      auto zero_bytes = [&](int st, uint32_t a_box) -> uint32_t {
+        return zero_pad && dirty[st] > a_box ? (dirty[st] - a_box) * BK : 0u;
+      };
+      auto zero_fill = [&](int st, uint32_t a_box, uint32_t zb) {
+        if (zb != 0) bulk_load(a_s + st * kATileBytes + a_box * BK, p.zeros, zb, &full[st]);
+        dirty[st] = a_box;
+      };
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       bool withhold = p.inject_fault != 0 && cta == 0;
-      // A rows of a tile that belong to its expert decide the A box height; the MMA still
-      // reads 128 rows, the rest are leftovers whose accumulator rows are dropped.  (A
-      // 16-row A region only ever gets the 16-row box.)
+      // A rows of a tile that belong to its expert decide the A box height (16, 32, 64 or 128
+      // rows; never more than the A region, which holds the host-chosen bm rows); the MMA still
+      // reads 128 rows, the rest are leftovers whose accumulator rows are dropped.
       auto a_box_of = [&](const TileCoord& c) {
-        const int rows_here = min(BM, c.count - c.mt * BM);
-        return kATileBytes <= 16 * BK || rows_here <= 16 ? 0 : rows_here <= 32 ? 1 : rows_here <= 64 ? 2 : 3;
+        return c.rows <= 16 ? 0 : c.rows <= 32 ? 1 : c.rows <= 64 ? 2 : 3;
       };
       auto load_b = [&](const TileCoord& c, int st, int kt) {
         if constexpr (MODE == 1) {
@@ -480,19 +556,32 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       // A rows and all scale factors follow the wait.  (Not with the withheld-stage test hook,
       // whose stage must stay empty.)
       int npre = 0;
-      if (cta < total_tiles && !withhold) {
-        const TileCoord c0 = decode_tile(p, cta);
+      TileCursor cur(p, cta, n_ctas, total_tiles);
+      if (cur.more() && !withhold) {
+        const TileCoord c0 = decode_tile_entry(p, cta, cur.next);
         const uint32_t a_box = 16u << a_box_of(c0);
         npre = min(S, KT);
         for (int kt = 0; kt < npre; ++kt) {       // first use of these stages: nothing to wait for
-          mbar_arrive_expect_tx(&full[kt], kStageTxNoA + a_box * BK);
+          const uint32_t zb = zero_bytes(kt, a_box);
+          mbar_arrive_expect_tx(&full[kt], kStageTxNoA + a_box * BK + zb);
           load_b(c0, kt, kt);
+          zero_fill(kt, a_box, zb);
         }
       }
       griddep_wait();
       griddep_launch_dependents();
-      for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
-        const TileCoord c = decode_tile(p, tile);
+      // single-kernel forward: the A rows of every tile exist once the grid's scatter is done
+      bool rows_ok = true;
+      if (p.rows_ready != nullptr) {
+        rows_ok = wait_counter(p.rows_ready, p.rows_ready_need, ctl.status, ctl.timeout_ns, kWhereGemmDependency,
+                               ctl.abort_flag);
+        if (!rows_ok) *ctl.abort_flag = 1;
+        fence_proxy_async_global();          // the acquired rows before this thread's TMA reads
+        if (p.stamp_rows != nullptr) p.stamp_rows[cta] = globaltimer_ns();
+      }
+      for (; cur.more() && ok; cur.advance()) {
+        const int tile = cur.tile;
+        const TileCoord c = cur.take(p);
         const uint8_t* sfa_tile = p.sfa + (long)c.gmt * KT * kSfaBytes;
         const uint8_t* sfb_tile = p.sfb + ((long)c.e * p.n_tiles_n + c.nt) * KT * kSfbBytes;
         const int a_sel = a_box_of(c);
@@ -500,19 +589,12 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
         // chained kernel: this tile's A rows exist once every linear1 tile of its expert is
         // stored (bounded wait; on expiry the stages already requested are still completed, so
         // that the drain below finds every copy accounted for, and nothing further is loaded)
-        bool dep_ok = true;
-        if (p.dep_wait != nullptr) {
-          const uint32_t need = (uint32_t)(((c.count + BM - 1) / BM) * p.dep_per_mtile);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_gpu(p.dep_wait + c.e) < need) {
-            if (*ctl.abort_flag) { dep_ok = false; break; }
-            if (globaltimer_ns() - t0 > ctl.timeout_ns) {
-              report_status(ctl.status, kStatusTimeout, kWhereGemmDependency, (uint32_t)c.e);
-              *ctl.abort_flag = 1;
-              dep_ok = false;
-              break;
-            }
-          }
+        bool dep_ok = rows_ok;
+        if (dep_ok && p.dep_wait != nullptr) {
+          const uint32_t need = (uint32_t)(((c.count + p.bm - 1) / p.bm) * p.dep_per_mtile);
+          dep_ok = wait_counter(p.dep_wait + c.e, need, ctl.status, ctl.timeout_ns, kWhereGemmDependency,
+                                ctl.abort_flag);
+          if (!dep_ok) *ctl.abort_flag = 1;
           fence_proxy_async_global();      // the acquired rows before this thread's TMA reads
         }
         for (int kt = 0; kt < KT; ++kt) {
@@ -523,8 +605,10 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
             withhold = false;            // test hook: this stage never fills
           } else {
             if (!pre) {
-              mbar_arrive_expect_tx(&full[stage], kStageTxNoA + a_box * BK);
+              const uint32_t zb = zero_bytes(stage, a_box);
+              mbar_arrive_expect_tx(&full[stage], kStageTxNoA + a_box * BK + zb);
               load_b(c, stage, kt);
+              zero_fill(stage, a_box, zb);
             }
             tma_load_2d(a_s + stage * kATileBytes, &tmA.m[a_sel], kt * BK, c.row0, &full[stage]);
             bulk_load(sfa_s + stage * kSfaBytes, sfa_tile + kt * kSfaBytes, kSfaBytes, &full[stage]);
@@ -550,9 +634,9 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       uint32_t uses0 = 0, uses1 = 0;      // completed uses of each accumulator slot
       int next_slot = 0;
       bool ok = true;
-      for (int tile = cta; tile < total_tiles && ok; tile += n_ctas) {
-        const TileCoord c = decode_tile(p, tile);
-        const SlotPlan sp = plan_slots<TM::kDouble>(p, c, next_slot);
+      for (TileCursor cur(p, cta, n_ctas, total_tiles); cur.more() && ok; cur.advance()) {
+        const TileCoord c = cur.take(p);
+        const SlotPlan sp = plan_slots<TM::kDouble, kSwapOk>(p, c, next_slot);
         for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
           ok = mbar_wait(&acce[sl], ((sl ? uses1 : uses0) & 1) ^ 1, ctl, kWhereGemmMma);
         if (!ok) break;
@@ -605,42 +689,51 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
     const int q = warp & 3;               // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;      // which half of the accumulator columns
     uint8_t* obuf = L::kStaging ? smem + L::stage_out + (warp - 2) * 2048 : nullptr;
+    const int epi_id = cta * kEpiWarps + (warp - 2), n_epi = n_ctas * kEpiWarps;
+    pre(epi_id, n_epi, true);
     uint32_t uses0 = 0, uses1 = 0;
     int next_slot = 0;
     int buf = 0;
-    for (int tile = cta; tile < total_tiles; tile += n_ctas) {
-      const TileCoord c = decode_tile(p, tile);
-      const SlotPlan sp = plan_slots<TM::kDouble>(p, c, next_slot);
+    bool all_ok = true;
+    for (TileCursor cur(p, cta, n_ctas, total_tiles); cur.more(); cur.advance()) {
+      const TileCoord c = cur.take(p);
+      const SlotPlan sp = plan_slots<TM::kDouble, kSwapOk>(p, c, next_slot);
       bool ok = true;
       for (int sl = sp.lo; sl <= sp.hi && ok; ++sl)
         ok = mbar_wait(&accf[sl], (sl ? uses1 : uses0) & 1, ctl, kWhereGemmEpilogue);
       // epilogue-uniform decision: tcgen05.ld below is .sync.aligned and the epilogue syncs
-      if (!epi_all(ok)) break;
+      if (!epi_all(ok)) {
+        all_ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t acc = tmem_base + kAccCol + sp.lo * TM::slot_stride;
-      if (sp.swap) {
+      if (kSwapOk && sp.swap) {
         if (sp.nt_tok == 32)
           epilogue_swap<MODE, 32, NB>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
         else
           epilogue_swap<MODE, 64, NB>(p, c, acc, q, half, lane, &acce[sp.lo], amax_s, buf);
       } else {
-        epilogue_tile<MODE, NB>(p, c, acc, q, half, lane, TM::kDouble ? &acce[sp.lo] : acce, 0u, amax_s, buf,
-                                obuf);
+        epilogue_tile<MODE, NB, L::kAmaxRows>(p, c, acc, q, half, lane, TM::kDouble ? &acce[sp.lo] : acce, 0u,
+                                              amax_s, buf, obuf);
       }
-      if (p.dep_signal != nullptr) {
-        // chained kernel: publish this tile's h rows and scale words to the linear2 producers
-        // (generic stores -> other CTAs' TMA reads: proxy fence, CTA barrier, gpu-scope release)
+      if (p.dep_signal != nullptr || p.tiles_done != nullptr) {
+        // chained kernel / single-kernel forward: publish this tile's rows (h and its scale words
+        // to the linear2 producers; bf16 rows to the combine): generic stores -> other CTAs'
+        // TMA or generic reads: proxy fence, CTA barrier, gpu-scope release
         fence_proxy_async_global();
         epi_bar();
         if (threadIdx.x == 2 * 32) {
           __threadfence();
-          atomicAdd(p.dep_signal + c.e, 1u);
+          if (p.dep_signal != nullptr) atomicAdd(p.dep_signal + c.e, 1u);
+          if (p.tiles_done != nullptr) atomicAdd(p.tiles_done, 1u);
         }
       }
       uses0 += sp.lo == 0;
       uses1 += sp.hi == 1;
       buf ^= 1;
     }
+    post(epi_id, n_epi, all_ok && !*abort_flag);
   }
 
   __syncthreads();
@@ -1137,9 +1230,14 @@ __global__ void split_router_weights_kernel(const float* __restrict__ W, __nv_bf
 
 // ------------------------------------------------------------------ the single persistent forward
 // Shared memory of the fused kernel: the largest step layout, then the kernel-lifetime words.
-constexpr uint32_t kFusedMiscOffset = (SmemLayout::total + 15) & ~15u;
-static_assert(kFusedMiscOffset >= RouterSmem::total && kFusedMiscOffset >= sizeof(TopkSmem),
-              "every step's shared memory must fit below the fused kernel's own words");
+template <class L>
+struct FusedSmem {
+  static constexpr uint32_t misc = (L::total + 15) & ~15u;
+  static constexpr uint32_t bytes = misc + 16 + 1024;
+  static_assert(misc >= RouterSmem::total && misc >= sizeof(TopkSmem) + 3 * 32 * 4,
+                "every step's shared memory must fit below the fused kernel's own words");
+  static_assert(bytes <= 232448, "fused kernel exceeds shared memory");
+};
 // Grid-wide barrier for a cooperative launch: bar[0] counts arrivals, bar[1] is the
 // generation the last arrival advances.  The wait is bounded; on expiry the CTA records
 // MOE_ERR_DEVICE_TIMEOUT and the barrier reports false.  All threads call it.
@@ -1156,21 +1254,22 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32
       st_release_gpu(&bar[1], gen + 1);
     } else {
       const uint64_t t0 = globaltimer_ns();
-      for (uint32_t spin = 0; ld_acquire_gpu(&bar[1]) == gen; ++spin) {
-        if ((spin & 63) == 63 && globaltimer_ns() - t0 > timeout_ns) {
+      uint32_t pause = 32;
+      while (ld_relaxed_gpu(&bar[1]) == gen) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
           report_status(status, kStatusTimeout, kWhereGridBarrier, gen);
           ok = false;
           break;
         }
+        poll_pause(pause);
       }
+      fence_acq_rel_gpu();
     }
     *ok_smem = ok && ld_acquire_gpu(status) == 0u;
   }
   __syncthreads();
   return *ok_smem != 0;
 }
-
-// Generic-proxy stores made visible to later TMA (async-proxy) reads of the same data.
 
 template <int KMAX, int U>
 __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, long first, long stride) {
@@ -1182,18 +1281,76 @@ __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, lo
   }
 }
 
+// Before its first linear1 tile, each epilogue warp of the grid scatters (and quantises) its
+// share of the (token, 256-channel slice) items; once all eight of a CTA's have, one thread adds
+// 1 to the scatter counter (one atomic per CTA, not per warp); the producers load A rows only
+// once every CTA has done so.
+struct ScatterWork {
+  const FusedArgs* a;
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool) const {
+    const FusedArgs& f = *a;
+    const int slices = (f.H + 255) / 256;
+    if ((long)f.T * slices >= 32768) {
+      // many items: four slices per item, their x loads issued before the position lookups
+      const long items = (long)f.T * ((slices + 3) / 4);
+      for (long it = epi_id; it < items; it += n_epi)
+        scatter_items<4>(it, f.x, f.topk_ids, f.local_rank, f.group_base, f.offsets, f.mtile_start, f.slot_pos,
+                         f.perm, f.xq, f.xsf, f.T, f.H, f.E, f.k, f.shared, f.bm);
+    } else {
+      const long items = (long)f.T * slices;
+      for (long it = epi_id; it < items; it += n_epi)
+        scatter_item(it, f.x, f.topk_ids, f.local_rank, f.group_base, f.offsets, f.mtile_start, f.slot_pos, f.perm,
+                     f.xq, f.xsf, f.T, f.H, f.E, f.k, f.shared, f.bm);
+    }
+    // generic stores -> other CTAs' TMA reads: proxy fence, CTA barrier, gpu-scope release
+    fence_proxy_async_global();
+    epi_bar();
+    if (threadIdx.x == 2 * 32) {
+      if (f.stamps != nullptr) f.stamps[kStampScatterDone * kStampMaxCtas + blockIdx.x] = globaltimer_ns();
+      __threadfence();
+      atomicAdd(f.counters + 0, 1u);
+    }
+  }
+};
+
+// After its last linear2 tile, each epilogue warp waits (bounded) until every linear2 tile of
+// the grid is stored, then combines its share of the (token, slice) items.
+struct CombineWork {
+  const FusedArgs* a;
+  uint32_t tiles2;                 // linear2 tiles of the forward
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool ok) const {
+    const FusedArgs& f = *a;
+    if (!ok) return;
+    // lane 0 polls for the warp
+    bool ready = true;
+    if (threadIdx.x % 32 == 0)
+      ready = wait_counter(f.counters + 1, tiles2, f.status, f.timeout_ns, kWhereGemmDependency + 1, nullptr);
+    ready = __shfl_sync(0xffffffffu, ready, 0);
+    __syncwarp();
+    if (!ready) return;
+    if (f.stamps != nullptr && threadIdx.x == 2 * 32) f.stamps[kStampCombine * kStampMaxCtas + blockIdx.x] = globaltimer_ns();
+    const long items = (long)f.T * ((f.H + 255) / 256);
+    // several items per warp in flight: one CTA per SM leaves only 8 epilogue warps to hide latency
+    if (f.k <= 2) fused_combine<2, 4>(f, items, epi_id, n_epi);
+    else if (f.k <= 4) fused_combine<4, 4>(f, items, epi_id, n_epi);
+    else if (f.k <= 8) fused_combine<8, 2>(f, items, epi_id, n_epi);
+    else fused_combine<16, 1>(f, items, epi_id, n_epi);
+  }
+};
+
+template <class L, int NB2>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fused_forward_kernel(const __grid_constant__ AMaps amA1, const __grid_constant__ AMaps amA2,
                          const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                          const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWhi,
                          const __grid_constant__ CUtensorMap tmWlo, const FusedArgs a) {
+  using FS = FusedSmem<L>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // kernel-lifetime words past every step's own layout
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kFusedMiscOffset);
-  volatile int* ok_smem = reinterpret_cast<volatile int*>(smem + kFusedMiscOffset + 8);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  (void)lane;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + FS::misc);
+  volatile int* ok_smem = reinterpret_cast<volatile int*>(smem + FS::misc + 8);
+  const int warp = threadIdx.x / 32;
   constexpr int NW = kGemmThreads / 32;
   const int cta = blockIdx.x, n_ctas = gridDim.x;
   if (warp == 1) {
@@ -1201,11 +1358,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  // the readiness counters start at zero (visible to every CTA after the first grid barrier)
+  if (cta == 0)
+    for (int i = threadIdx.x; i < 2 + a.E + a.shared; i += blockDim.x) a.counters[i] = 0u;
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long wstride = (long)n_ctas * NW, wfirst = (long)cta * NW + warp;
   const int G = (a.T + 31) / 32;
+  auto stamp = [&](int id) {
+    if (a.stamps != nullptr && threadIdx.x == 0) a.stamps[id * kStampMaxCtas + cta] = globaltimer_ns();
+  };
+  stamp(kStampStart);
 
   bool ok = true;
   // S1 router
@@ -1216,6 +1380,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       router_tc_item(tmX, tmWhi, tmWlo, a.ra, smem, tmem_base, (tile / nt) * 128, (tile % nt) * RBN, split,
                      a.router_parts);
     }
+  } else if (a.router_kind == kRouterSplitK) {
+    router_splitk_items<kSplitKMaxT, kSplitKMaxChunks>(a.x, a.W_router, a.logits, a.T, a.H, a.E, a.router_parts,
+                                                       wfirst, wstride);
   } else if (a.router_kind == kRouterSplitBlock) {
     float* part = reinterpret_cast<float*>(smem);
     for (int it = cta; it < a.E * a.T; it += n_ctas)
@@ -1225,51 +1392,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     router_warp_items<2>(a.x, a.W_router, a.logits, a.T, a.H, a.E, wfirst, wstride);
   }
+  if (a.stamps != nullptr) {
+    __syncthreads();
+    stamp(kStampRouterDone);
+  }
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem);
-  // S2 top-k, gates, ranks inside each group of 32 tokens
-  if (ok) {
-    TopkSmem& tsm = *reinterpret_cast<TopkSmem*>(smem);
-    for (int g = cta; g < G; g += n_ctas)
-      topk_rank_group<kGemmThreads>(g, 0, a.logits, a.router_parts, a.bias, a.topk_ids, a.gates, a.local_rank,
+  stamp(kStampRouted);
+  // S2 + dispatch scans
+  if (G == 1) {
+    // one token group: top-k, ranks, counts and the expert scan in CTA 0 (the group's per-expert
+    // masks stay in shared memory)
+    if (ok && cta == 0) {
+      TopkSmem& tsm = *reinterpret_cast<TopkSmem*>(smem);
+      int32_t(*wsum)[32] = reinterpret_cast<int32_t(*)[32]>(smem + sizeof(TopkSmem));
+      topk_rank_group<kGemmThreads>(0, 0, a.logits, a.router_parts, a.bias, a.topk_ids, a.gates, a.local_rank,
                                     a.group_counts, a.status, a.T, a.E, a.k, tsm);
+      stamp(kStampTopkDone);
+      // topk_rank_group leaves the masks in place (its last barrier follows the count writes)
+      int32_t* cnt_s = reinterpret_cast<int32_t*>(tsm.mask);
+      for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        const int c = __popc(tsm.mask[e]);
+        cnt_s[e] = c;
+        a.counts[e] = c;
+        a.group_base[e] = 0;
+      }
+      __syncthreads();
+      expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.tile_info, a.ptile_info,
+                                      a.T, a.E, a.shared, a.bm, wsum, cnt_s);
+      stamp(kStampScanDone);
+    }
+  } else {
+    if (ok) {
+      TopkSmem& tsm = *reinterpret_cast<TopkSmem*>(smem);
+      for (int g = cta; g < G; g += n_ctas)
+        topk_rank_group<kGemmThreads>(g, 0, a.logits, a.router_parts, a.bias, a.topk_ids, a.gates, a.local_rank,
+                                      a.group_counts, a.status, a.T, a.E, a.k, tsm);
+      stamp(kStampTopkDone);
+    }
+    ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+    if (ok)
+      for (long e = wfirst; e < a.E; e += wstride)
+        column_scan_warp((int)e, a.group_counts, a.group_base, a.counts, G, a.E);
+    ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+    if (ok && cta == 0) {
+      expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.tile_info, a.ptile_info,
+                                      a.T, a.E, a.shared, a.bm, reinterpret_cast<int32_t(*)[32]>(smem));
+      stamp(kStampScanDone);
+    }
   }
   ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
-  // S3 dispatch: per-expert group scan, expert scan, then scatter + quantisation
-  if (ok)
-    for (long e = wfirst; e < a.E; e += wstride) column_scan_warp((int)e, a.group_counts, a.group_base, a.counts, G, a.E);
-  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
-  if (ok && cta == 0)
-    expert_scan_block<kGemmThreads>(a.counts, a.offsets, a.mtile_start, a.ptile_start, a.tile_info, a.ptile_info,
-                                    a.T, a.E, a.shared, reinterpret_cast<int32_t(*)[32]>(smem));
-  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
+  stamp(kStampScanned);
+  // S3 scatter (epilogue warps, before their first linear1 tile) + S4 linear1: the producers
+  // stream weights at once and load A rows once every epilogue warp of the grid has scattered
   if (ok) {
-    const long items = (long)a.T * ((a.H + 255) / 256);
-    for (long it = wfirst; it < items; it += wstride)
-      scatter_item(it, a.x, a.topk_ids, a.local_rank, a.group_base, a.offsets, a.mtile_start, a.slot_pos, a.perm,
-                   a.xq, a.xsf, a.T, a.H, a.E, a.k, a.shared);
-  }
-  fence_proxy_async_global();
-  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
-  // S4 linear1 + SwiGLU + requantisation
-  if (ok) gemm_body<1>(amA1, tmB1, a.g1, smem, tmem_base, cta, n_ctas);
-  fence_proxy_async_global();
-  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
-  // S5 linear2
-  if (ok) {
-    if (a.g2.bn == kGemmBN2Double)
-      gemm_body<2, SmemLayout, kGemmBN2Double>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
-    else
-      gemm_body<2>(amA2, tmB2, a.g2, smem, tmem_base, cta, n_ctas);
-  }
-  ok = grid_sync(a.gridbar, n_ctas, a.status, a.timeout_ns, ok_smem) && ok;
-  // S6 combine
-  if (ok) {
-    const long items = (long)a.T * ((a.H + 255) / 256);
-    // several items per warp in flight: one CTA per SM leaves only 10 warps to hide latency
-    if (a.k <= 2) fused_combine<2, 4>(a, items, wfirst, wstride);
-    else if (a.k <= 4) fused_combine<4, 4>(a, items, wfirst, wstride);
-    else if (a.k <= 8) fused_combine<8, 2>(a, items, wfirst, wstride);
-    else fused_combine<16, 1>(a, items, wfirst, wstride);
+    GemmArgs g1 = a.g1;
+    g1.rows_ready = a.counters + 0;
+    g1.rows_ready_need = (uint32_t)n_ctas;
+    g1.dep_signal = a.counters + 2;
+    g1.stamp_rows = a.stamps != nullptr ? a.stamps + kStampRowsReady * kStampMaxCtas : nullptr;
+    gemm_body<1, L, 256, ScatterWork>(amA1, tmB1, g1, smem, tmem_base, cta, n_ctas, ScatterWork{&a});
+    stamp(kStampLinear1);
+    // S5 linear2: each tile's producer waits only for its expert's linear1 tiles; S6 combine by
+    // the epilogue warps once every linear2 tile is stored
+    GemmArgs g2 = a.g2;
+    g2.dep_wait = a.counters + 2;
+    g2.dep_per_mtile = a.g1.n_tiles_n;
+    g2.tiles_done = a.counters + 1;
+    const uint32_t tiles2 = (uint32_t)(ld_cg(a.mtile_start + a.E + a.shared) * a.g2.n_tiles_n);
+    gemm_body<2, L, NB2, NoEpilogueWork, CombineWork>(amA2, tmB2, g2, smem, tmem_base, cta, n_ctas,
+                                                      NoEpilogueWork(), CombineWork{&a, tiles2});
+    stamp(kStampEnd);
   }
   __syncthreads();
   if (warp == 1) {
@@ -1309,8 +1501,11 @@ cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* 
 size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
 size_t gemm_small_smem_bytes() { return SmallSmem::total + 1024; }
 size_t gemm_pair_smem_bytes() { return PairSmem::total + 1024; }
-size_t fused_smem_bytes() { return kFusedMiscOffset + 16 + 1024; }
 int g_fused_ctas[64] = {};
+struct FusedVariant {
+  const void* fn;
+  size_t smem;
+};
 int g_pair_clusters[64] = {};
 
 cudaError_t gemm_prepare_device() {
@@ -1366,16 +1561,25 @@ cudaError_t gemm_prepare_device() {
   e = cudaOccupancyMaxActiveClusters(&clusters, (const void*)grouped_gemm_pair_kernel<1>, &cfg);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64) g_pair_clusters[dev] = clusters;
-  // the fused forward: one CTA per SM, all co-resident (cooperative launch)
-  e = cudaFuncSetAttribute(fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem_bytes());
-  if (e != cudaSuccess) return e;
-  int per_sm = 0, sms = 0, coop = 0;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_forward_kernel, kGemmThreads,
-                                                         fused_smem_bytes())) != cudaSuccess)
-    return e;
+  // the fused forward: one CTA per SM, all co-resident (cooperative launch); every variant has the
+  // same block shape and (nearly) all of shared memory, so the smallest co-resident count counts
+  int per_sm_min = 1 << 30, sms = 0, coop = 0;
+  const FusedVariant variants[] = {
+      {(const void*)fused_forward_kernel<SmemLayout, kGemmBN>, FusedSmem<SmemLayout>::bytes},
+      {(const void*)fused_forward_kernel<SmemLayout, kGemmBN2Double>, FusedSmem<SmemLayout>::bytes},
+      {(const void*)fused_forward_kernel<SmallSmem, kGemmBN>, FusedSmem<SmallSmem>::bytes},
+      {(const void*)fused_forward_kernel<SmallSmem, kGemmBN2Double>, FusedSmem<SmallSmem>::bytes}};
+  for (const FusedVariant& v : variants) {
+    e = cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)v.smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, kGemmThreads, v.smem)) != cudaSuccess)
+      return e;
+    per_sm_min = per_sm < per_sm_min ? per_sm : per_sm_min;
+  }
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64) g_fused_ctas[dev] = coop ? per_sm * sms : 0;
+  if (dev >= 0 && dev < 64) g_fused_ctas[dev] = coop ? per_sm_min * sms : 0;
   return cudaSuccess;
 }
 
@@ -1387,13 +1591,25 @@ int fused_max_ctas() {
 
 cudaError_t launch_fused_forward(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
                                  const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
-                                 const FusedArgs& args, int ctas, cudaStream_t s) {
+                                 const FusedArgs& args, int ctas, bool small_tiles, cudaStream_t s) {
   if (ctas < 1 || ctas > fused_max_ctas()) return cudaErrorInvalidValue;
+  if (args.g2.bn != kGemmBN && args.g2.bn != kGemmBN2Double) return cudaErrorInvalidValue;
+  if (small_tiles && (args.bm != kGemmBMSmall || args.g1.swap_rows != 0 || args.g2.swap_rows != 0))
+    return cudaErrorInvalidValue;
+  if (args.router_kind == kRouterSplitK &&
+      (args.T > kSplitKMaxT || args.router_parts < 1 ||
+       ((args.H + 255) / 256 + args.router_parts - 1) / args.router_parts > kSplitKMaxChunks))
+    return cudaErrorInvalidValue;
   void* params[] = {const_cast<AMaps*>(&a1), const_cast<AMaps*>(&a2), const_cast<CUtensorMap*>(&b1),
                     const_cast<CUtensorMap*>(&b2), const_cast<CUtensorMap*>(&x), const_cast<CUtensorMap*>(&whi),
                     const_cast<CUtensorMap*>(&wlo), const_cast<FusedArgs*>(&args)};
-  return cudaLaunchCooperativeKernel((const void*)fused_forward_kernel, dim3(ctas), dim3(kGemmThreads), params,
-                                    fused_smem_bytes(), s);
+  const bool d = args.g2.bn == kGemmBN2Double;
+  const void* fn = small_tiles ? (d ? (const void*)fused_forward_kernel<SmallSmem, kGemmBN2Double>
+                                    : (const void*)fused_forward_kernel<SmallSmem, kGemmBN>)
+                               : (d ? (const void*)fused_forward_kernel<SmemLayout, kGemmBN2Double>
+                                    : (const void*)fused_forward_kernel<SmemLayout, kGemmBN>);
+  const size_t smem = small_tiles ? FusedSmem<SmallSmem>::bytes : FusedSmem<SmemLayout>::bytes;
+  return cudaLaunchCooperativeKernel(fn, dim3(ctas), dim3(kGemmThreads), params, smem, s);
 }
 
 int gemm_pair_max_clusters() {
@@ -1404,28 +1620,32 @@ int gemm_pair_max_clusters() {
 
 cudaError_t launch_gemm_pair_linear1(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
                                      const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
+  if (args.bm != kGemmBM) return cudaErrorInvalidValue;
   return launch_kernel(grouped_gemm_pair_kernel<1>, 2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s, a, b, sfa,
                        sfb, args);
 }
 
 cudaError_t launch_gemm_pair_linear2(const AMaps& a, const CUtensorMap& b, const CUtensorMap& sfa,
                                      const CUtensorMap& sfb, const GemmArgs& args, int pairs, cudaStream_t s) {
+  if (args.bm != kGemmBM) return cudaErrorInvalidValue;
   return launch_kernel(grouped_gemm_pair_kernel<2>, 2 * pairs, kGemmThreads, gemm_pair_smem_bytes(), s, a, b, sfa,
                        sfb, args);
 }
 
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s, bool few_rows) {
-  if (few_rows)
+                                cudaStream_t s, bool small_tiles) {
+  if (small_tiles && (args.bm > kGemmBMSmall || args.swap_rows != 0)) return cudaErrorInvalidValue;
+  if (small_tiles)
     return launch_kernel(grouped_gemm_kernel<1, SmallSmem>, grid, kGemmThreads, gemm_small_smem_bytes(), s, a, b, args);
   return launch_kernel(grouped_gemm_kernel<1, SmemLayout>, grid, kGemmThreads, gemm_smem_bytes(), s, a, b, args);
 }
 
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s, bool few_rows) {
+                                cudaStream_t s, bool small_tiles) {
   constexpr int D = kGemmBN2Double;
   if (args.bn != kGemmBN && args.bn != D) return cudaErrorInvalidValue;
-  if (few_rows)
+  if (small_tiles && (args.bm > kGemmBMSmall || args.swap_rows != 0)) return cudaErrorInvalidValue;
+  if (small_tiles)
     return args.bn == D ? launch_kernel(grouped_gemm_kernel<2, SmallSmem, D>, grid, kGemmThreads,
                                         gemm_small_smem_bytes(), s, a, b, args)
                         : launch_kernel(grouped_gemm_kernel<2, SmallSmem>, grid, kGemmThreads,
@@ -1445,6 +1665,8 @@ cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMa
   const void* k = g2.bn == kGemmBN2Double ? reinterpret_cast<const void*>(chained_gemm_kernel<kGemmBN2Double>)
                                           : reinterpret_cast<const void*>(chained_gemm_kernel<kGemmBN>);
   if (g2.bn != kGemmBN && g2.bn != kGemmBN2Double) return cudaErrorInvalidValue;
+  if (g1.bm > kGemmBMSmall || g2.bm > kGemmBMSmall || g1.swap_rows != 0 || g2.swap_rows != 0)
+    return cudaErrorInvalidValue;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kGemmThreads, gemm_small_smem_bytes())) !=
       cudaSuccess)
     return e;

@@ -38,6 +38,10 @@ int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 
 // ---- grouped block-scaled GEMMs (gemm_sm100.cu) --------------------------------
 constexpr int kGemmBM = 128;      // rows (tokens) per tile
+// Row tiles of 32 rows: for layers whose experts get few rows each (decode), the GEMMs use a
+// shared-memory layout with 32-row A regions and 6 pipeline stages (more weight bytes in
+// flight per SM); the MMA still has M = 128, the rows past the tile are never stored.
+constexpr int kGemmBMSmall = 32;
 constexpr int kGemmBN = 256;      // accumulator columns per tile
 constexpr int kGemmBK = 128;      // K per pipeline stage
 constexpr int kGemmStages = 4;
@@ -50,10 +54,11 @@ constexpr int kGemmThreads = 320; // 10 warps: TMA, MMA, 8 x epilogue
 // Scale-factor atoms (the unit the MMA's scale copy reads): 128 rows x 4 K-blocks
 // of 32, row r at byte (r%32)*16 + (r/32)*4, K-block b at +b.
 //   activations: [row tile g = mtile_start[e] + mt][K/128] atoms of 512 B, the
-//                row's power-of-two code in all four bytes;
+//                row's power-of-two code in all four bytes (row r < bm of the tile);
 //   weights:     [expert][n-tile][K/128] units of 1024 B (two atoms: the tile's
 //                B rows 0..127 and 128..255).
 struct GemmArgs {
+  int bm;              // rows per row tile: kGemmBM, or kGemmBMSmall (small-tile layout only)
   int K;               // reduction length (H for linear1, I for linear2)
   int N;               // linear1: I (SwiGLU width); linear2: H (output width)
   int rows_b;          // B rows per expert (2I or H)
@@ -64,7 +69,7 @@ struct GemmArgs {
   int swap_rows;       // tiles with at most this many expert rows run transposed (0, 32 or 64)
   const int32_t* counts;       // [n_experts]
   const int32_t* offsets;      // [n_experts + 1]
-  const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/128)
+  const int32_t* mtile_start;  // [n_experts + 1] prefix sum of ceil(count/bm)
   const int32_t* ptile_start;  // [n_experts + 1] prefix sum of ceil(ceil(count/128)/2) (CTA pairs)
   // Row-tile table: entry g in [mtile_start[e], mtile_start[e + 1]) holds {e, mtile_start[e],
   // counts[e], offsets[e]}; the CTA-pair table the same over ptile_start with ptile_start[e]
@@ -73,10 +78,19 @@ struct GemmArgs {
   const int4* ptile_info;
   // Chained linear1 -> linear2 in one kernel: linear1's epilogue adds 1 to dep_signal[e] when a
   // tile of expert e is stored; linear2's producer loads a tile's A rows only once
-  // dep_wait[e] >= ceil(count_e / 128) * dep_per_mtile.  Null outside the chained kernel.
+  // dep_wait[e] >= ceil(count_e / bm) * dep_per_mtile.  Null outside the chained kernel.
   uint32_t* dep_signal;
   const uint32_t* dep_wait;
   int dep_per_mtile;
+  // Single-kernel forward (null elsewhere): the producer loads no A rows or activation scales
+  // before *rows_ready >= rows_ready_need (the grid's scatter is done); the epilogue adds 1 to
+  // *tiles_done after each stored tile.
+  const uint32_t* rows_ready;
+  uint32_t rows_ready_need;
+  uint32_t* tiles_done;
+  // phase timing of the single-kernel forward (null unless asked for): the producer writes the
+  // global timer into stamp_rows[cta] once the rows are ready
+  unsigned long long* stamp_rows;
   const uint8_t* sfa;          // activation scale atoms
   const uint8_t* sfb;          // weight scale units
   uint8_t* hq;                 // linear1 out: [rows_total][I] E4M3
@@ -85,7 +99,11 @@ struct GemmArgs {
   uint32_t* status;
   uint64_t timeout_ns;
   int inject_fault;
+  // 16 KB of zeros (16-byte aligned): with 128-row A regions, the A rows past a tile's box are
+  // zeroed from it (null = leave them as they are)
+  const uint8_t* zeros;
 };
+constexpr size_t kGemmZeroBytes = 16384;
 
 size_t gemm_smem_bytes();
 cudaError_t gemm_prepare_device();   // sets the kernels' shared-memory attributes
@@ -99,13 +117,13 @@ cudaError_t launch_tile_weight_scales(const uint8_t* src, uint8_t* dst, int n_ex
 struct AMaps {
   CUtensorMap m[4];
 };
-// few_rows: every expert has at most 16 rows (T <= 16), so the kernel may use 16-row A regions
-// and 6 pipeline stages.
+// small_tiles: args.bm == kGemmBMSmall, so the kernel uses the layout with 32-row A regions and
+// 6 pipeline stages (no transposed tiles: args.swap_rows must be 0).
 cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s, bool few_rows = false);
+                                cudaStream_t s, bool small_tiles = false);
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
-                                cudaStream_t s, bool few_rows = false);
-// linear1 + linear2 in one cooperative launch (few-row layout, at most 16 rows per expert):
+                                cudaStream_t s, bool small_tiles = false);
+// linear1 + linear2 in one cooperative launch (small-tile layout, bm == kGemmBMSmall):
 // g1.dep_signal == g2.dep_wait (n_experts counters, zero before the launch), g2.dep_per_mtile =
 // g1.n_tiles_n; b2's box height = g2.bn.  grid <= the co-resident CTAs of the device.
 cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
@@ -141,14 +159,22 @@ cudaError_t launch_router_tc(const CUtensorMap& x, const CUtensorMap& whi, const
 cudaError_t launch_split_router_weights(const float* W, uint16_t* hi, uint16_t* lo, long n, cudaStream_t s);
 
 // ---- the single persistent forward (gemm_sm100.cu) -------------------------------
-// Every step of the forward in one cooperative launch of one CTA per SM (kGemmThreads
-// threads), the steps separated by grid-wide barriers: router, top-k + rank, per-expert
-// group scan, expert scan, dispatch + quantisation, linear1, linear2, combine.
-enum : int { kRouterSplitBlock = 0, kRouterWarp8 = 1, kRouterWarp2 = 2, kRouterTensor = 3 };
+// Every step of the forward in one cooperative launch of one CTA per SM (kGemmThreads threads).
+// Grid-wide barriers only where every CTA needs every other CTA's result: after the router, and
+// after the top-k / dispatch scans (with more than 32 tokens also between top-k, the per-expert
+// group scan and the expert scan).  From there on readiness counters replace barriers: the
+// GEMM producers stream weights at once and load A rows when the grid's scatter (done by the
+// epilogue warps before their first linear1 tile) is complete; linear2 tiles wait per expert for
+// its linear1 tiles; the combine (epilogue warps after their last linear2 tile) waits for all
+// linear2 tiles.
+enum : int { kRouterSplitBlock = 0, kRouterWarp8 = 1, kRouterWarp2 = 2, kRouterTensor = 3, kRouterSplitK = 4 };
+// kRouterSplitK: tokens per launch and 256-channel chunks per K part it handles
+constexpr int kSplitKMaxT = 16, kSplitKMaxChunks = 8;
 struct FusedArgs {
   int T, H, E, k, shared;
+  int bm;                          // rows per row tile of the GEMMs
   int router_kind;                 // kRouter*
-  int router_parts;                // partial logit arrays (tensor-core router K splits)
+  int router_parts;                // partial logit arrays (tensor-core router K splits, split-K parts)
   const uint16_t* x;
   const float* W_router;
   const float* bias;
@@ -171,14 +197,36 @@ struct FusedArgs {
   const uint16_t* y;
   uint16_t* out;
   uint32_t* status;
-  uint32_t* gridbar;               // [2] arrival count, generation (zeroed once per workspace)
+  uint32_t* gridbar;               // [2] arrival count, generation (zeroed before each launch)
+  // [0] scatter warps done, [1] linear2 tiles stored, [2 .. 2 + n) linear1 tiles stored per
+  // expert: zeroed inside the kernel before the first grid barrier
+  uint32_t* counters;
+  // phase timing (MOE_OPT_PHASE_EVENTS; null otherwise): stamps[id * kStampMaxCtas + cta] = the
+  // global timer (ns) when CTA cta passed point id (kStamp*)
+  unsigned long long* stamps;
   uint64_t timeout_ns;
   RouterArgs ra;
   GemmArgs g1, g2;
 };
+enum : int {
+  kStampStart = 0,     // TMEM allocated
+  kStampRouted,        // past the grid barrier that follows the router
+  kStampScanned,       // past the grid barrier that follows top-k and the dispatch scans
+  kStampRowsReady,     // the linear1 producer saw every CTA's scatter done
+  kStampLinear1,       // the CTA's linear1 tiles stored
+  kStampCombine,       // every linear2 tile stored, combine starts (first epilogue warp)
+  kStampEnd,           // the CTA's combine items written
+  kStampRouterDone,    // the CTA's own router items done (before the barrier)
+  kStampTopkDone,      // top-k of the CTA's token groups done (before the scans)
+  kStampScanDone,      // the expert scan done (CTA 0)
+  kStampScatterDone,   // the CTA's epilogue warps finished their scatter items
+  kStampCount
+};
+constexpr int kStampMaxCtas = 1024;
+// small_tiles: the 32-row, 6-stage GEMM layout (g1.bm == kGemmBMSmall); g2.bn = 224 or 256.
 cudaError_t launch_fused_forward(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
                                  const CUtensorMap& x, const CUtensorMap& whi, const CUtensorMap& wlo,
-                                 const FusedArgs& args, int ctas, cudaStream_t s);
+                                 const FusedArgs& args, int ctas, bool small_tiles, cudaStream_t s);
 int fused_max_ctas();                // co-resident CTAs of the fused kernel (after gemm_prepare_device)
 
 // ---- routing / dispatch / combine (path_kernels.cu) -----------------------------
@@ -198,17 +246,18 @@ cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_part
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
                                       int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                      int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s);
-// counts, offsets, mtile_start, ptile_start (n + 1 entries), the row-tile tables (see GemmArgs)
-// and group_base[g][e] = rows of expert e in token groups < g (relative to offsets[e]).
+                                      int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s);
+// counts, offsets, mtile_start (bm-row tiles), ptile_start (pairs of 128-row tiles) (n + 1
+// entries), the row-tile tables (see GemmArgs) and group_base[g][e] = rows of expert e in token
+// groups < g (relative to offsets[e]).
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                 int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s);
-// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms.
+                                 int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s);
+// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms (bm-row tiles).
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
-                                 int k, int shared, cudaStream_t s);
+                                 int k, int shared, int bm, cudaStream_t s);
 // Token-order quantisation (debug entry point).
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s);
 // Auxiliary-loss-free balancing step from the routed experts' loads.

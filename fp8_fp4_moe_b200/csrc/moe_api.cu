@@ -34,6 +34,8 @@ struct moe_plan_s {
   int dep_launch = 1;               // MOE_OPT_DEPENDENT_LAUNCH
   int l2_tile_rows = 0;             // MOE_OPT_L2_TILE_ROWS
   int chain = 0;                    // MOE_OPT_CHAIN
+  int tile_rows = 0;                // MOE_OPT_TILE_ROWS
+  int zero_pad = 0;                 // MOE_OPT_ZERO_PAD
   int router_splits = 1;            // K splits of the tensor-core router (partial logit arrays)
   // workspace layout
   size_t region_off[MOE_REGION_COUNT_];
@@ -42,7 +44,11 @@ struct moe_plan_s {
   size_t off_tinfo, off_ptinfo;     // row-tile tables of the grouped GEMMs (mt_cap int4 each)
   size_t off_dep;                   // per-expert linear1 tile counters of the chained GEMM kernel
   size_t off_gridbar;               // grid barrier words of the fused forward
-  long long mt_cap;                 // bound on row tiles: ceil(rows/128) + n
+  size_t off_zeros;                 // kGemmZeroBytes of zeros (A-region padding source)
+  size_t off_counters;              // readiness counters of the fused forward (2 + n words)
+  int fused_ctas_last = 0;          // CTAs of the last fused launch with stamps (0: none)
+  int splitk_parts = 1;             // K parts of the fused forward's split-K router (few tokens)
+  long long mt_cap;                 // bound on row tiles: ceil(rows/32) + n (any row-tile height)
   size_t total;
   // bound state
   uint8_t* ws = nullptr;
@@ -130,9 +136,33 @@ int check_bound(moe_plan_t p) {
   return MOE_OK;
 }
 
-// CTA-pair GEMMs (M = 256 per pair) when experts average at least 256 rows, or when forced.
+// Rows per GEMM row tile: 32 (small-tile layout: 32-row A regions, 6 stages) when the routed
+// experts average at most 32 rows -- decode, where each expert's weights stream past a handful
+// of rows and the pipeline depth decides the bandwidth -- unless transposed tiles or forced CTA
+// pairs are asked for; 128 otherwise.
+// Experts average at most 32 routed rows (decode-shaped: every row tile is mostly padding).
+bool decode_shaped(moe_plan_t p) { return (long long)p->T * p->k <= (long long)kGemmBMSmall * p->E; }
+
+int plan_bm(moe_plan_t p) {
+  if (p->tile_rows != 0) return p->tile_rows;
+  if (p->swap_rows != 0 || p->pair_mode == 2) return kGemmBM;
+  return decode_shaped(p) && p->T <= 32 ? kGemmBMSmall : kGemmBM;
+}
+
+// Zero padding of the A rows a 128-row tile leaves empty: automatic for decode-shaped layers with
+// more than 32 tokens, where the MMAs of mostly-empty tiles and the weight stream together hold
+// the part at its power limit (zero operands lower the power drawn and so raise the clock);
+// measured slower where tiles are mostly full (the extra copies cost more than they save).
+bool plan_zero_pad(moe_plan_t p) {
+  if (p->zero_pad == 1) return true;
+  if (p->zero_pad == 2) return false;
+  return plan_bm(p) == kGemmBM && decode_shaped(p);
+}
+
+// CTA-pair GEMMs (M = 256 per pair) when experts average at least 256 rows, or when forced
+// (128-row tiles only).
 bool use_pairs(moe_plan_t p) {
-  if (p->pair_mode == 0 || gemm_pair_max_clusters() < 1) return false;
+  if (p->pair_mode == 0 || gemm_pair_max_clusters() < 1 || plan_bm(p) != kGemmBM) return false;
   return p->pair_mode == 2 || (long long)p->T * p->k >= 256ll * p->E;
 }
 
@@ -148,6 +178,7 @@ int linear2_bn(moe_plan_t p) {
 
 GemmArgs gemm_args(moe_plan_t p, int mode) {
   GemmArgs a{};
+  a.bm = plan_bm(p);
   a.n_experts = p->n;
   a.rows_total = (int)p->rows;
   a.counts = region<int32_t>(p, MOE_REGION_COUNTS);
@@ -159,6 +190,7 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.timeout_ns = p->timeout_ns;
   a.swap_rows = p->swap_rows;
+  a.zeros = plan_zero_pad(p) ? at<uint8_t>(p, p->off_zeros) : nullptr;
   if (mode == 1) {
     a.K = p->H;
     a.N = p->I;
@@ -185,7 +217,8 @@ GemmArgs gemm_args(moe_plan_t p, int mode) {
 }
 
 int gemm_grid(moe_plan_t p, int n_tiles_n) {
-  const long long mt_bound = (p->rows + kGemmBM - 1) / kGemmBM + p->n;
+  const int bm = plan_bm(p);
+  const long long mt_bound = (p->rows + bm - 1) / bm + p->n;
   long long tiles = mt_bound * n_tiles_n;
   int sms = p->num_sms;
   if (p->max_sms > 0 && p->max_sms < sms) sms = p->max_sms;
@@ -228,6 +261,20 @@ int run_router(moe_plan_t p, const uint16_t* x, const float* W_router, cudaStrea
   return cuda_rc(launch_router_tc(p->tmX, p->tmWhi, p->tmWlo, ra, s));
 }
 
+// K parts of the fused forward's split-K router: a warp per (expert, part) computes all T tokens,
+// so with few tokens every warp of the grid streams a slice of W_router.  0 = not used (more
+// than kSplitKMaxT tokens, or E beyond what the top-k adds up in parts).  Enough parts for
+// about one item per warp of a 148-SM grid, each at most kSplitKMaxChunks chunks of 256 channels.
+int splitk_parts(int T, int H, int E) {
+  if (T > kSplitKMaxT || E > kTopkMaxSplitE || E % 4 != 0) return 0;
+  const int C = (H + 255) / 256;
+  int s = (148 * (kGemmThreads / 32) + E - 1) / E;
+  const int s_min = (C + kSplitKMaxChunks - 1) / kSplitKMaxChunks;
+  if (s < s_min) s = s_min;
+  if (s > C) s = C;
+  return s;
+}
+
 // partial logit arrays the router leaves for top-k
 int logit_parts(moe_plan_t p) { return use_tc_router(p) ? p->router_splits : 1; }
 
@@ -251,7 +298,7 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
                                         region<int32_t>(p, MOE_REGION_COUNTS), region<int32_t>(p, MOE_REGION_OFFSETS),
                                         at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
                                         at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
-                                        p->shared, s)) != cudaSuccess)
+                                        p->shared, plan_bm(p), s)) != cudaSuccess)
       return cuda_rc(e);
     mark(p, 1 + MOE_PHASE_TOPK, s);
   } else {
@@ -264,7 +311,7 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
                                   region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_gbase),
                                   at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
                                   at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
-                                  p->shared, s)) != cudaSuccess)
+                                  p->shared, plan_bm(p), s)) != cudaSuccess)
       return cuda_rc(e);
   }
   mark(p, 1 + MOE_PHASE_SCAN, s);
@@ -272,7 +319,7 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
                            region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile),
                            region<int32_t>(p, MOE_REGION_SLOT_POS), region<int32_t>(p, MOE_REGION_PERM),
                            region<uint8_t>(p, MOE_REGION_XQ), region<uint8_t>(p, MOE_REGION_XSF), p->T, p->H,
-                           p->E, p->k, p->shared, s);
+                           p->E, p->k, p->shared, plan_bm(p), s);
   mark(p, 1 + MOE_PHASE_SCATTER_QUANT, s);
   return cuda_rc(e);
 }
@@ -323,9 +370,11 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
   }
   FusedArgs a{};
   a.T = p->T; a.H = p->H; a.E = p->E; a.k = p->k; a.shared = p->shared;
+  a.bm = plan_bm(p);
   a.router_kind = tc ? kRouterTensor
-                     : (long long)p->T * p->E <= 4096 ? kRouterSplitBlock : p->E <= 32 ? kRouterWarp8 : kRouterWarp2;
-  a.router_parts = tc ? p->router_splits : 1;
+                  : p->splitk_parts > 0 ? kRouterSplitK
+                  : (long long)p->T * p->E <= 4096 ? kRouterSplitBlock : p->E <= 32 ? kRouterWarp8 : kRouterWarp2;
+  a.router_parts = tc ? p->router_splits : p->splitk_parts > 0 ? p->splitk_parts : 1;
   a.x = x;
   a.W_router = W_router;
   a.bias = bias;
@@ -349,16 +398,21 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
   a.out = static_cast<uint16_t*>(out);
   a.status = region<uint32_t>(p, MOE_REGION_STATUS);
   a.gridbar = at<uint32_t>(p, p->off_gridbar);
+  a.counters = at<uint32_t>(p, p->off_counters);
+  a.stamps = (p->phase_events && p->events_ready) ? region<unsigned long long>(p, MOE_REGION_STAMPS) : nullptr;
   a.timeout_ns = p->timeout_ns;
   a.ra = RouterArgs{p->T, p->H, p->E, a.router_parts, a.logits, a.status, p->timeout_ns};
   a.g1 = gemm_args(p, 1);
   a.g2 = gemm_args(p, 2);
   int ctas = fused_max_ctas();
   if (p->max_sms > 0 && p->max_sms < ctas) ctas = p->max_sms;
+  if (ctas > kStampMaxCtas) ctas = kStampMaxCtas;
+  p->fused_ctas_last = a.stamps != nullptr ? ctas : 0;
   // a launch that ran out of time may have left arrivals behind
   if (cudaMemsetAsync(a.gridbar, 0, 8, s) != cudaSuccess) return MOE_ERR_CUDA;
   const CUtensorMap& b2 = a.g2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
-  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, b2, p->tmX, p->tmWhi, p->tmWlo, a, ctas, s) != cudaSuccess)
+  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, b2, p->tmX, p->tmWhi, p->tmWlo, a, ctas,
+                           plan_bm(p) == kGemmBMSmall, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // one kernel: its whole time is reported under the first phase
   for (int i = 1; i <= MOE_PHASE_COUNT_; ++i) mark(p, i, s);
@@ -394,10 +448,9 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
       return MOE_ERR_CUDA;
     mark(p, 1 + MOE_PHASE_LINEAR2, s);
   } else {
-    // an expert never gets more rows than there are tokens
-    const bool few_rows = p->T <= 16;
+    const bool small_tiles = plan_bm(p) == kGemmBMSmall;
     const CUtensorMap& b2 = a2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
-    if (few_rows && p->chain) {
+    if (small_tiles && p->T <= 16 && p->chain) {
       // one cooperative launch: linear2 tiles start as soon as their expert's linear1 tiles are
       // stored (per-expert counters, zeroed here); reported under linear1
       uint32_t* dep = at<uint32_t>(p, p->off_dep);
@@ -410,10 +463,10 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
       mark(p, 1 + MOE_PHASE_LINEAR1, s);
       mark(p, 1 + MOE_PHASE_LINEAR2, s);
     } else {
-      if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, few_rows) != cudaSuccess)
+      if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, small_tiles) != cudaSuccess)
         return MOE_ERR_CUDA;
       mark(p, 1 + MOE_PHASE_LINEAR1, s);
-      if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, few_rows) != cudaSuccess)
+      if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, small_tiles) != cudaSuccess)
         return MOE_ERR_CUDA;
       mark(p, 1 + MOE_PHASE_LINEAR2, s);
     }
@@ -510,15 +563,18 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   reg(MOE_REGION_PERM, (size_t)R * 4);
   reg(MOE_REGION_SLOT_POS, Tk * 4);
   reg(MOE_REGION_XQ, (size_t)rows * H);
-  p->mt_cap = (rows + kGemmBM - 1) / kGemmBM + p->n;
+  p->mt_cap = (rows + kGemmBMSmall - 1) / kGemmBMSmall + p->n;
   reg(MOE_REGION_XSF, (size_t)p->mt_cap * (H / 128) * 512);
   reg(MOE_REGION_HQ, (size_t)rows * I);
   reg(MOE_REGION_HSF, (size_t)p->mt_cap * (I / 128) * 512);
   reg(MOE_REGION_Y, (size_t)rows * H * 2);
+  reg(MOE_REGION_STAMPS, (size_t)kStampCount * kStampMaxCtas * 8);
   // the tensor-core router's split count depends on the shape only, so results do not
   // depend on the device or on options
   p->router_splits = (E >= 16 && E % 16 == 0) ? router_tc_splits(T, H, E) : 1;
-  p->off_logits = add((size_t)p->router_splits * T * E * 4);
+  p->splitk_parts = splitk_parts(T, H, E);
+  const int parts = p->router_splits > p->splitk_parts ? p->router_splits : p->splitk_parts;
+  p->off_logits = add((size_t)parts * T * E * 4);
   p->off_rank = add(Tk * 4);
   p->off_gcounts = add((size_t)p->G * E * 4);
   p->off_gbase = add((size_t)p->G * E * 4);
@@ -528,6 +584,8 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out) {
   p->off_ptinfo = add((size_t)p->mt_cap * 16);
   p->off_dep = add((size_t)p->n * 4);
   p->off_gridbar = add(8);
+  p->off_zeros = add(kGemmZeroBytes);
+  p->off_counters = add((size_t)(2 + p->n) * 4);
   p->off_w1sf = add((size_t)p->n * (I / 128) * (H / 128) * 1024);
   // linear2 weight scale units for the narrower of the two tile heights (more tiles)
   p->off_w2sf = add((size_t)p->n * ((H + kGemmBN2Double - 1) / kGemmBN2Double) * (I / 128) * 1024);
@@ -590,14 +648,47 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       return MOE_OK;
     case MOE_OPT_PAIR_TILES:
       if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+      if (value == 2 && p->tile_rows == kGemmBMSmall) return MOE_ERR_INVALID_ARG;
       p->pair_mode = (int)value;
       return MOE_OK;
     case MOE_OPT_SWAP_ROWS:
       if (value != 0 && value != 32 && value != 64) return MOE_ERR_INVALID_ARG;
+      if (value != 0 && p->tile_rows == kGemmBMSmall) return MOE_ERR_INVALID_ARG;
       p->swap_rows = (int)value;
+      return MOE_OK;
+    case MOE_OPT_ZERO_PAD:
+      if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+      p->zero_pad = (int)value;
+      return MOE_OK;
+    case MOE_OPT_TILE_ROWS:
+      if (value != 0 && value != kGemmBMSmall && value != kGemmBM) return MOE_ERR_INVALID_ARG;
+      if (value == kGemmBMSmall && (p->swap_rows != 0 || p->pair_mode == 2)) return MOE_ERR_INVALID_ARG;
+      p->tile_rows = (int)value;
       return MOE_OK;
     default:
       return MOE_ERR_INVALID_ARG;
+  }
+}
+
+int moe_plan_get_option(moe_plan_t p, int key, long long* value) {
+  if (!p || !value) return MOE_ERR_INVALID_ARG;
+  switch (key) {
+    case MOE_OPT_GRAPH: *value = p->use_graph; return MOE_OK;
+    case MOE_OPT_MAX_SMS: *value = p->max_sms; return MOE_OK;
+    case MOE_OPT_TIMEOUT_NS: *value = (long long)p->timeout_ns; return MOE_OK;
+    case MOE_OPT_INJECT_FAULT: *value = p->inject_fault; return MOE_OK;
+    case MOE_OPT_STATIC_WEIGHTS: *value = p->static_weights; return MOE_OK;
+    case MOE_OPT_ROUTER_TC: *value = p->router_tc; return MOE_OK;
+    case MOE_OPT_PHASE_EVENTS: *value = p->phase_events; return MOE_OK;
+    case MOE_OPT_FUSED: *value = p->fused; return MOE_OK;
+    case MOE_OPT_CHAIN: *value = p->chain; return MOE_OK;
+    case MOE_OPT_L2_TILE_ROWS: *value = linear2_bn(p); return MOE_OK;
+    case MOE_OPT_DEPENDENT_LAUNCH: *value = p->dep_launch; return MOE_OK;
+    case MOE_OPT_PAIR_TILES: *value = p->pair_mode; return MOE_OK;
+    case MOE_OPT_SWAP_ROWS: *value = p->swap_rows; return MOE_OK;
+    case MOE_OPT_TILE_ROWS: *value = plan_bm(p); return MOE_OK;
+    case MOE_OPT_ZERO_PAD: *value = plan_zero_pad(p) ? 1 : 2; return MOE_OK;
+    default: return MOE_ERR_INVALID_ARG;
   }
 }
 
@@ -664,6 +755,7 @@ int moe_set_workspace(moe_plan_t p, void* ws, size_t bytes) {
   }
   if (cudaMemset(region<uint32_t>(p, MOE_REGION_STATUS), 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemset(at<uint32_t>(p, p->off_gridbar), 0, 8) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(at<uint8_t>(p, p->off_zeros), 0, kGemmZeroBytes) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -713,6 +805,39 @@ int moe_phase_times(moe_plan_t p, float* ms, int capacity) {
   if (cudaEventSynchronize(p->ev[MOE_PHASE_COUNT_]) != cudaSuccess) return MOE_ERR_CUDA;
   for (int i = 0; i < MOE_PHASE_COUNT_; ++i)
     if (cudaEventElapsedTime(&ms[i], p->ev[i], p->ev[i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+  if (p->fused && p->fused_ctas_last > 0) {
+    // one kernel: split its event time by the phase stamps (the latest CTA at each point; the
+    // router phase runs from the earliest start)
+    const int n = p->fused_ctas_last;
+    std::vector<unsigned long long> h((size_t)kStampCount * n);
+    for (int id = 0; id < kStampCount; ++id)
+      if (cudaMemcpy(h.data() + (size_t)id * n, region<unsigned long long>(p, MOE_REGION_STAMPS) + (size_t)id * kStampMaxCtas,
+                     n * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    unsigned long long t[kStampCount];
+    for (int id = 0; id < kStampCount; ++id) {
+      unsigned long long v = id == kStampStart ? ~0ull : 0ull;
+      for (int c = 0; c < n; ++c) {
+        const unsigned long long s = h[(size_t)id * n + c];
+        if (id == kStampCombine && s == 0) continue;            // CTAs without combine items skip it
+        v = id == kStampStart ? (s < v ? s : v) : (s > v ? s : v);
+      }
+      t[id] = v;
+    }
+    if (t[kStampCombine] == 0) t[kStampCombine] = t[kStampLinear1];
+    const float total = ms[MOE_PHASE_ROUTER];
+    auto d = [&](int a, int b) { return t[b] > t[a] ? (float)((t[b] - t[a]) * 1e-6) : 0.f; };
+    for (int i = 0; i < MOE_PHASE_COUNT_; ++i) ms[i] = 0.f;
+    ms[MOE_PHASE_TOPK] = d(kStampRouted, kStampScanned);
+    ms[MOE_PHASE_SCATTER_QUANT] = d(kStampScanned, kStampRowsReady);
+    ms[MOE_PHASE_LINEAR1] = d(kStampRowsReady, kStampLinear1);
+    ms[MOE_PHASE_LINEAR2] = d(kStampLinear1, kStampCombine);
+    ms[MOE_PHASE_COMBINE] = d(kStampCombine, kStampEnd);
+    // the router phase carries the launch and the rest of the event time
+    float rest = total;
+    for (int i = 1; i < MOE_PHASE_COUNT_; ++i) rest -= ms[i];
+    ms[MOE_PHASE_ROUTER] = rest > 0.f ? rest : d(kStampStart, kStampRouted);
+  }
   return MOE_PHASE_COUNT_;
 }
 
@@ -754,12 +879,12 @@ int moe_debug_dispatch(moe_plan_t p, const int32_t* topk_ids, int32_t* counts, i
   if ((e = launch_dispatch_scan(at<int32_t>(p, p->off_gcounts), counts, offsets, at<int32_t>(p, p->off_gbase),
                                 at<int32_t>(p, p->off_mtile), at<int32_t>(p, p->off_ptile),
                                 at<int4>(p, p->off_tinfo), at<int4>(p, p->off_ptinfo), p->T, p->E, p->k,
-                                p->shared, s)) != cudaSuccess)
+                                p->shared, plan_bm(p), s)) != cudaSuccess)
     return MOE_ERR_CUDA;
   // positions = offsets (written just above into the caller's buffer) + group base + rank
   e = launch_scatter_quant(nullptr, topk_ids, at<int32_t>(p, p->off_rank), at<int32_t>(p, p->off_gbase), offsets,
                            at<int32_t>(p, p->off_mtile), slot_pos, perm, nullptr, nullptr, p->T, p->H, p->E, p->k,
-                           p->shared, s);
+                           p->shared, plan_bm(p), s);
   return cuda_rc(e);
 }
 

@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     int mode, const float* __restrict__ logits, int n_parts, const float* __restrict__ bias, int32_t* topk_ids,
     float* gates, int32_t* __restrict__ local_rank, int32_t* __restrict__ group_counts, uint32_t* status,
     int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start,
-    int4* tile_info, int4* ptile_info, int T, int E, int k, int shared) {
+    int4* tile_info, int4* ptile_info, int T, int E, int k, int shared, int bm) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ TopkSmem sm;
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     group_base[e] = 0;
   }
   __syncthreads();
-  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum,
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, bm, wsum,
                           cnt_s);
 }
 
@@ -227,11 +227,11 @@ __global__ void __launch_bounds__(256) column_scan_kernel(const int32_t* __restr
 
 __global__ void __launch_bounds__(1024) expert_scan_kernel(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
                                                            int32_t* ptile_start, int4* tile_info, int4* ptile_info,
-                                                           int T, int E, int shared) {
+                                                           int T, int E, int shared, int bm) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ int32_t wsum[3][32];
-  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, wsum);
+  expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, bm, wsum);
 }
 
 // --------------------------------------------------------------------------- scatter + quant
@@ -245,11 +245,12 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
                                                             const int32_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ mtile_start,
                                                             int32_t* slot_pos, int32_t* perm, uint8_t* xq,
-                                                            uint8_t* xsf, int T, int H, int E, int k, int shared) {
+                                                            uint8_t* xsf, int T, int H, int E, int k, int shared,
+                                                            int bm) {
   griddep_wait();
   griddep_launch_dependents();
   scatter_items<SL>((long)blockIdx.x * 8 + threadIdx.x / 32, x, topk_ids, local_rank, group_base, offsets,
-                    mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared);
+                    mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
 }
 
 // Token-order quantisation for the debug entry point: xq[t][H], xs[t][H/128] = 2^p.
@@ -368,37 +369,37 @@ cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_part
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
                                       int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                      int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
+                                      int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s) {
   if (T > 32 || n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
   return launch_kernel(topk_scan_one_group_kernel, 1, 1024, 0, s, mode, logits, n_parts, bias, topk_ids, gates,
                        local_rank, group_counts, status, group_base, counts, offsets, mtile_start, ptile_start,
-                       tile_info, ptile_info, T, E, k, shared);
+                       tile_info, ptile_info, T, E, k, shared, bm);
 }
 
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                 int4* ptile_info, int T, int E, int k, int shared, cudaStream_t s) {
+                                 int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s) {
   const int G = (T + 31) / 32;
   cudaError_t e = launch_kernel(column_scan_kernel, (E + 7) / 8, 256, 0, s, group_counts, group_base, counts, G, E);
   if (e != cudaSuccess) return e;
   return launch_kernel(expert_scan_kernel, 1, 1024, 0, s, counts, offsets, mtile_start, ptile_start, tile_info,
-                       ptile_info, T, E, shared);
+                       ptile_info, T, E, shared, bm);
 }
 
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
-                                 int k, int shared, cudaStream_t s) {
+                                 int k, int shared, int bm, cudaStream_t s) {
   const long slices = (long)T * (x == nullptr ? 1 : (H + 255) / 256);
   // Mixtral T = 4096 (65,536 slices): 4 per warp, the scatter 26 -> 19 us; DSV3 T = 512
   // (14,336) and T = 1 (28) keep one per warp, four would leave too few warps in flight
   if (x != nullptr && slices >= 32768) {
     const long items = (long)T * (((H + 255) / 256 + 3) / 4);
     return launch_kernel(scatter_quant_kernel<4>, (unsigned)((items + 7) / 8), 256, 0, s, x, topk_ids, local_rank,
-                         group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared);
+                         group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
   }
   return launch_kernel(scatter_quant_kernel<1>, (unsigned)((slices + 7) / 8), 256, 0, s, x, topk_ids, local_rank,
-                       group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared);
+                       group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
 }
 
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s) {

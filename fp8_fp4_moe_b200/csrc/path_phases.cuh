@@ -118,6 +118,71 @@ __device__ __forceinline__ void router_split_block(const uint16_t* __restrict__ 
   }
   __syncthreads();                     // part[] is free again
 }
+// Few tokens inside a persistent kernel: a warp per (expert e, K part s) computes the partial
+// logits of ALL T <= TMAX tokens over its part of the channels, so every warp streams a slice of
+// W_router once (the whole grid reads it at HBM speed) instead of one block per (expert, token).
+// Part s covers the 256-channel chunks [s*C/S, (s+1)*C/S) (C = ceil(H/256)); lane l owns channels
+// [c + 8l, c + 8l + 8) of each chunk, all W loads of the part are issued before the FMAs.  Writes
+// logits[s][t][e]; the top-k adds the S parts in part order (deterministic).
+// Called by whole warps: items first, first + stride, ... over E * S items.
+template <int TMAX, int CMAX>
+__device__ __forceinline__ void router_splitk_items(const uint16_t* __restrict__ x, const float* __restrict__ W,
+                                                   float* __restrict__ logits, int T, int H, int E, int S,
+                                                   long first, long stride) {
+  const int lane = threadIdx.x % 32;
+  const int C = (H + 255) / 256;
+  for (long item = first; item < (long)E * S; item += stride) {
+    const int e = (int)(item / S), s = (int)(item % S);
+    const int c_lo = s * C / S, c_hi = (s + 1) * C / S;       // at most CMAX chunks (host-chosen S)
+    float4 w[CMAX][2];
+#pragma unroll
+    for (int i = 0; i < CMAX; ++i) {
+      const int c0 = (c_lo + i) * 256 + lane * 8;
+      if (c_lo + i < c_hi && c0 < H) {
+        const float4* wr = reinterpret_cast<const float4*>(W + (long)e * H + c0);
+        w[i][0] = __ldg(wr);
+        w[i][1] = __ldg(wr + 1);
+      } else {
+        w[i][0] = w[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float acc[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) acc[t] = 0.f;
+#pragma unroll
+    for (int i = 0; i < CMAX; ++i) {
+      const int c0 = (c_lo + i) * 256 + lane * 8;
+      if (c_lo + i < c_hi && c0 < H) {                          // lane-uniform per chunk except the H tail
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+          if (t < T) {
+            const uint4 r = __ldg(reinterpret_cast<const uint4*>(x + (long)t * H + c0));
+            float a = acc[t];
+            a = fmaf(__uint_as_float(r.x << 16), w[i][0].x, a);
+            a = fmaf(__uint_as_float(r.x & 0xFFFF0000u), w[i][0].y, a);
+            a = fmaf(__uint_as_float(r.y << 16), w[i][0].z, a);
+            a = fmaf(__uint_as_float(r.y & 0xFFFF0000u), w[i][0].w, a);
+            a = fmaf(__uint_as_float(r.z << 16), w[i][1].x, a);
+            a = fmaf(__uint_as_float(r.z & 0xFFFF0000u), w[i][1].y, a);
+            a = fmaf(__uint_as_float(r.w << 16), w[i][1].z, a);
+            a = fmaf(__uint_as_float(r.w & 0xFFFF0000u), w[i][1].w, a);
+            acc[t] = a;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+      if (t < T) {
+        float v = acc[t];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) logits[((long)s * T + t) * E + e] = v;
+      }
+    }
+  }
+}
+
 // --------------------------------------------------------------------------- top-k + rank
 // One block of NT threads per group of 32 tokens; warp w selects for tokens 32*g + w,
 // 32*g + w + NT/32, ...  Then warp 0 ranks the group's copies: lane = token, and each
@@ -286,8 +351,8 @@ __device__ __forceinline__ void topk_rank_group(int g, int mode, const float* __
 // Two steps.  Per routed expert e (one warp): counts[e] = sum over groups and the relative
 // group base group_base[g][e] = rows of e in groups < g (warp scan over the groups, 32 at a
 // time).  Then one block: exclusive scans over the n = E + shared experts (shared expert
-// last, T rows) of counts -> offsets, of ceil(count/128) -> mtile_start and of
-// ceil(ceil(count/128)/2) -> ptile_start (row-tile pairs of the CTA-pair GEMM).
+// last, T rows) of counts -> offsets, of ceil(count/bm) -> mtile_start (bm-row tiles of the
+// GEMMs) and of ceil(ceil(count/128)/2) -> ptile_start (128-row tile pairs of the CTA-pair GEMM).
 __device__ __forceinline__ void column_scan_warp(int e, const int32_t* __restrict__ group_counts,
                                                  int32_t* __restrict__ group_base, int32_t* __restrict__ counts,
                                                  int G, int E) {
@@ -315,7 +380,7 @@ __device__ __forceinline__ void column_scan_warp(int e, const int32_t* __restric
 template <int NT>
 __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offsets, int32_t* mtile_start,
                                                   int32_t* ptile_start, int4* tile_info, int4* ptile_info, int T,
-                                                  int E, int shared, int32_t (*wsum)[32],
+                                                  int E, int shared, int bm, int32_t (*wsum)[32],
                                                   const int32_t* cnt_src = nullptr) {
   if (cnt_src == nullptr) cnt_src = counts;
   constexpr int PER = (1024 + NT - 1) / NT;   // consecutive experts per thread
@@ -328,10 +393,9 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
   for (int j = 0; j < PER; ++j) {
     const int e = threadIdx.x * PER + j;
     c[j] = e < E ? cnt_src[e] : (e == E && shared ? T : 0);
-    const int mt = (c[j] + kGemmBM - 1) / kGemmBM;
     tc += c[j];
-    tm += mt;
-    tp += (mt + 1) / 2;
+    tm += (c[j] + bm - 1) / bm;
+    tp += ((c[j] + kGemmBM - 1) / kGemmBM + 1) / 2;
   }
   int ic = tc, im = tm, ip = tp;
 #pragma unroll
@@ -356,26 +420,27 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
   }
   __syncthreads();
   int bc = (warp > 0 ? wsum[0][warp - 1] : 0) + ic - tc;
-  int bm = (warp > 0 ? wsum[1][warp - 1] : 0) + im - tm;
+  int bt = (warp > 0 ? wsum[1][warp - 1] : 0) + im - tm;
   int bp = (warp > 0 ? wsum[2][warp - 1] : 0) + ip - tp;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int e = threadIdx.x * PER + j;
-    const int mt = (c[j] + kGemmBM - 1) / kGemmBM;
+    const int mt = (c[j] + bm - 1) / bm;
+    const int pt = ((c[j] + kGemmBM - 1) / kGemmBM + 1) / 2;
     if (e < n) {
       if (e >= E) counts[e] = c[j];
       offsets[e] = bc;
-      mtile_start[e] = bm;
+      mtile_start[e] = bt;
       ptile_start[e] = bp;
-      for (int g = 0; g < mt; ++g) tile_info[bm + g] = make_int4(e, bm, c[j], bc);
-      for (int g = 0; g < (mt + 1) / 2; ++g) ptile_info[bp + g] = make_int4(e, bp, c[j], bc);
+      for (int g = 0; g < mt; ++g) tile_info[bt + g] = make_int4(e, bt, c[j], bc);
+      for (int g = 0; g < pt; ++g) ptile_info[bp + g] = make_int4(e, bp, c[j], bc);
     }
     bc += c[j];
-    bm += mt;
-    bp += (mt + 1) / 2;
+    bt += mt;
+    bp += pt;
     if (e == n - 1) {
       offsets[n] = bc;
-      mtile_start[n] = bm;
+      mtile_start[n] = bt;
       ptile_start[n] = bp;
     }
   }
@@ -384,7 +449,8 @@ __device__ __forceinline__ void expert_scan_block(int32_t* counts, int32_t* offs
 
 // --------------------------------------------------------------------------- scatter + quant
 // One warp per (token, 256-channel slice).  Positions: slot_pos[t][j] = offsets[e] +
-// group_base[g][e] + rank (group_base relative to the expert's first row);
+// group_base[g][e] + rank (group_base relative to the expert's first row); a row's scale
+// word goes to the atom of its bm-row tile;
 // the shared expert's row for token t is R + t.  Quantisation: per 128-channel
 // block, smallest 2^p with amax <= 448 * 2^p (p >= -126; p = 0 if all zero),
 // codes = E4M3 round-to-nearest-even of x * 2^-p (exact scaling), written once
@@ -400,7 +466,7 @@ __device__ __forceinline__ void scatter_items(long item, const uint16_t* __restr
                                               const int32_t* __restrict__ offsets,
                                               const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
                                               int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E, int k,
-                                              int shared) {
+                                              int shared, int bm) {
   const int lane = threadIdx.x % 32;
   const int n_slices = (x == nullptr) ? 1 : (H + 255) / 256;
   const int n_grp = (n_slices + SL - 1) / SL;
@@ -436,8 +502,8 @@ __device__ __forceinline__ void scatter_items(long item, const uint16_t* __restr
   long sf_off = 0;
   if (e >= 0) {
     const int rank = row - offsets[e];
-    const int r = rank % 128;
-    sf_off = ((long)(mtile_start[e] + rank / 128) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
+    const int r = rank % bm;
+    sf_off = ((long)(mtile_start[e] + rank / bm) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
   }
   const int ndst = k + shared;
 #pragma unroll
@@ -482,9 +548,9 @@ __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restri
                                              const int32_t* __restrict__ offsets,
                                              const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
                                              int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E, int k,
-                                             int shared) {
+                                             int shared, int bm) {
   scatter_items<1>(item, x, topk_ids, local_rank, group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H,
-                   E, k, shared);
+                   E, k, shared, bm);
 }
 
 // --------------------------------------------------------------------------- combine

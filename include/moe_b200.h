@@ -124,7 +124,7 @@ enum moe_option {
                                   narrower tile leaves TMEM room for two accumulators, so
                                   one tile's epilogue overlaps the next tile's MMAs;
                                   256 = always.  CTA-pair GEMMs always use 256.            */
-  MOE_OPT_CHAIN = 13           /* 1 = with at most 16 tokens, linear1 and linear2 run as
+  MOE_OPT_CHAIN = 13,          /* 1 = with at most 16 tokens, linear1 and linear2 run as
                                   one cooperative launch: each linear2 tile's producer
                                   streams its weights at once and waits (bounded) only
                                   for the linear1 tiles of its own expert.  moe_phase_times
@@ -132,6 +132,26 @@ enum moe_option {
                                   CUDA graph (the cooperative launch cannot start early
                                   as the dependent launches do).  0 (default) = two
                                   launches.                                                */
+  MOE_OPT_TILE_ROWS = 14,      /* rows of the grouped GEMMs' row tiles: 0 (default) = 32
+                                  when T <= 32 and the routed experts average at most 32
+                                  rows (T*k <= 32*E) and neither transposed tiles nor
+                                  forced CTA pairs are asked for, else 128; 32 or 128 =
+                                  always.  32-row tiles run on a shared-memory layout with
+                                  32-row A regions and 6 pipeline stages (more weight bytes
+                                  in flight per SM); the MMA still spans 128 rows.  32 is
+                                  incompatible with MOE_OPT_SWAP_ROWS != 0 and
+                                  MOE_OPT_PAIR_TILES = 2 (MOE_ERR_INVALID_ARG).  The
+                                  activation scale atoms (and moe_workspace_region's "xsf"
+                                  and "hsf" regions) are laid out per row tile.            */
+  MOE_OPT_ZERO_PAD = 15        /* on 128-row tiles, the A rows a tile does not fill are
+                                  zeroed (a bulk copy from a zero buffer in the workspace)
+                                  before the MMA, which spans all 128 rows, reads them:
+                                  zero operands draw less power than stale rows of earlier
+                                  tiles, which raises the clock where the power limit holds
+                                  it down.  The results do not change.  0 (default) = when
+                                  the routed experts average at most 32 rows (T*k <= 32*E)
+                                  and the tiles have 128 rows; 1 = always (128-row tiles);
+                                  2 = never.  moe_plan_get_option reports 1 (on) or 2.     */
 };
 
 /* Phases of moe_forward, in launch order (moe_phase_times). */
@@ -155,6 +175,9 @@ enum moe_region {
   MOE_REGION_HQ,           /* uint8  [R + shared*T, I]   E4M3 SwiGLU output               */
   MOE_REGION_HSF,          /* scale atoms of HQ: [row tile][I/128] x 512 B               */
   MOE_REGION_Y,            /* bf16   [R + shared*T, H]   expert output rows               */
+  MOE_REGION_STAMPS,       /* uint64 [stamp point][1024]: global-timer ns at which each CTA of
+                              the last MOE_OPT_FUSED forward run with MOE_OPT_PHASE_EVENTS = 1
+                              passed each point of the kernel (debug; see moe_phase_times)  */
   MOE_REGION_COUNT_
 };
 
@@ -172,6 +195,11 @@ int moe_plan(int T, int H, int I, int E, int k, int shared, moe_plan_t* out);
 
 /* Set a moe_option.  Returns MOE_ERR_INVALID_ARG for an unknown key/value. */
 int moe_plan_set_option(moe_plan_t plan, int key, long long value);
+/* The value an option has for this plan, resolved: MOE_OPT_TILE_ROWS and
+ * MOE_OPT_L2_TILE_ROWS report the row-tile heights the next forward uses (32 or
+ * 128; 224 or 256), every other key the value last set (or its default).
+ * MOE_ERR_INVALID_ARG for an unknown key or a NULL pointer.  No device work. */
+int moe_plan_get_option(moe_plan_t plan, int key, long long* value);
 
 /* Bytes of device workspace the plan needs (0 for a NULL plan). */
 size_t moe_workspace_bytes(moe_plan_t plan);

@@ -183,23 +183,24 @@ def slack_needed_fraction(gpu_out_bits, ref_y, slack) -> float:
     return float(np.mean(base > MAX_ABS_RMS_TOL * rms))
 
 
-def untile_scales(atoms, counts, offsets) -> np.ndarray:
+def untile_scales(atoms, counts, offsets, bm: int = 128) -> np.ndarray:
     """Per-row UE8M0 codes [rows, K/128] from scale atoms [row tiles, K/128, 512] (uint8).
 
-    Row tile g of expert e = (row tiles of experts before e) + rank // 128; the
-    row's code sits at byte (r % 32) * 16 + (r // 32) * 4 of the atom, r = rank % 128.
+    Row tile g of expert e = (row tiles of experts before e) + rank // bm (bm = the plan's
+    row-tile height, MOE_OPT_TILE_ROWS); the row's code sits at byte (r % 32) * 16 + (r // 32) * 4
+    of the atom, r = rank % bm.
     """
     atoms = np.asarray(atoms, dtype=np.uint8)
     counts = np.asarray(counts, dtype=np.int64)
     offsets = np.asarray(offsets, dtype=np.int64)
-    mt = (counts + 127) // 128
+    mt = (counts + bm - 1) // bm
     mstart = np.concatenate([[0], np.cumsum(mt)])
     rows = int(offsets[-1])
     out = np.zeros((rows, atoms.shape[1]), dtype=np.int64)
     for e in range(len(counts)):
         for rank in range(int(counts[e])):
-            g = mstart[e] + rank // 128
-            r = rank % 128
+            g = mstart[e] + rank // bm
+            r = rank % bm
             word = atoms[g, :, (r % 32) * 16 + (r // 32) * 4:(r % 32) * 16 + (r // 32) * 4 + 4]
             assert np.all(word == word[:, :1]), "code replicated in all four bytes"
             out[offsets[e] + rank] = word[:, 0]

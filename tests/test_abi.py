@@ -177,6 +177,52 @@ def test_options_and_unbound_plan(L):
     L.moe_plan_destroy(None)
 
 
+def test_tile_rows_option_and_get_option(L):
+    import ctypes as C
+
+    def get(h, key):
+        v = C.c_longlong()
+        assert L.moe_plan_get_option(h, key, C.byref(v)) == 0
+        return v.value
+
+    # few tokens on decode-sized experts (T <= 32, T*k <= 32*E): 32-row tiles by default; more
+    # tokens: 128-row tiles, zero-padded while the experts still average <= 32 rows
+    rc, h1 = _plan(L, 16, 7168, 2048, 256, 8, 1)
+    assert rc == 0 and get(h1, binding.MOE_OPT_TILE_ROWS) == 32 and get(h1, binding.MOE_OPT_ZERO_PAD) == 2
+    L.moe_plan_destroy(h1)
+    rc, h2 = _plan(L, 8192, 7168, 2048, 256, 8, 1)
+    assert rc == 0 and get(h2, binding.MOE_OPT_TILE_ROWS) == 128 and get(h2, binding.MOE_OPT_ZERO_PAD) == 2
+    assert L.moe_plan_set_option(h2, binding.MOE_OPT_ZERO_PAD, 1) == 0 and get(h2, binding.MOE_OPT_ZERO_PAD) == 1
+    assert L.moe_plan_set_option(h2, binding.MOE_OPT_ZERO_PAD, 3) == binding.MOE_ERR_INVALID_ARG
+    L.moe_plan_destroy(h2)
+    rc, h = _plan(L, 512, 7168, 2048, 256, 8, 1)
+    assert rc == 0 and get(h, binding.MOE_OPT_TILE_ROWS) == 128 and get(h, binding.MOE_OPT_ZERO_PAD) == 1
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_ZERO_PAD, 2) == 0 and get(h, binding.MOE_OPT_ZERO_PAD) == 2
+    # forced heights; transposed tiles and forced CTA pairs need 128-row tiles
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 128) == 0 and get(h, binding.MOE_OPT_TILE_ROWS) == 128
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 64) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 32) == 0 and get(h, binding.MOE_OPT_TILE_ROWS) == 32
+    assert get(h, binding.MOE_OPT_ZERO_PAD) == 2                     # no padding on 32-row tiles
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 0) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, 64) == 0
+    assert get(h, binding.MOE_OPT_TILE_ROWS) == 128                 # transposed tiles need 128 rows
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 32) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, 0) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_TILE_ROWS, 32) == 0
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_SWAP_ROWS, 32) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_PAIR_TILES, 2) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_PAIR_TILES, 1) == 0
+    # other keys report what was set; the linear2 tile height resolves (H = 7168 = 32 * 224)
+    assert get(h, binding.MOE_OPT_PAIR_TILES) == 1
+    assert get(h, binding.MOE_OPT_DEPENDENT_LAUNCH) == 1
+    assert get(h, binding.MOE_OPT_L2_TILE_ROWS) == 256
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, 224) == 0 and get(h, binding.MOE_OPT_L2_TILE_ROWS) == 224
+    v = C.c_longlong()
+    assert L.moe_plan_get_option(h, 12345, C.byref(v)) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_get_option(None, binding.MOE_OPT_GRAPH, C.byref(v)) == binding.MOE_ERR_INVALID_ARG
+    L.moe_plan_destroy(h)
+
+
 def test_dense_gemm_validation_without_a_device(L):
     assert L.moe_gemm_workspace_bytes(0, 128, 128) == 0
     assert L.moe_gemm_workspace_bytes(4, 100, 128) == 0          # N % 128

@@ -44,8 +44,10 @@ SMALL = {
 }
 
 
-def plan_for(w, swap_rows=None, pair_tiles=None, fused=None):
+def plan_for(w, swap_rows=None, pair_tiles=None, fused=None, tile_rows=None):
     p = binding.Plan(w.T, w.H, w.I, w.E, w.k, w.shared)
+    if tile_rows is not None:
+        p.set_option(binding.MOE_OPT_TILE_ROWS, tile_rows)
     if w.H % 224 == 0:
         # these shapes run linear2 on 224-row weight tiles (double-buffered accumulator) at any
         # T; by default only T <= 16 does
@@ -203,7 +205,8 @@ def test_forward_matches_oracle(cuda_lib, name, swap_rows):
     assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
     # dispatched activation codes: row slot_pos[t, j] holds token t's codes
     xq = p.region("xq").cpu().numpy()
-    xsf = untile_scales(p.region("xsf").cpu().numpy(), ref["counts"], ref["offsets"])
+    xsf = untile_scales(p.region("xsf").cpu().numpy(), ref["counts"], ref["offsets"],
+                        p.get_option(binding.MOE_OPT_TILE_ROWS))
     rows = ref["slot_pos"]
     for j in range(w.k):
         assert np.array_equal(xq[rows[:, j]], ref["xq"])
@@ -214,17 +217,26 @@ def test_forward_matches_oracle(cuda_lib, name, swap_rows):
     assert_output_close(bits(out), ref["y"], name, slack)
 
 
-@pytest.mark.parametrize("name,swap_rows", [("ragged_shared", 64), ("ragged_shared", 0), ("dsv3_like", 64),
-                                            ("h896", 0), ("h896", 64)])
-def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows):
+# swap_rows as above; tile_rows 32: row tiles of 32 rows on the 6-stage small-tile layout (the
+# default when experts average <= 32 rows), here also on shapes whose experts span several such
+# tiles (ragged_shared: ~83 rows per expert, the shared expert 333); 128: the 4-stage layout
+@pytest.mark.parametrize("name,swap_rows,tile_rows", [("ragged_shared", 64, None), ("ragged_shared", 0, 128),
+                                                      ("ragged_shared", 0, 32), ("dsv3_like", 64, None),
+                                                      ("dsv3_like", 0, 32), ("dsv3_like", 0, 128),
+                                                      ("t16_shared", 0, 32), ("h896", 0, None), ("h896", 64, None),
+                                                      ("h896", 0, 32)])
+def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows, tile_rows):
     w = SMALL[name]
     case = make_case(w, seed=8)
     d = to_device(case)
-    p = plan_for(w, swap_rows)
+    p = plan_for(w, swap_rows, tile_rows=tile_rows)
+    if tile_rows is not None:
+        assert p.get_option(binding.MOE_OPT_TILE_ROWS) == tile_rows
     p.forward(**d)
     ref = oracle_forward(case, w, keep_rows=True)
     hq = p.region("hq").cpu().numpy()
-    hsf = untile_scales(p.region("hsf").cpu().numpy(), ref["counts"], ref["offsets"])
+    hsf = untile_scales(p.region("hsf").cpu().numpy(), ref["counts"], ref["offsets"],
+                        p.get_option(binding.MOE_OPT_TILE_ROWS))
     y = F.bf16_to_f64(bits(p.region("y")))
     offsets = ref["offsets"]
     differ = ambiguous = 0
@@ -555,3 +567,21 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     assert p.check_status()[0] == 0
     ref, slack = oracle_forward_with_slack(case, w)
     assert_output_close(bits(out), ref["y"], "after timeout", slack)
+
+
+# zero padding of the A rows a 128-row tile does not fill changes no result: the padded rows only
+# reach accumulator rows that are never stored
+@pytest.mark.parametrize("name", ["ragged_shared", "dsv3_like", "h896"])
+def test_zero_padding_changes_no_bit(cuda_lib, name):
+    w = SMALL[name]
+    d = to_device(make_case(w, seed=31, screened=False))
+    outs = []
+    for zero_pad in (2, 1):                       # never, always
+        p = plan_for(w, tile_rows=128)
+        p.set_option(binding.MOE_OPT_ZERO_PAD, zero_pad)
+        assert p.get_option(binding.MOE_OPT_ZERO_PAD) == zero_pad
+        outs.append(p.forward(**d).clone())
+        assert p.check_status()[0] == 0
+        outs.append(p.region("y").clone())
+    assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
+    assert torch.equal(outs[1].view(torch.int16), outs[3].view(torch.int16))
