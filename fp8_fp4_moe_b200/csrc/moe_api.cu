@@ -31,7 +31,7 @@ struct moe_plan_s {
   int swap_rows = 0;
   int pair_mode = 0;                // MOE_OPT_PAIR_TILES
   int fused = 0;                    // MOE_OPT_FUSED
-  int dep_launch = 1;               // MOE_OPT_DEPENDENT_LAUNCH
+  int dep_launch = 2;               // MOE_OPT_DEPENDENT_LAUNCH (2 = automatic)
   int l2_tile_rows = 0;             // MOE_OPT_L2_TILE_ROWS
   int chain = 0;                    // MOE_OPT_CHAIN
   int tile_rows = 0;                // MOE_OPT_TILE_ROWS
@@ -147,6 +147,15 @@ int plan_bm(moe_plan_t p) {
   if (p->tile_rows != 0) return p->tile_rows;
   if (p->swap_rows != 0 || p->pair_mode == 2) return kGemmBM;
   return decode_shaped(p) && p->T <= 32 ? kGemmBMSmall : kGemmBM;
+}
+
+// Programmatic dependent launches: automatic for at most 64 tokens, where each kernel is short
+// and launch latency and the GEMMs' early weight requests matter; with more tokens the GEMM's
+// early-resident CTAs take the registers the scatter's blocks need, and the forward measured
+// 1.5-2 % slower (T = 8192 and 32768).
+bool plan_dep_launch(moe_plan_t p) {
+  if (p->dep_launch != 2) return p->dep_launch != 0;
+  return p->T <= 64;
 }
 
 // Zero padding of the A rows a 128-row tile leaves empty: automatic for decode-shaped layers with
@@ -289,7 +298,7 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
   mark(p, 1 + MOE_PHASE_ROUTER, s);
   // every later kernel of the forward may start before its predecessor ends (it waits for it
   // on the device); not between the per-phase events
-  set_dependent_launch(p->dep_launch != 0 && !p->phase_events);
+  set_dependent_launch(plan_dep_launch(p) && !p->phase_events);
   if (p->T <= 32) {
     // one token group: top-k, ranks and the scans in one block (reported under top-k)
     if ((e = launch_topk_scan_one_group(0, at<float>(p, p->off_logits), logit_parts(p), bias, ids, gates,
@@ -643,7 +652,7 @@ int moe_plan_set_option(moe_plan_t p, int key, long long value) {
       p->l2_tile_rows = (int)value;
       return MOE_OK;
     case MOE_OPT_DEPENDENT_LAUNCH:
-      if (value != 0 && value != 1) return MOE_ERR_INVALID_ARG;
+      if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
       p->dep_launch = (int)value;
       return MOE_OK;
     case MOE_OPT_PAIR_TILES:
@@ -683,7 +692,7 @@ int moe_plan_get_option(moe_plan_t p, int key, long long* value) {
     case MOE_OPT_FUSED: *value = p->fused; return MOE_OK;
     case MOE_OPT_CHAIN: *value = p->chain; return MOE_OK;
     case MOE_OPT_L2_TILE_ROWS: *value = linear2_bn(p); return MOE_OK;
-    case MOE_OPT_DEPENDENT_LAUNCH: *value = p->dep_launch; return MOE_OK;
+    case MOE_OPT_DEPENDENT_LAUNCH: *value = plan_dep_launch(p) ? 1 : 0; return MOE_OK;
     case MOE_OPT_PAIR_TILES: *value = p->pair_mode; return MOE_OK;
     case MOE_OPT_SWAP_ROWS: *value = p->swap_rows; return MOE_OK;
     case MOE_OPT_TILE_ROWS: *value = plan_bm(p); return MOE_OK;

@@ -112,12 +112,15 @@ enum moe_option {
                                   T*E <= 4096, warp per token and expert chunk otherwise).
                                   moe_phase_times reports the whole kernel under the router
                                   phase.  No CUDA graph is recorded.  Default 0.          */
-  MOE_OPT_DEPENDENT_LAUNCH = 11, /* 1 (default): the kernels after the first of a
-                                  moe_forward are launched as programmatic dependents
-                                  (each waits on the device for its predecessor; the
-                                  grouped GEMMs request their first weight tiles before
-                                  that wait).  0 = plain stream order.  Off while
-                                  MOE_OPT_PHASE_EVENTS is 1.                              */
+  MOE_OPT_DEPENDENT_LAUNCH = 11, /* 1: the kernels after the first of a moe_forward are
+                                  launched as programmatic dependents (each waits on the
+                                  device for its predecessor; the grouped GEMMs request
+                                  their first weight tiles before that wait).  0 = plain
+                                  stream order.  2 (default) = automatic: dependent
+                                  launches for T <= 64 (short kernels, where launch latency
+                                  counts), plain order above (there the GEMMs' early CTAs
+                                  slowed the scatter).  Off while MOE_OPT_PHASE_EVENTS is
+                                  1.  moe_plan_get_option reports 1 or 0.                  */
   MOE_OPT_L2_TILE_ROWS = 12,   /* linear2 weight rows per tile: 0 (default) = 224 when
                                   T <= 16 and H % 224 == 0, else 256; 224 = always when
                                   H % 224 == 0 (else MOE_ERR_UNSUPPORTED_SHAPE): the

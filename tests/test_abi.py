@@ -151,9 +151,9 @@ def test_options_and_unbound_plan(L):
     for v in (0, 1):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_FUSED, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_FUSED, 2) == binding.MOE_ERR_INVALID_ARG
-    for v in (0, 1):
+    for v in (0, 1, 2):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, v) == 0
-    assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, 2) == binding.MOE_ERR_INVALID_ARG
+    assert L.moe_plan_set_option(h, binding.MOE_OPT_DEPENDENT_LAUNCH, 3) == binding.MOE_ERR_INVALID_ARG
     for v in (0, 1):
         assert L.moe_plan_set_option(h, binding.MOE_OPT_CHAIN, v) == 0
     assert L.moe_plan_set_option(h, binding.MOE_OPT_CHAIN, 2) == binding.MOE_ERR_INVALID_ARG
@@ -214,7 +214,7 @@ def test_tile_rows_option_and_get_option(L):
     assert L.moe_plan_set_option(h, binding.MOE_OPT_PAIR_TILES, 1) == 0
     # other keys report what was set; the linear2 tile height resolves (H = 7168 = 32 * 224)
     assert get(h, binding.MOE_OPT_PAIR_TILES) == 1
-    assert get(h, binding.MOE_OPT_DEPENDENT_LAUNCH) == 1
+    assert get(h, binding.MOE_OPT_DEPENDENT_LAUNCH) == 0          # automatic: off above 64 tokens
     assert get(h, binding.MOE_OPT_L2_TILE_ROWS) == 256
     assert L.moe_plan_set_option(h, binding.MOE_OPT_L2_TILE_ROWS, 224) == 0 and get(h, binding.MOE_OPT_L2_TILE_ROWS) == 224
     v = C.c_longlong()
