@@ -100,8 +100,9 @@ enum moe_option {
                                   0 = always 128 token rows.  Single-CTA kernel only.     */
   MOE_OPT_PAIR_TILES = 9,      /* grouped GEMMs on CTA pairs (2-CTA clusters, one
                                   M = 256 MMA across the pair, each CTA loading half of
-                                  the weight tile): 0 (default) = never, 1 = when the
-                                  experts average >= 256 rows (T*k >= 256*E), 2 = always */
+                                  the weight tile): 0 = never, 1 (default) = when the
+                                  experts average >= 1024 rows (T*k >= 1024*E), 2 = always.
+                                  Needs 128-row tiles.                                     */
   MOE_OPT_FUSED = 10,          /* 1 = moe_forward runs every step (router, top-k, dispatch
                                   scans, scatter + quantisation, linear1, linear2, combine)
                                   in ONE persistent cooperative kernel, one CTA per SM,

@@ -220,16 +220,19 @@ def test_forward_matches_oracle(cuda_lib, name, swap_rows):
 # swap_rows as above; tile_rows 32: row tiles of 32 rows on the 6-stage small-tile layout (the
 # default when experts average <= 32 rows), here also on shapes whose experts span several such
 # tiles (ragged_shared: ~83 rows per expert, the shared expert 333); 128: the 4-stage layout
-@pytest.mark.parametrize("name,swap_rows,tile_rows", [("ragged_shared", 64, None), ("ragged_shared", 0, 128),
-                                                      ("ragged_shared", 0, 32), ("dsv3_like", 64, None),
-                                                      ("dsv3_like", 0, 32), ("dsv3_like", 0, 128),
-                                                      ("t16_shared", 0, 32), ("h896", 0, None), ("h896", 64, None),
-                                                      ("h896", 0, 32)])
-def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows, tile_rows):
+# pair_tiles 2: every GEMM on CTA pairs (odd row-tile counts leave the second CTA of a pair
+# without rows)
+@pytest.mark.parametrize("name,swap_rows,tile_rows,pair_tiles",
+                         [("ragged_shared", 64, None, None), ("ragged_shared", 0, 128, None),
+                          ("ragged_shared", 0, 32, None), ("dsv3_like", 64, None, None),
+                          ("dsv3_like", 0, 32, None), ("dsv3_like", 0, 128, None), ("t16_shared", 0, 32, None),
+                          ("h896", 0, None, None), ("h896", 64, None, None), ("h896", 0, 32, None),
+                          ("ragged_shared", 0, None, 2), ("wide_router", 0, None, 2), ("h896", 0, None, 2)])
+def test_forward_intermediates_match_oracle(cuda_lib, name, swap_rows, tile_rows, pair_tiles):
     w = SMALL[name]
     case = make_case(w, seed=8)
     d = to_device(case)
-    p = plan_for(w, swap_rows, tile_rows=tile_rows)
+    p = plan_for(w, swap_rows, tile_rows=tile_rows, pair_tiles=pair_tiles)
     if tile_rows is not None:
         assert p.get_option(binding.MOE_OPT_TILE_ROWS) == tile_rows
     p.forward(**d)
