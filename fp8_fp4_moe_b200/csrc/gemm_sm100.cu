@@ -83,6 +83,28 @@ struct TileCoord {
   int rows;                          // rows of the expert in this tile (1..128)
 };
 
+// Order of an expert's (m, n) tiles, `local` in [0, m_count * n_count): bands of kBand row tiles,
+// every column tile of a band before the next band, row tiles fastest inside a band.  While the
+// grid works through one band, its rows (and the expert's weight tiles) stay in L2; with the plain
+// n-major order an expert of many row tiles -- the shared expert of a large batch -- streamed all
+// of its rows from DRAM once per column tile.  An expert of at most kBand row tiles is one band:
+// n-major, m fastest.
+constexpr int kBand = 8;
+__device__ __forceinline__ void banded_mn(int local, int m_count, int n_count, int& m, int& n) {
+  const int full = m_count / kBand;                 // complete bands
+  const int in_full = full * kBand * n_count;
+  if (local < in_full) {
+    const int band = local / (kBand * n_count), rem = local - band * kBand * n_count;
+    n = rem / kBand;
+    m = band * kBand + (rem - n * kBand);
+  } else {
+    const int last = m_count - full * kBand;        // row tiles of the last, shorter band
+    const int rem = local - in_full;
+    n = rem / last;
+    m = full * kBand + (rem - n * last);
+  }
+}
+
 // The tiles of expert e are [mtile_start[e], mtile_start[e + 1]) x n_tiles_n, so tile / n_tiles_n
 // is one of e's row tiles and its table entry names e: one load per tile instead of a search
 // over the experts.  Each role loads the entry of its next tile while it works on the current
@@ -99,8 +121,7 @@ __device__ __forceinline__ TileCoord decode_tile_entry(const GemmArgs& p, int ti
   const int mtiles = (c.count + bm - 1) / bm;
   const int mstart = info.y;
   const int local = tile - mstart * p.n_tiles_n;
-  c.nt = local / mtiles;             // tiles of one expert: n-major, m fastest
-  c.mt = local - c.nt * mtiles;
+  banded_mn(local, mtiles, p.n_tiles_n, c.mt, c.nt);
   c.row0 = info.w + c.mt * bm;
   c.gmt = mstart + c.mt;
   c.rows = min(bm, c.count - c.mt * bm);
@@ -837,8 +858,9 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const GemmArgs& p, int til
   const int mtiles = (c.count + BM - 1) / BM;
   const int ptiles = (mtiles + 1) / 2;
   const int local = tile - info.y * p.n_tiles_n;
-  c.nt = local / ptiles;
-  c.mt = 2 * (local - c.nt * ptiles) + rank;
+  int pm;
+  banded_mn(local, ptiles, p.n_tiles_n, pm, c.nt);
+  c.mt = 2 * pm + rank;
   c.row0 = info.w + c.mt * BM;
   c.gmt = ld_cg(p.mtile_start + c.e) + c.mt;
   c.rows = max(0, min(BM, c.count - c.mt * BM));

@@ -73,7 +73,8 @@ struct GemmArgs {
   const int32_t* ptile_start;  // [n_experts + 1] prefix sum of ceil(ceil(count/128)/2) (CTA pairs)
   // Row-tile table: entry g in [mtile_start[e], mtile_start[e + 1]) holds {e, mtile_start[e],
   // counts[e], offsets[e]}; the CTA-pair table the same over ptile_start with ptile_start[e]
-  // in .y.  Tile t of the n-major order belongs to the expert of entry t / n_tiles_n.
+  // in .y.  An expert's tiles are consecutive (banded row-tile order inside the expert), so
+  // tile t belongs to the expert of entry t / n_tiles_n.
   const int4* tile_info;
   const int4* ptile_info;
   // Chained linear1 -> linear2 in one kernel: linear1's epilogue adds 1 to dep_signal[e] when a
