@@ -1698,11 +1698,13 @@ cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMa
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = gemm_small_smem_bytes();
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;      // co-resident CTAs (also when recorded in a graph)
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = dependent_launch() ? 2 : 1;
   if (g2.bn == kGemmBN2Double) return cudaLaunchKernelEx(&cfg, chained_gemm_kernel<kGemmBN2Double>, a1, a2, b1, b2, g1, g2);
   return cudaLaunchKernelEx(&cfg, chained_gemm_kernel<kGemmBN>, a1, a2, b1, b2, g1, g2);
 }

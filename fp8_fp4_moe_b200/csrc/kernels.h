@@ -124,7 +124,8 @@ cudaError_t launch_gemm_linear1(const AMaps& a, const CUtensorMap& b, const Gemm
                                 cudaStream_t s, bool small_tiles = false);
 cudaError_t launch_gemm_linear2(const AMaps& a, const CUtensorMap& b, const GemmArgs& args, int grid,
                                 cudaStream_t s, bool small_tiles = false);
-// linear1 + linear2 in one cooperative launch (small-tile layout, bm == kGemmBMSmall):
+// linear1 + linear2 in one cooperative launch (small-tile layout, bm == kGemmBMSmall), a
+// programmatic dependent of the kernel before it while dependent launches are on:
 // g1.dep_signal == g2.dep_wait (n_experts counters, zero before the launch), g2.dep_per_mtile =
 // g1.n_tiles_n; b2's box height = g2.bn.  grid <= the co-resident CTAs of the device.
 cudaError_t launch_gemm_chain(const AMaps& a1, const AMaps& a2, const CUtensorMap& b1, const CUtensorMap& b2,
@@ -254,11 +255,13 @@ cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_part
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
                                  int32_t* group_base, int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
                                  int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s);
-// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms (bm-row tiles).
+// Writes slot_pos/perm and (if x != nullptr) the dispatched E4M3 rows + scale atoms (bm-row tiles);
+// also zeroes zero[0 .. n_zero) (if given) for the kernels that follow.
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
-                                 int k, int shared, int bm, cudaStream_t s);
+                                 int k, int shared, int bm, cudaStream_t s, uint32_t* zero = nullptr,
+                                 int n_zero = 0);
 // Token-order quantisation (debug entry point).
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s);
 // Auxiliary-loss-free balancing step from the routed experts' loads.

@@ -149,6 +149,9 @@ int plan_bm(moe_plan_t p) {
   return decode_shaped(p) && p->T <= 32 ? kGemmBMSmall : kGemmBM;
 }
 
+// linear1 and linear2 as one cooperative launch (MOE_OPT_CHAIN; 32-row tiles, at most 16 tokens)
+bool use_chain(moe_plan_t p) { return p->chain && plan_bm(p) == kGemmBMSmall && p->T <= 16; }
+
 // Programmatic dependent launches: automatic for at most 64 tokens, where each kernel is short
 // and launch latency and the GEMMs' early weight requests matter; with more tokens the GEMM's
 // early-resident CTAs take the registers the scatter's blocks need, and the forward measured
@@ -330,7 +333,8 @@ int run_front(moe_plan_t p, const uint16_t* x, const float* W_router, const floa
                            region<int32_t>(p, MOE_REGION_OFFSETS), at<int32_t>(p, p->off_mtile),
                            region<int32_t>(p, MOE_REGION_SLOT_POS), region<int32_t>(p, MOE_REGION_PERM),
                            region<uint8_t>(p, MOE_REGION_XQ), region<uint8_t>(p, MOE_REGION_XSF), p->T, p->H,
-                           p->E, p->k, p->shared, plan_bm(p), s);
+                           p->E, p->k, p->shared, plan_bm(p), s,
+                           use_chain(p) ? at<uint32_t>(p, p->off_dep) : nullptr, p->n);
   mark(p, 1 + MOE_PHASE_SCATTER_QUANT, s);
   return cuda_rc(e);
 }
@@ -461,11 +465,10 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
   } else {
     const bool small_tiles = plan_bm(p) == kGemmBMSmall;
     const CUtensorMap& b2 = a2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
-    if (small_tiles && p->T <= 16 && p->chain) {
+    if (use_chain(p)) {
       // one cooperative launch: linear2 tiles start as soon as their expert's linear1 tiles are
-      // stored (per-expert counters, zeroed here); reported under linear1
+      // stored (per-expert counters, zeroed by the scatter kernel); reported under linear1
       uint32_t* dep = at<uint32_t>(p, p->off_dep);
-      if (cudaMemsetAsync(dep, 0, (size_t)p->n * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
       a1.dep_signal = dep;
       a2.dep_wait = dep;
       a2.dep_per_mtile = a1.n_tiles_n;

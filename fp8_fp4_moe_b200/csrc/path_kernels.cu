@@ -246,9 +246,13 @@ __global__ void __launch_bounds__(256) scatter_quant_kernel(const uint16_t* __re
                                                             const int32_t* __restrict__ mtile_start,
                                                             int32_t* slot_pos, int32_t* perm, uint8_t* xq,
                                                             uint8_t* xsf, int T, int H, int E, int k, int shared,
-                                                            int bm) {
+                                                            int bm, uint32_t* zero, int n_zero) {
   griddep_wait();
   griddep_launch_dependents();
+  // counters the next kernel starts from (the chained GEMM's per-expert linear1 counts): zeroed
+  // here, once every kernel before this one has finished, so no memset sits between the launches
+  if (zero != nullptr && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
   scatter_items<SL>((long)blockIdx.x * 8 + threadIdx.x / 32, x, topk_ids, local_rank, group_base, offsets,
                     mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
 }
@@ -389,17 +393,19 @@ cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, i
 cudaError_t launch_scatter_quant(const uint16_t* x, const int32_t* topk_ids, const int32_t* local_rank,
                                  const int32_t* group_base, const int32_t* offsets, const int32_t* mtile_start,
                                  int32_t* slot_pos, int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
-                                 int k, int shared, int bm, cudaStream_t s) {
+                                 int k, int shared, int bm, cudaStream_t s, uint32_t* zero, int n_zero) {
   const long slices = (long)T * (x == nullptr ? 1 : (H + 255) / 256);
   // Mixtral T = 4096 (65,536 slices): 4 per warp, the scatter 26 -> 19 us; DSV3 T = 512
   // (14,336) and T = 1 (28) keep one per warp, four would leave too few warps in flight
   if (x != nullptr && slices >= 32768) {
     const long items = (long)T * (((H + 255) / 256 + 3) / 4);
     return launch_kernel(scatter_quant_kernel<4>, (unsigned)((items + 7) / 8), 256, 0, s, x, topk_ids, local_rank,
-                         group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
+                         group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm, zero,
+                         n_zero);
   }
   return launch_kernel(scatter_quant_kernel<1>, (unsigned)((slices + 7) / 8), 256, 0, s, x, topk_ids, local_rank,
-                       group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm);
+                       group_base, offsets, mtile_start, slot_pos, perm, xq, xsf, T, H, E, k, shared, bm, zero,
+                       n_zero);
 }
 
 cudaError_t launch_quant_tokens(const uint16_t* x, uint8_t* xq, float* xs, int T, int H, cudaStream_t s) {
