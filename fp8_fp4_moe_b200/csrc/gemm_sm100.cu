@@ -460,9 +460,10 @@ __device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t need,
 
 // Work an epilogue warp does before its first tile or after its last one (the single-kernel
 // forward's scatter and combine); called with the warp's index among all epilogue warps of the
-// grid, their number, and whether the GEMM ran without a device-side failure.
+// grid, their number, whether the GEMM ran without a device-side failure, and the CTA's
+// (1024-aligned) dynamic shared memory.
 struct NoEpilogueWork {
-  __device__ __forceinline__ void operator()(int, int, bool) const {}
+  __device__ __forceinline__ void operator()(int, int, bool, uint8_t*) const {}
 };
 
 // One grouped GEMM over tiles cta, cta + n_ctas, ... by all kGemmThreads threads of the CTA,
@@ -711,7 +712,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
     const int half = (warp - 2) / 4;      // which half of the accumulator columns
     uint8_t* obuf = L::kStaging ? smem + L::stage_out + (warp - 2) * 2048 : nullptr;
     const int epi_id = cta * kEpiWarps + (warp - 2), n_epi = n_ctas * kEpiWarps;
-    pre(epi_id, n_epi, true);
+    pre(epi_id, n_epi, true, smem);
     uint32_t uses0 = 0, uses1 = 0;
     int next_slot = 0;
     int buf = 0;
@@ -754,7 +755,7 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       uses1 += sp.hi == 1;
       buf ^= 1;
     }
-    post(epi_id, n_epi, all_ok && !*abort_flag);
+    post(epi_id, n_epi, all_ok && !*abort_flag, smem);
   }
 
   __syncthreads();
@@ -1309,7 +1310,7 @@ __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, lo
 // once every CTA has done so.
 struct ScatterWork {
   const FusedArgs* a;
-  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool) const {
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool, uint8_t*) const {
     const FusedArgs& f = *a;
     const int slices = (f.H + 255) / 256;
     if ((long)f.T * slices >= 32768) {
@@ -1336,27 +1337,122 @@ struct ScatterWork {
 };
 
 // After its last linear2 tile, each epilogue warp waits (bounded) until every linear2 tile of
-// the grid is stored, then combines its share of the (token, slice) items.
+// the grid is stored, then combines its share of the (token, 256-channel slice) items.  With one
+// CTA per SM only eight warps per SM do this, so they gather with bulk copies: per batch of items
+// each lane of a warp copies one expert row slice (512 B) into the warp's 16 KB slice of the
+// weight-stage buffers (idle once the CTA's last linear2 tile is done), all completing on one
+// mbarrier of the warp (in the amax area, which linear2 does not use); the lanes then sum the
+// rows from shared memory in slot order, gate-weighted, add the shared row and store bf16.
+constexpr uint32_t kCombineSlice = 16384;        // shared memory per epilogue warp
+template <class L>
 struct CombineWork {
+  static_assert(L::sfa - L::b >= kEpiWarps * kCombineSlice, "the weight-stage region holds the combine slices");
+  static_assert(L::stage_out - L::amax >= kEpiWarps * 8, "the amax area holds the combine barriers");
   const FusedArgs* a;
   uint32_t tiles2;                 // linear2 tiles of the forward
-  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool ok) const {
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool ok, uint8_t* smem) const {
     const FusedArgs& f = *a;
-    if (!ok) return;
+    if (!__all_sync(0xffffffffu, ok)) return;             // warp-uniform from here on
+    const int lane = threadIdx.x % 32;
     // lane 0 polls for the warp
     bool ready = true;
-    if (threadIdx.x % 32 == 0)
+    if (lane == 0)
       ready = wait_counter(f.counters + 1, tiles2, f.status, f.timeout_ns, kWhereGemmDependency + 1, nullptr);
     ready = __shfl_sync(0xffffffffu, ready, 0);
-    __syncwarp();
     if (!ready) return;
+    __syncwarp();
+    fence_proxy_async_global();            // the acquired rows, before this lane's bulk copies
     if (f.stamps != nullptr && threadIdx.x == 2 * 32) f.stamps[kStampCombine * kStampMaxCtas + blockIdx.x] = globaltimer_ns();
-    const long items = (long)f.T * ((f.H + 255) / 256);
-    // several items per warp in flight: one CTA per SM leaves only 8 epilogue warps to hide latency
-    if (f.k <= 2) fused_combine<2, 4>(f, items, epi_id, n_epi);
-    else if (f.k <= 4) fused_combine<4, 4>(f, items, epi_id, n_epi);
-    else if (f.k <= 8) fused_combine<8, 2>(f, items, epi_id, n_epi);
-    else fused_combine<16, 1>(f, items, epi_id, n_epi);
+    const int w = epi_id % kEpiWarps;
+    uint8_t* buf = smem + L::b + w * kCombineSlice;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::amax) + w;
+    if (lane == 0) {
+      mbar_init(bar, 1);
+      fence_mbarrier_init();
+    }
+    __syncwarp();
+    const int R = f.k + f.shared;                        // rows per item
+    const int nb = max(1, min(min(8, 32 / R), (int)(kCombineSlice / (R * 512))));   // items per batch (R <= 32)
+    const int slices = (f.H + 255) / 256;
+    const long items = (long)f.T * slices;
+    const long Rk = (long)f.T * f.k;
+    uint32_t parity = 0;
+    for (long base = epi_id; base < items; base += (long)n_epi * nb) {
+      // lane l < nb * R copies row j = l % R of item i = l / R of this batch
+      const int i = lane / R, j = lane % R;
+      const long it = base + (long)i * n_epi;
+      const bool act = i < nb && it < items;
+      int t = 0, c0 = 0;
+      uint32_t bytes = 0;
+      long row = 0;
+      float g = 0.f;
+      if (act) {
+        t = (int)(it / slices);
+        c0 = (int)(it % slices) * 256;
+        bytes = (uint32_t)min(256, f.H - c0) * 2;
+        if (j < f.k) {
+          row = ld_cg(f.slot_pos + (long)t * f.k + j);
+          g = f.gates[(long)t * f.k + j];
+        } else {
+          row = Rk + t;                                  // the shared expert's row
+          g = 1.f;
+        }
+      }
+      uint32_t total = bytes;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
+      if (lane == 0) mbar_arrive_expect_tx(bar, total);
+      __syncwarp();
+      if (act) bulk_load(buf + lane * 512, f.y + row * f.H + c0, bytes, bar);
+      const bool landed = __all_sync(0xffffffffu, mbar_wait_drain(bar, parity, f.timeout_ns));
+      if (!landed) {
+        if (lane == 0) report_status(f.status, kStatusTimeout, kWhereGemmDrain + 2, (uint32_t)base);
+        return;                        // (the barrier stays valid; nothing else uses this memory)
+      }
+      parity ^= 1;
+      // each lane: 8 channels of every item of the batch
+      for (int b = 0; b < nb; ++b) {
+        const long itb = base + (long)b * n_epi;
+        if (itb >= items) break;
+        const int tb = (int)(itb / slices), cb = (int)(itb % slices) * 256;
+        const int ch = lane * 8;
+        const bool live = cb + ch < f.H;         // (not warp-uniform on a ragged last slice)
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int r = 0; r < R; ++r) {
+          const float gr = __shfl_sync(0xffffffffu, g, b * R + r);     // every lane takes part
+          if (!live) continue;
+          const uint4 v = *reinterpret_cast<const uint4*>(buf + (b * R + r) * 512 + ch * 2);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          if (r < f.k) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[2 * q] = fmaf(gr, __uint_as_float(wv[q] << 16), acc[2 * q]);
+              acc[2 * q + 1] = fmaf(gr, __uint_as_float(wv[q] & 0xFFFF0000u), acc[2 * q + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[2 * q] += __uint_as_float(wv[q] << 16);
+              acc[2 * q + 1] += __uint_as_float(wv[q] & 0xFFFF0000u);
+            }
+          }
+        }
+        uint4 o;
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(acc[0], acc[1]);
+        __nv_bfloat162 b1 = __floats2bfloat162_rn(acc[2], acc[3]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[4], acc[5]);
+        __nv_bfloat162 b3 = __floats2bfloat162_rn(acc[6], acc[7]);
+        o.x = *reinterpret_cast<uint32_t*>(&b0);
+        o.y = *reinterpret_cast<uint32_t*>(&b1);
+        o.z = *reinterpret_cast<uint32_t*>(&b2);
+        o.w = *reinterpret_cast<uint32_t*>(&b3);
+        if (live) *reinterpret_cast<uint4*>(f.out + (long)tb * f.H + cb + ch) = o;
+      }
+      __syncwarp();                    // every lane has read the batch before the next copies land
+    }
+    if (lane == 0) mbar_inval(bar);
   }
 };
 
@@ -1481,8 +1577,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     g2.dep_per_mtile = a.g1.n_tiles_n;
     g2.tiles_done = a.counters + 1;
     const uint32_t tiles2 = (uint32_t)(ld_cg(a.mtile_start + a.E + a.shared) * a.g2.n_tiles_n);
-    gemm_body<2, L, NB2, NoEpilogueWork, CombineWork>(amA2, tmB2, g2, smem, tmem_base, cta, n_ctas,
-                                                      NoEpilogueWork(), CombineWork{&a, tiles2});
+    gemm_body<2, L, NB2, NoEpilogueWork, CombineWork<L>>(amA2, tmB2, g2, smem, tmem_base, cta, n_ctas,
+                                                         NoEpilogueWork(), CombineWork<L>{&a, tiles2});
     stamp(kStampEnd);
   }
   __syncthreads();

@@ -32,10 +32,9 @@ TILE_STRIDE = {"mixtral": 16, "dsv3_t1": 1, "dsv3_t512": 1, "dsv3_t8192_zipf": 1
 SLACK_NEEDED_MAX = 1e-3
 # expert rows (bf16 linear2 output) against the oracle's, relative Frobenius per expert
 ROW_REL_TOL = 5e-3
-# separate launches for every workload; the single persistent kernel for three of them; the
-# chained linear1 -> linear2 launch for single-token decode
-CASES = [(n, 0, 0) for n in RANDOM_TOKENS] + [("dsv3_t1", 1, 0), ("dsv3_t512", 1, 0), ("mixtral", 1, 0),
-                                              ("dsv3_t1", 0, 1)]
+# separate launches and the single persistent kernel for every workload; the chained
+# linear1 -> linear2 launch for single-token decode
+CASES = [(n, 0, 0) for n in RANDOM_TOKENS] + [(n, 1, 0) for n in RANDOM_TOKENS] + [("dsv3_t1", 0, 1)]
 
 
 def stratified_rows(counts, offsets, stride, busiest, rng):
