@@ -105,14 +105,22 @@ enum moe_option {
                                   Needs 128-row tiles.                                     */
   MOE_OPT_FUSED = 10,          /* 1 = moe_forward runs every step (router, top-k, dispatch
                                   scans, scatter + quantisation, linear1, linear2, combine)
-                                  in ONE persistent cooperative kernel, one CTA per SM,
-                                  the steps separated by grid-wide barriers (bounded
-                                  waits); weight preparation, when needed, runs before it.
-                                  Router: tensor cores when MOE_OPT_ROUTER_TC applies,
-                                  else CUDA cores (block per expert and token for
-                                  T*E <= 4096, warp per token and expert chunk otherwise).
-                                  moe_phase_times reports the whole kernel under the router
-                                  phase.  No CUDA graph is recorded.  Default 0.          */
+                                  in ONE persistent cooperative kernel, one CTA per SM:
+                                  grid-wide barriers after the router and after top-k and
+                                  the scans; from there on readiness counters (bounded
+                                  waits) -- the linear1 producers start once every CTA has
+                                  scattered its share (done by the epilogue warps before
+                                  their first tile), linear2 tiles once their expert's
+                                  linear1 tiles are stored, the combine (epilogue warps,
+                                  bulk copies into the idle operand buffers) once every
+                                  linear2 tile is.  Weight preparation, when needed, runs
+                                  before it.  Router: tensor cores when MOE_OPT_ROUTER_TC
+                                  applies; with at most 16 tokens (E a multiple of 4, at
+                                  most 256) a warp per (expert, K part) over all tokens;
+                                  else CUDA cores as the separate launches.  With MOE_OPT_PHASE_EVENTS = 1 every CTA writes
+                                  the global timer at each step into the "stamps" region
+                                  and moe_phase_times splits the kernel's time by them.
+                                  No CUDA graph is recorded.  Default 0.                  */
   MOE_OPT_DEPENDENT_LAUNCH = 11, /* 1: the kernels after the first of a moe_forward are
                                   launched as programmatic dependents (each waits on the
                                   device for its predecessor; the grouped GEMMs request
