@@ -1304,28 +1304,118 @@ __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, lo
   }
 }
 
+// The single-kernel forward's scatter of many tokens, one item = 8 slices (2048 channels) of one
+// token's x row: the warp quantises them as scatter_items does, stages the E4M3 bytes in its 2 KB
+// of the epilogue staging area (idle before the first tile) and sends them to each of the token's
+// k (+ shared) dispatched rows with one bulk copy, in place of 8 x 32 eight-byte stores per row;
+// the scale bytes and positions are plain stores.  `pending`: this warp has bulk copies whose
+// staging bytes may still be read.
+constexpr int kScatterBulkSlices = 8;
+__device__ __forceinline__ void scatter_item_bulk(long item, const FusedArgs& f, uint8_t* stage, bool& pending) {
+  constexpr int SL = kScatterBulkSlices;
+  const int lane = threadIdx.x % 32;
+  const int n_slices = (f.H + 255) / 256;
+  const int n_grp = (n_slices + SL - 1) / SL;
+  const int t = (int)(item / n_grp);
+  const int grp = (int)(item % n_grp);
+  const int g = t / 32;
+  const long R = (long)f.T * f.k;
+  const int kw = f.H / 128;
+  // the token's 8 channels of this lane in each slice, loaded before the position lookups
+  uint4 raw[SL];
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    raw[s] = c0 < f.H ? *reinterpret_cast<const uint4*>(f.x + (long)t * f.H + c0) : make_uint4(0, 0, 0, 0);
+  }
+  int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
+  int e = -1;
+  if (lane < f.k) {
+    e = f.topk_ids[(long)t * f.k + lane];
+    row = f.offsets[e] + f.group_base[(long)g * f.E + e] + f.local_rank[(long)t * f.k + lane];
+    if (grp == 0) {
+      f.slot_pos[(long)t * f.k + lane] = row;
+      f.perm[row] = t * f.k + lane;
+    }
+  } else if (lane == f.k && f.shared) {
+    e = f.E;
+    row = (int)(R + t);
+  }
+  long sf_off = 0;                       // this destination row's word inside its tile's scale atoms
+  if (e >= 0) {
+    const int rank = row - f.offsets[e];
+    const int r = rank % f.bm;
+    sf_off = ((long)(f.mtile_start[e] + rank / f.bm) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
+  }
+  const int ndst = f.k + f.shared;
+  // the previous item's copies must have read the staging bytes before they are overwritten
+  if (pending && lane < ndst) bulk_wait_read<0>();
+  __syncwarp();
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    if ((grp * SL + s) * 256 >= f.H) break;      // warp-uniform: the slice starts past H
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    const bool active = c0 < f.H;                // H % 128 == 0: whole half-warps
+    const uint4 rw = raw[s];
+    float v[8];
+    v[0] = __uint_as_float(rw.x << 16); v[1] = __uint_as_float(rw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(rw.y << 16); v[3] = __uint_as_float(rw.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(rw.z << 16); v[5] = __uint_as_float(rw.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(rw.w << 16); v[7] = __uint_as_float(rw.w & 0xFFFF0000u);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int p = pow2_exp_e4m3(amax);
+    const float sc = exp2_neg(p);
+    uint2 q;
+    q.x = pack_e4m3x4(v[0] * sc, v[1] * sc, v[2] * sc, v[3] * sc);
+    q.y = pack_e4m3x4(v[4] * sc, v[5] * sc, v[6] * sc, v[7] * sc);
+    if (active) *reinterpret_cast<uint2*>(stage + s * 256 + lane * 8) = q;
+    const uint32_t code = (uint32_t)(p + 127) * 0x01010101u;
+    const int blk = c0 / 128;
+    for (int d = 0; d < ndst; ++d) {
+      const long so = __shfl_sync(0xffffffffu, sf_off, d);
+      if (active && (lane & 15) == 0) *reinterpret_cast<uint32_t*>(f.xsf + so + (long)blk * 512) = code;
+    }
+  }
+  fence_proxy_async_smem();              // this lane's staging bytes, before the copies read them
+  __syncwarp();
+  if (lane < ndst) {
+    const int c_base = grp * SL * 256;
+    const uint32_t bytes = (uint32_t)min(SL * 256, f.H - c_base);   // E4M3: one byte a channel
+    bulk_store(f.xq + (long)row * f.H + c_base, stage, bytes);
+    bulk_commit();
+  }
+  pending = true;
+}
+
 // Before its first linear1 tile, each epilogue warp of the grid scatters (and quantises) its
-// share of the (token, 256-channel slice) items; once all eight of a CTA's have, one thread adds
-// 1 to the scatter counter (one atomic per CTA, not per warp); the producers load A rows only
-// once every CTA has done so.
+// share of the (token, channel group) items; once all eight of a CTA's have, one thread adds 1 to
+// the scatter counter (one atomic per CTA, not per warp); the producers load A rows only once
+// every CTA has done so.
+template <class L>
 struct ScatterWork {
   const FusedArgs* a;
-  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool, uint8_t*) const {
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool, uint8_t* smem) const {
     const FusedArgs& f = *a;
     const int slices = (f.H + 255) / 256;
-    if ((long)f.T * slices >= 32768) {
-      // many items: four slices per item, their x loads issued before the position lookups
-      const long items = (long)f.T * ((slices + 3) / 4);
-      for (long it = epi_id; it < items; it += n_epi)
-        scatter_items<4>(it, f.x, f.topk_ids, f.local_rank, f.group_base, f.offsets, f.mtile_start, f.slot_pos,
-                         f.perm, f.xq, f.xsf, f.T, f.H, f.E, f.k, f.shared, f.bm);
+    bool pending = false;
+    if (L::kStaging && (long)f.T * slices >= 32768) {
+      // many items: eight slices per item through the warp's 2 KB of staging memory
+      uint8_t* stage = smem + L::stage_out + (epi_id % kEpiWarps) * 2048;
+      const long items = (long)f.T * ((slices + kScatterBulkSlices - 1) / kScatterBulkSlices);
+      for (long it = epi_id; it < items; it += n_epi) scatter_item_bulk(it, f, stage, pending);
     } else {
       const long items = (long)f.T * slices;
       for (long it = epi_id; it < items; it += n_epi)
         scatter_item(it, f.x, f.topk_ids, f.local_rank, f.group_base, f.offsets, f.mtile_start, f.slot_pos, f.perm,
                      f.xq, f.xsf, f.T, f.H, f.E, f.k, f.shared, f.bm);
     }
-    // generic stores -> other CTAs' TMA reads: proxy fence, CTA barrier, gpu-scope release
+    // bulk copies complete (their writes performed), generic stores -> other CTAs' TMA reads:
+    // proxy fence, CTA barrier, gpu-scope release
+    if (pending && (threadIdx.x % 32) < f.k + f.shared) bulk_wait<0>();
     fence_proxy_async_global();
     epi_bar();
     if (threadIdx.x == 2 * 32) {
@@ -1337,93 +1427,63 @@ struct ScatterWork {
 };
 
 // After its last linear2 tile, each epilogue warp waits (bounded) until every linear2 tile of
-// the grid is stored, then combines its share of the (token, 256-channel slice) items.  With one
-// CTA per SM only eight warps per SM do this, so they gather with bulk copies: per batch of items
-// each lane of a warp copies one expert row slice (512 B) into the warp's 16 KB slice of the
-// weight-stage buffers (idle once the CTA's last linear2 tile is done), all completing on one
-// mbarrier of the warp (in the amax area, which linear2 does not use); the lanes then sum the
-// rows from shared memory in slot order, gate-weighted, add the shared row and store bf16.
-constexpr uint32_t kCombineSlice = 16384;        // shared memory per epilogue warp
+// the grid is stored, then combines its share of the (token, channel chunk) items.  With one CTA
+// per SM only eight warps per SM do this, so they gather with bulk copies into the operand stage
+// buffers (idle once the CTA's last linear2 tile is done): per item, lane j < k + shared copies
+// expert row j's chunk (1024 channels, 2 KB; 512 when k + shared > 12 rows would not fit) into
+// the warp's slice of that memory, completing on one mbarrier of the warp (in the amax area,
+// which linear2 does not use); the lanes then sum the rows from shared memory in slot order,
+// gate-weighted, add the shared row and store bf16.
 template <class L>
 struct CombineWork {
-  static_assert(L::sfa - L::b >= kEpiWarps * kCombineSlice, "the weight-stage region holds the combine slices");
+  static constexpr uint32_t kSlice = ((L::sfa - L::a) / kEpiWarps) & ~1023u;   // per warp
+  static_assert(kSlice >= 12 * 2048 && kSlice >= 17 * 1024, "a warp's slice holds one item");
   static_assert(L::stage_out - L::amax >= kEpiWarps * 8, "the amax area holds the combine barriers");
   const FusedArgs* a;
   uint32_t tiles2;                 // linear2 tiles of the forward
-  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool ok, uint8_t* smem) const {
+
+  template <int CW>
+  __device__ __forceinline__ bool run(int epi_id, int n_epi, uint8_t* buf, uint64_t* bar) const {
     const FusedArgs& f = *a;
-    if (!__all_sync(0xffffffffu, ok)) return;             // warp-uniform from here on
     const int lane = threadIdx.x % 32;
-    // lane 0 polls for the warp
-    bool ready = true;
-    if (lane == 0)
-      ready = wait_counter(f.counters + 1, tiles2, f.status, f.timeout_ns, kWhereGemmDependency + 1, nullptr);
-    ready = __shfl_sync(0xffffffffu, ready, 0);
-    if (!ready) return;
-    __syncwarp();
-    fence_proxy_async_global();            // the acquired rows, before this lane's bulk copies
-    if (f.stamps != nullptr && threadIdx.x == 2 * 32) f.stamps[kStampCombine * kStampMaxCtas + blockIdx.x] = globaltimer_ns();
-    const int w = epi_id % kEpiWarps;
-    uint8_t* buf = smem + L::b + w * kCombineSlice;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::amax) + w;
-    if (lane == 0) {
-      mbar_init(bar, 1);
-      fence_mbarrier_init();
-    }
-    __syncwarp();
     const int R = f.k + f.shared;                        // rows per item
-    const int nb = max(1, min(min(8, 32 / R), (int)(kCombineSlice / (R * 512))));   // items per batch (R <= 32)
-    const int slices = (f.H + 255) / 256;
-    const long items = (long)f.T * slices;
+    const int chunks = (f.H + CW - 1) / CW;
+    const long items = (long)f.T * chunks;
     const long Rk = (long)f.T * f.k;
     uint32_t parity = 0;
-    for (long base = epi_id; base < items; base += (long)n_epi * nb) {
-      // lane l < nb * R copies row j = l % R of item i = l / R of this batch
-      const int i = lane / R, j = lane % R;
-      const long it = base + (long)i * n_epi;
-      const bool act = i < nb && it < items;
-      int t = 0, c0 = 0;
-      uint32_t bytes = 0;
+    for (long it = epi_id; it < items; it += n_epi) {
+      const int t = (int)(it / chunks);
+      const int c0 = (int)(it % chunks) * CW;
+      const int w_ch = min(CW, f.H - c0);                // channels of this chunk (a multiple of 128)
       long row = 0;
       float g = 0.f;
-      if (act) {
-        t = (int)(it / slices);
-        c0 = (int)(it % slices) * 256;
-        bytes = (uint32_t)min(256, f.H - c0) * 2;
-        if (j < f.k) {
-          row = ld_cg(f.slot_pos + (long)t * f.k + j);
-          g = f.gates[(long)t * f.k + j];
-        } else {
-          row = Rk + t;                                  // the shared expert's row
-          g = 1.f;
-        }
+      if (lane < f.k) {
+        row = ld_cg(f.slot_pos + (long)t * f.k + lane);
+        g = f.gates[(long)t * f.k + lane];
+      } else if (lane < R) {
+        row = Rk + t;                                    // the shared expert's row
+        g = 1.f;
       }
-      uint32_t total = bytes;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) total += __shfl_xor_sync(0xffffffffu, total, off);
-      if (lane == 0) mbar_arrive_expect_tx(bar, total);
+      if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(R * w_ch * 2));
       __syncwarp();
-      if (act) bulk_load(buf + lane * 512, f.y + row * f.H + c0, bytes, bar);
-      const bool landed = __all_sync(0xffffffffu, mbar_wait_drain(bar, parity, f.timeout_ns));
-      if (!landed) {
-        if (lane == 0) report_status(f.status, kStatusTimeout, kWhereGemmDrain + 2, (uint32_t)base);
-        return;                        // (the barrier stays valid; nothing else uses this memory)
+      if (lane < R) bulk_load(buf + lane * (CW * 2), f.y + row * f.H + c0, (uint32_t)w_ch * 2, bar);
+      if (!__all_sync(0xffffffffu, mbar_wait_drain(bar, parity, f.timeout_ns))) {
+        if (lane == 0) report_status(f.status, kStatusTimeout, kWhereGemmDrain + 2, (uint32_t)it);
+        return false;                  // (the barrier stays valid; nothing else uses this memory)
       }
       parity ^= 1;
-      // each lane: 8 channels of every item of the batch
-      for (int b = 0; b < nb; ++b) {
-        const long itb = base + (long)b * n_epi;
-        if (itb >= items) break;
-        const int tb = (int)(itb / slices), cb = (int)(itb % slices) * 256;
-        const int ch = lane * 8;
-        const bool live = cb + ch < f.H;         // (not warp-uniform on a ragged last slice)
+      // lane: 8 channels in each 256-channel group of the chunk
+#pragma unroll
+      for (int q4 = 0; q4 < CW / 256; ++q4) {
+        const int ch = q4 * 256 + lane * 8;
+        const bool live = ch < w_ch;                     // warp-uniform per half-warp (128-channel steps)
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
         for (int r = 0; r < R; ++r) {
-          const float gr = __shfl_sync(0xffffffffu, g, b * R + r);     // every lane takes part
+          const float gr = __shfl_sync(0xffffffffu, g, r);             // every lane takes part
           if (!live) continue;
-          const uint4 v = *reinterpret_cast<const uint4*>(buf + (b * R + r) * 512 + ch * 2);
+          const uint4 v = *reinterpret_cast<const uint4*>(buf + r * (CW * 2) + ch * 2);
           const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
           if (r < f.k) {
 #pragma unroll
@@ -1448,11 +1508,36 @@ struct CombineWork {
         o.y = *reinterpret_cast<uint32_t*>(&b1);
         o.z = *reinterpret_cast<uint32_t*>(&b2);
         o.w = *reinterpret_cast<uint32_t*>(&b3);
-        if (live) *reinterpret_cast<uint4*>(f.out + (long)tb * f.H + cb + ch) = o;
+        if (live) *reinterpret_cast<uint4*>(f.out + (long)t * f.H + c0 + ch) = o;
       }
-      __syncwarp();                    // every lane has read the batch before the next copies land
+      __syncwarp();                    // every lane has read the item before the next copies land
     }
-    if (lane == 0) mbar_inval(bar);
+    return true;
+  }
+
+  __device__ __forceinline__ void operator()(int epi_id, int n_epi, bool ok, uint8_t* smem) const {
+    const FusedArgs& f = *a;
+    if (!__all_sync(0xffffffffu, ok)) return;             // warp-uniform from here on
+    const int lane = threadIdx.x % 32;
+    // lane 0 polls for the warp
+    bool ready = true;
+    if (lane == 0)
+      ready = wait_counter(f.counters + 1, tiles2, f.status, f.timeout_ns, kWhereGemmDependency + 1, nullptr);
+    ready = __shfl_sync(0xffffffffu, ready, 0);
+    if (!ready) return;
+    __syncwarp();
+    fence_proxy_async_global();            // the acquired rows, before this lane's bulk copies
+    if (f.stamps != nullptr && threadIdx.x == 2 * 32) f.stamps[kStampCombine * kStampMaxCtas + blockIdx.x] = globaltimer_ns();
+    const int w = epi_id % kEpiWarps;
+    uint8_t* buf = smem + L::a + w * kSlice;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::amax) + w;
+    if (lane == 0) {
+      mbar_init(bar, 1);
+      fence_mbarrier_init();
+    }
+    __syncwarp();
+    const bool done = f.k + f.shared <= 12 ? run<1024>(epi_id, n_epi, buf, bar) : run<512>(epi_id, n_epi, buf, bar);
+    if (done && lane == 0) mbar_inval(bar);
   }
 };
 
@@ -1568,7 +1653,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     g1.rows_ready_need = (uint32_t)n_ctas;
     g1.dep_signal = a.counters + 2;
     g1.stamp_rows = a.stamps != nullptr ? a.stamps + kStampRowsReady * kStampMaxCtas : nullptr;
-    gemm_body<1, L, 256, ScatterWork>(amA1, tmB1, g1, smem, tmem_base, cta, n_ctas, ScatterWork{&a});
+    gemm_body<1, L, 256, ScatterWork<L>>(amA1, tmB1, g1, smem, tmem_base, cta, n_ctas, ScatterWork<L>{&a});
     stamp(kStampLinear1);
     // S5 linear2: each tile's producer waits only for its expert's linear1 tiles; S6 combine by
     // the epilogue warps once every linear2 tile is stored

@@ -588,3 +588,56 @@ def test_zero_padding_changes_no_bit(cuda_lib, name):
         outs.append(p.region("y").clone())
     assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
     assert torch.equal(outs[1].view(torch.int16), outs[3].view(torch.int16))
+
+
+# A grid of a few CTAs (MOE_OPT_MAX_SMS) gives every CTA many tiles and every epilogue warp many
+# scatter and combine batches (the fused kernel's per-warp mbarrier phases wrap many times): the
+# arithmetic of a tile or an item does not depend on which CTA runs it, so the output equals the
+# full grid's bit for bit, and the oracle's within tolerance.
+@pytest.mark.parametrize("name,fused,pair_tiles", [("ragged_shared", 1, None), ("k10", 1, None), ("h896", 1, None),
+                                                   ("ragged_shared", 0, None), ("tc_router", 0, 2)])
+def test_few_ctas_match_the_full_grid(cuda_lib, name, fused, pair_tiles):
+    w = SMALL[name]
+    case = make_case(w, seed=41)
+    d = to_device(case)
+    outs = []
+    for max_sms in (0, 2, 7):
+        p = plan_for(w, fused=fused, pair_tiles=pair_tiles)
+        p.set_option(binding.MOE_OPT_MAX_SMS, max_sms)
+        outs.append(p.forward(**d).clone())
+        assert p.check_status()[0] == 0, max_sms
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert_output_close(bits(outs[1]), ref["y"], f"{name} fused={fused} on 2 CTAs", slack)
+
+
+# Enough (token, 256-channel slice) items (T * slices >= 32768) for the single kernel's scatter
+# to stage eight quantised slices at a time in shared memory and send them to each dispatched
+# row with one bulk copy: the dispatched codes and scale bytes are the oracle's bit for bit, with
+# one group of 8 slices per token (H = 2048) and with a ragged second group ending in half a
+# slice (H = 2176)
+@pytest.mark.parametrize("H", [2048, 2176])
+def test_fused_bulk_scatter_matches_oracle(cuda_lib, H):
+    w = W(f"bulk_scatter_{H}", T=4096, H=H, I_=256, E=16, k=4, shared=1, router_std=0.05, bias="uniform")
+    case = make_case(w, seed=43)
+    d = to_device(case)
+    p = plan_for(w, fused=1)
+    out = p.forward(**d)
+    assert p.check_status()[0] == 0
+    ref, slack = oracle_forward_with_slack(case, w)
+    assert np.array_equal(p.region("topk_ids").cpu().numpy(), ref["ids"])
+    assert np.array_equal(p.region("offsets").cpu().numpy(), ref["offsets"])
+    assert np.array_equal(p.region("slot_pos").cpu().numpy(), ref["slot_pos"])
+    assert np.array_equal(p.region("perm").cpu().numpy()[:w.T * w.k], ref["perm"])
+    xq = p.region("xq").cpu().numpy()
+    xsf = untile_scales(p.region("xsf").cpu().numpy(), ref["counts"], ref["offsets"],
+                        p.get_option(binding.MOE_OPT_TILE_ROWS))
+    rows = ref["slot_pos"]
+    for j in range(w.k):
+        assert np.array_equal(xq[rows[:, j]], ref["xq"])
+        assert np.array_equal(xsf[rows[:, j]] - 127, ref["xexp"])
+    R = w.T * w.k
+    assert np.array_equal(xq[R:R + w.T], ref["xq"])
+    assert np.array_equal(xsf[R:R + w.T] - 127, ref["xexp"])
+    assert_output_close(bits(out), ref["y"], w.name, slack)
