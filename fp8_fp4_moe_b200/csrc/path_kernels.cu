@@ -344,7 +344,9 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, float* log
     router_logits_smem_kernel<<<grid, 256, (size_t)E * H * 4, s>>>(x, W_r, logits, T, H, E);
   } else if ((long)T * E <= 4096) {
     router_logits_split_kernel<<<dim3(E, T), 256, 0, s>>>(x, W_r, logits, T, H, E);
-  } else if (E <= 32 || (long)T * E <= 16384) {
+  } else if (E <= 32 || (long)T * E <= 16384 || (long)((T + 63) / 64) * ((E + 63) / 64) < 148) {
+    // (also whenever the tiled router would have fewer blocks than SMs: with 64 x 64 (token,
+    // expert) tiles over all of H, a handful of blocks takes milliseconds at H = 7168)
     // warp per (token, expert chunk)
     const int ec = (E <= 32) ? 8 : 2;
     const long items = (long)T * ((E + ec - 1) / ec);

@@ -72,7 +72,7 @@ enum moe_option {
                                   fills its first pipeline stage, so the MMA warp's
                                   bounded wait runs out and the call reports
                                   MOE_ERR_DEVICE_TIMEOUT                                  */
-  MOE_OPT_ROUTER_TC = 4,       /* 1 (default): router logits on tensor cores when T >= 256
+  MOE_OPT_ROUTER_TC = 4,       /* 1 (default): router logits on tensor cores when T >= 64
                                   and E % 16 == 0, as x (bf16) times W_router split into two
                                   bf16 parts (hi = bf16(W), lo = bf16(W - hi); |residual| <=
                                   2^-18 |W|) accumulated in fp32; 0: fp32 FMA on CUDA cores */

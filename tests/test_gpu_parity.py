@@ -32,9 +32,10 @@ SMALL = {
     "t16_shared": W("t16_shared", T=16, H=512, I_=384, E=4, k=2, shared=1, bias="uniform"),
     "k_eq_E": W("k_eq_E", T=50, H=256, I_=384, E=6, k=6, shared=1),
     "dsv3_like": W("dsv3_like", T=96, H=512, I_=256, E=64, k=8, shared=1, router_std=0.01, bias="uniform"),
-    # T >= 256 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
+    # T >= 64 and E % 16 == 0: tensor-core router; E = 48 leaves most of the 128-expert tile masked
     "tc_router": W("tc_router", T=300, H=1024, I_=256, E=48, k=4, shared=1, router_std=0.02, bias="uniform"),
-    # E > 32 with T * E > 16384 and E % 16 != 0: the tiled CUDA-core router
+    # E > 32 with T * E > 16384 and E % 16 != 0: a warp per (token, 2 experts) on CUDA cores (the
+    # tiled router would have fewer blocks than SMs)
     "wide_router": W("wide_router", T=500, H=512, I_=256, E=40, k=6, shared=1, router_std=0.02, bias="uniform"),
     # k > 8: the combine keeps up to 16 rows a lane in registers
     "k10": W("k10", T=40, H=256, I_=256, E=24, k=10, shared=1, router_std=0.05, bias="uniform"),
@@ -346,8 +347,9 @@ def test_forward_pair_tiles_match_oracle(cuda_lib, name):
 
 
 # every step in one persistent cooperative kernel: each router variant (tensor cores for
-# tc_router, block per expert and token for tiny / t1_k1 / k_eq_E, warp per token and expert
-# chunk for ragged_shared / dsv3_like), routing and dispatch bit-exact, outputs in tolerance
+# ragged_shared / dsv3_like / tc_router, a warp per (expert, K part) over all tokens for t1_k1 /
+# t16_shared / h1792_t8, block per expert and token for tiny / k_eq_E / k10 / h896, warp per
+# token and 2 experts for wide_router), routing and dispatch bit-exact, outputs in tolerance
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_fused_matches_oracle(cuda_lib, name):
     w = SMALL[name]

@@ -36,7 +36,8 @@ CASES = {
     "split_router": dict(T=4, H=512, E=16, k=4),       # T * E <= 4096: block per (expert, token)
     "warp8_router": dict(T=200, H=384, E=32, k=6),     # E <= 32: warp per (token, 8 experts)
     "warp2_router": dict(T=100, H=512, E=64, k=8),     # T * E <= 16384: warp per (token, 2 experts)
-    "tiled_router": dict(T=333, H=512, E=64, k=8),     # otherwise: the tiled router
+    "warp2_few_tiles": dict(T=333, H=512, E=64, k=8),  # T * E > 16384, but 6 router tiles: warp kernel
+    "tiled_router": dict(T=2400, H=256, E=256, k=8),   # >= 148 tiles of 64 x 64: the tiled router
 }
 
 
