@@ -1304,92 +1304,7 @@ __device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, lo
   }
 }
 
-// The single-kernel forward's scatter of many tokens, one item = 8 slices (2048 channels) of one
-// token's x row: the warp quantises them as scatter_items does, stages the E4M3 bytes in its 2 KB
-// of the epilogue staging area (idle before the first tile) and sends them to each of the token's
-// k (+ shared) dispatched rows with one bulk copy, in place of 8 x 32 eight-byte stores per row;
-// the scale bytes and positions are plain stores.  `pending`: this warp has bulk copies whose
-// staging bytes may still be read.
 constexpr int kScatterBulkSlices = 8;
-__device__ __forceinline__ void scatter_item_bulk(long item, const FusedArgs& f, uint8_t* stage, bool& pending) {
-  constexpr int SL = kScatterBulkSlices;
-  const int lane = threadIdx.x % 32;
-  const int n_slices = (f.H + 255) / 256;
-  const int n_grp = (n_slices + SL - 1) / SL;
-  const int t = (int)(item / n_grp);
-  const int grp = (int)(item % n_grp);
-  const int g = t / 32;
-  const long R = (long)f.T * f.k;
-  const int kw = f.H / 128;
-  // the token's 8 channels of this lane in each slice, loaded before the position lookups
-  uint4 raw[SL];
-#pragma unroll
-  for (int s = 0; s < SL; ++s) {
-    const int c0 = (grp * SL + s) * 256 + lane * 8;
-    raw[s] = c0 < f.H ? *reinterpret_cast<const uint4*>(f.x + (long)t * f.H + c0) : make_uint4(0, 0, 0, 0);
-  }
-  int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
-  int e = -1;
-  if (lane < f.k) {
-    e = f.topk_ids[(long)t * f.k + lane];
-    row = f.offsets[e] + f.group_base[(long)g * f.E + e] + f.local_rank[(long)t * f.k + lane];
-    if (grp == 0) {
-      f.slot_pos[(long)t * f.k + lane] = row;
-      f.perm[row] = t * f.k + lane;
-    }
-  } else if (lane == f.k && f.shared) {
-    e = f.E;
-    row = (int)(R + t);
-  }
-  long sf_off = 0;                       // this destination row's word inside its tile's scale atoms
-  if (e >= 0) {
-    const int rank = row - f.offsets[e];
-    const int r = rank % f.bm;
-    sf_off = ((long)(f.mtile_start[e] + rank / f.bm) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
-  }
-  const int ndst = f.k + f.shared;
-  // the previous item's copies must have read the staging bytes before they are overwritten
-  if (pending && lane < ndst) bulk_wait_read<0>();
-  __syncwarp();
-#pragma unroll
-  for (int s = 0; s < SL; ++s) {
-    if ((grp * SL + s) * 256 >= f.H) break;      // warp-uniform: the slice starts past H
-    const int c0 = (grp * SL + s) * 256 + lane * 8;
-    const bool active = c0 < f.H;                // H % 128 == 0: whole half-warps
-    const uint4 rw = raw[s];
-    float v[8];
-    v[0] = __uint_as_float(rw.x << 16); v[1] = __uint_as_float(rw.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(rw.y << 16); v[3] = __uint_as_float(rw.y & 0xFFFF0000u);
-    v[4] = __uint_as_float(rw.z << 16); v[5] = __uint_as_float(rw.z & 0xFFFF0000u);
-    v[6] = __uint_as_float(rw.w << 16); v[7] = __uint_as_float(rw.w & 0xFFFF0000u);
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const int p = pow2_exp_e4m3(amax);
-    const float sc = exp2_neg(p);
-    uint2 q;
-    q.x = pack_e4m3x4(v[0] * sc, v[1] * sc, v[2] * sc, v[3] * sc);
-    q.y = pack_e4m3x4(v[4] * sc, v[5] * sc, v[6] * sc, v[7] * sc);
-    if (active) *reinterpret_cast<uint2*>(stage + s * 256 + lane * 8) = q;
-    const uint32_t code = (uint32_t)(p + 127) * 0x01010101u;
-    const int blk = c0 / 128;
-    for (int d = 0; d < ndst; ++d) {
-      const long so = __shfl_sync(0xffffffffu, sf_off, d);
-      if (active && (lane & 15) == 0) *reinterpret_cast<uint32_t*>(f.xsf + so + (long)blk * 512) = code;
-    }
-  }
-  fence_proxy_async_smem();              // this lane's staging bytes, before the copies read them
-  __syncwarp();
-  if (lane < ndst) {
-    const int c_base = grp * SL * 256;
-    const uint32_t bytes = (uint32_t)min(SL * 256, f.H - c_base);   // E4M3: one byte a channel
-    bulk_store(f.xq + (long)row * f.H + c_base, stage, bytes);
-    bulk_commit();
-  }
-  pending = true;
-}
 
 // Before its first linear1 tile, each epilogue warp of the grid scatters (and quantises) its
 // share of the (token, channel group) items; once all eight of a CTA's have, one thread adds 1 to
@@ -1406,7 +1321,10 @@ struct ScatterWork {
       // many items: eight slices per item through the warp's 2 KB of staging memory
       uint8_t* stage = smem + L::stage_out + (epi_id % kEpiWarps) * 2048;
       const long items = (long)f.T * ((slices + kScatterBulkSlices - 1) / kScatterBulkSlices);
-      for (long it = epi_id; it < items; it += n_epi) scatter_item_bulk(it, f, stage, pending);
+      for (long it = epi_id; it < items; it += n_epi)
+        scatter_items_bulk<kScatterBulkSlices>(it, f.x, f.topk_ids, f.local_rank, f.group_base, f.offsets,
+                                               f.mtile_start, f.slot_pos, f.perm, f.xq, f.xsf, f.T, f.H, f.E, f.k,
+                                               f.shared, f.bm, stage, pending);
     } else {
       const long items = (long)f.T * slices;
       for (long it = epi_id; it < items; it += n_epi)
@@ -1415,7 +1333,7 @@ struct ScatterWork {
     }
     // bulk copies complete (their writes performed), generic stores -> other CTAs' TMA reads:
     // proxy fence, CTA barrier, gpu-scope release
-    if (pending && (threadIdx.x % 32) < f.k + f.shared) bulk_wait<0>();
+    scatter_bulk_drain(pending, f.k, f.shared);
     fence_proxy_async_global();
     epi_bar();
     if (threadIdx.x == 2 * 32) {

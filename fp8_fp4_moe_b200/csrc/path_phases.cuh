@@ -541,6 +541,103 @@ __device__ __forceinline__ void scatter_items(long item, const uint16_t* __restr
     }
   }
 }
+// Many items: the same as scatter_items for one item of SL slices (SL * 256 <= 2048 channels),
+// except that the E4M3 bytes are staged in the warp's 2 KB of shared memory `stage` and sent to
+// each destination row with one bulk copy, in place of SL x 32 eight-byte stores per row; the
+// scale bytes and positions are plain stores.  `pending` (carried from item to item): the warp has
+// bulk copies that may still read `stage`; scatter_bulk_drain waits for all of them to complete.
+template <int SL>
+__device__ __forceinline__ void scatter_items_bulk(long item, const uint16_t* __restrict__ x,
+                                                   const int32_t* __restrict__ topk_ids,
+                                                   const int32_t* __restrict__ local_rank,
+                                                   const int32_t* __restrict__ group_base,
+                                                   const int32_t* __restrict__ offsets,
+                                                   const int32_t* __restrict__ mtile_start, int32_t* slot_pos,
+                                                   int32_t* perm, uint8_t* xq, uint8_t* xsf, int T, int H, int E,
+                                                   int k, int shared, int bm, uint8_t* stage, bool& pending) {
+  static_assert(SL * 256 <= 2048, "one item's codes fit the warp's 2 KB of staging memory");
+  const int lane = threadIdx.x % 32;
+  const int n_slices = (H + 255) / 256;
+  const int n_grp = (n_slices + SL - 1) / SL;
+  const int t = (int)(item / n_grp);
+  const int grp = (int)(item % n_grp);
+  const int g = t / 32;
+  const long R = (long)T * k;
+  const int kw = H / 128;
+  // the token's 8 channels of this lane in each slice, loaded before the position lookups
+  uint4 raw[SL];
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    raw[s] = c0 < H ? *reinterpret_cast<const uint4*>(x + (long)t * H + c0) : make_uint4(0, 0, 0, 0);
+  }
+  int row = -1;                          // lane j < k holds the row of slot j; lane k the shared row
+  int e = -1;
+  if (lane < k) {
+    e = topk_ids[(long)t * k + lane];
+    row = offsets[e] + group_base[(long)g * E + e] + local_rank[(long)t * k + lane];
+    if (grp == 0) {
+      slot_pos[(long)t * k + lane] = row;
+      perm[row] = t * k + lane;
+    }
+  } else if (lane == k && shared) {
+    e = E;
+    row = (int)(R + t);
+  }
+  long sf_off = 0;                       // this destination row's word inside its tile's scale atoms
+  if (e >= 0) {
+    const int rank = row - offsets[e];
+    const int r = rank % bm;
+    sf_off = ((long)(mtile_start[e] + rank / bm) * kw) * 512 + (r % 32) * 16 + (r / 32) * 4;
+  }
+  const int ndst = k + shared;
+  // the previous item's copies must have read the staging bytes before they are overwritten
+  if (pending && lane < ndst) bulk_wait_read<0>();
+  __syncwarp();
+#pragma unroll
+  for (int s = 0; s < SL; ++s) {
+    if ((grp * SL + s) * 256 >= H) break;        // warp-uniform: the slice starts past H
+    const int c0 = (grp * SL + s) * 256 + lane * 8;
+    const bool active = c0 < H;                  // H % 128 == 0: whole half-warps
+    const uint4 rw = raw[s];
+    float v[8];
+    v[0] = __uint_as_float(rw.x << 16); v[1] = __uint_as_float(rw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(rw.y << 16); v[3] = __uint_as_float(rw.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(rw.z << 16); v[5] = __uint_as_float(rw.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(rw.w << 16); v[7] = __uint_as_float(rw.w & 0xFFFF0000u);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const int p = pow2_exp_e4m3(amax);
+    const float sc = exp2_neg(p);
+    uint2 q;
+    q.x = pack_e4m3x4(v[0] * sc, v[1] * sc, v[2] * sc, v[3] * sc);
+    q.y = pack_e4m3x4(v[4] * sc, v[5] * sc, v[6] * sc, v[7] * sc);
+    if (active) *reinterpret_cast<uint2*>(stage + s * 256 + lane * 8) = q;
+    const uint32_t code = (uint32_t)(p + 127) * 0x01010101u;
+    const int blk = c0 / 128;
+    for (int d = 0; d < ndst; ++d) {
+      const long so = __shfl_sync(0xffffffffu, sf_off, d);
+      if (active && (lane & 15) == 0) *reinterpret_cast<uint32_t*>(xsf + so + (long)blk * 512) = code;
+    }
+  }
+  fence_proxy_async_smem();              // this lane's staging bytes, before the copies read them
+  __syncwarp();
+  if (lane < ndst) {
+    const int c_base = grp * SL * 256;
+    const uint32_t bytes = (uint32_t)min(SL * 256, H - c_base);   // E4M3: one byte a channel
+    bulk_store(xq + (long)row * H + c_base, stage, bytes);
+    bulk_commit();
+  }
+  pending = true;
+}
+// Waits until the warp's scatter bulk copies are complete (their writes performed).
+__device__ __forceinline__ void scatter_bulk_drain(bool pending, int k, int shared) {
+  if (pending && (threadIdx.x % 32) < k + shared) bulk_wait<0>();
+  __syncwarp();
+}
 __device__ __forceinline__ void scatter_item(long item, const uint16_t* __restrict__ x,
                                              const int32_t* __restrict__ topk_ids,
                                              const int32_t* __restrict__ local_rank,

@@ -614,17 +614,18 @@ def test_few_ctas_match_the_full_grid(cuda_lib, name, fused, pair_tiles):
     assert_output_close(bits(outs[1]), ref["y"], f"{name} fused={fused} on 2 CTAs", slack)
 
 
-# Enough (token, 256-channel slice) items (T * slices >= 32768) for the single kernel's scatter
-# to stage eight quantised slices at a time in shared memory and send them to each dispatched
-# row with one bulk copy: the dispatched codes and scale bytes are the oracle's bit for bit, with
-# one group of 8 slices per token (H = 2048) and with a ragged second group ending in half a
-# slice (H = 2176)
+# Enough (token, 256-channel slice) items (T * slices >= 32768) for the many-token scatters: the
+# scatter kernel's four slices per warp, and the single kernel's eight quantised slices staged in
+# shared memory and sent to each dispatched row with one bulk copy.  The dispatched codes and
+# scale bytes are the oracle's bit for bit, with one group of slices per token (H = 2048) and with
+# a ragged last group ending in half a slice (H = 2176)
+@pytest.mark.parametrize("fused", [0, 1])
 @pytest.mark.parametrize("H", [2048, 2176])
-def test_fused_bulk_scatter_matches_oracle(cuda_lib, H):
+def test_bulk_scatter_matches_oracle(cuda_lib, H, fused):
     w = W(f"bulk_scatter_{H}", T=4096, H=H, I_=256, E=16, k=4, shared=1, router_std=0.05, bias="uniform")
     case = make_case(w, seed=43)
     d = to_device(case)
-    p = plan_for(w, fused=1)
+    p = plan_for(w, fused=fused)
     out = p.forward(**d)
     assert p.check_status()[0] == 0
     ref, slack = oracle_forward_with_slack(case, w)
