@@ -565,9 +565,9 @@ __device__ __forceinline__ void gemm_body(const AMaps& tmA, const CUtensorMap& t
       };
       auto load_b = [&](const TileCoord& c, int st, int kt) {
         if constexpr (MODE == 1) {
-          const int brow = c.e * p.rows_b + c.nt * 128;
-          tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);
-          tma_load_2d(b_s + st * kBTileBytes + kBTileBytes / 2, &tmB, kt * BK, brow + p.N, &full[st]);
+          // the tile's 128 gate rows and the matching 128 up rows (I rows further on) in one box
+          // of the 3-D map [experts x {gate, up}][I][H]: gate half first, up half behind it
+          tma_load_3d(b_s + st * kBTileBytes, &tmB, kt * BK, c.nt * 128, c.e * 2, &full[st]);
         } else {
           const int brow = c.e * p.rows_b + c.nt * NB;
           tma_load_2d(b_s + st * kBTileBytes, &tmB, kt * BK, brow, &full[st]);

@@ -32,6 +32,10 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 
 // 2-D tiled tensor map (cuTensorMapEncodeTiled through the runtime's driver entry point):
 // dims {inner, outer}, row pitch in bytes, box {box_inner, box_outer}.  MOE_OK or MOE_ERR_CUDA.
+// 3-D map over [outer2][outer][inner] with byte strides row_bytes (outer) and slab_bytes (outer2).
+int encode_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t outer2, uint64_t row_bytes, uint64_t slab_bytes, uint32_t box_inner, uint32_t box_outer,
+              uint32_t box_outer2);
 int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);

@@ -57,6 +57,7 @@ struct moe_plan_s {
   int num_sms = 0;
   alignas(64) AMaps amA1, amA2;
   alignas(64) CUtensorMap tmB1, tmB2, tmB2d, tmX, tmWhi, tmWlo;   // tmB2d: 224-row boxes
+  alignas(64) CUtensorMap tmB1g;    // W1 as [experts x {gate, up}][I][H]: a tile's two halves in one box
   alignas(64) CUtensorMap tmB2p, tmSfa1, tmSfa2, tmSfb1, tmSfb2;   // CTA-pair GEMM operands
   const void* x_cached = nullptr;        // tmX encodes this x pointer
   const void* wr_prepared = nullptr;     // W_router the hi/lo split was made from
@@ -107,6 +108,20 @@ int encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int encode_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t outer2, uint64_t row_bytes, uint64_t slab_bytes, uint32_t box_inner, uint32_t box_outer,
+              uint32_t box_outer2) {
+  if (get_encode() != MOE_OK) return MOE_ERR_CUDA;
+  cuuint64_t dims[3] = {inner, outer, outer2};
+  cuuint64_t strides[2] = {row_bytes, slab_bytes};
+  cuuint32_t box[3] = {box_inner, box_outer, box_outer2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -428,7 +443,7 @@ int launch_fused(moe_plan_t p, const uint16_t* x, const float* W_router, const f
   // a launch that ran out of time may have left arrivals behind
   if (cudaMemsetAsync(a.gridbar, 0, 8, s) != cudaSuccess) return MOE_ERR_CUDA;
   const CUtensorMap& b2 = a.g2.bn == kGemmBN2Double ? p->tmB2d : p->tmB2;
-  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1, b2, p->tmX, p->tmWhi, p->tmWlo, a, ctas,
+  if (launch_fused_forward(p->amA1, p->amA2, p->tmB1g, b2, p->tmX, p->tmWhi, p->tmWlo, a, ctas,
                            plan_bm(p) == kGemmBMSmall, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // one kernel: its whole time is reported under the first phase
@@ -474,12 +489,12 @@ int launch_forward(moe_plan_t p, const uint16_t* x, const float* W_router, const
       a1.dep_signal = dep;
       a2.dep_wait = dep;
       a2.dep_per_mtile = a1.n_tiles_n;
-      if (launch_gemm_chain(p->amA1, p->amA2, p->tmB1, b2, a1, a2, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess)
+      if (launch_gemm_chain(p->amA1, p->amA2, p->tmB1g, b2, a1, a2, gemm_grid(p, a1.n_tiles_n), s) != cudaSuccess)
         return MOE_ERR_CUDA;
       mark(p, 1 + MOE_PHASE_LINEAR1, s);
       mark(p, 1 + MOE_PHASE_LINEAR2, s);
     } else {
-      if (launch_gemm_linear1(p->amA1, p->tmB1, a1, gemm_grid(p, a1.n_tiles_n), s, small_tiles) != cudaSuccess)
+      if (launch_gemm_linear1(p->amA1, p->tmB1g, a1, gemm_grid(p, a1.n_tiles_n), s, small_tiles) != cudaSuccess)
         return MOE_ERR_CUDA;
       mark(p, 1 + MOE_PHASE_LINEAR1, s);
       if (launch_gemm_linear2(p->amA2, b2, a2, gemm_grid(p, a2.n_tiles_n), s, small_tiles) != cudaSuccess)
@@ -786,6 +801,9 @@ int moe_forward(moe_plan_t p, const void* x, const float* W_router, const float*
   if (W1 != p->w1_cached) {
     rc = encode_2d(&p->tmB1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W1, p->H, (uint64_t)p->n * 2 * p->I, p->H / 2,
                    128, 128);
+    if (rc == MOE_OK)
+      rc = encode_3d(&p->tmB1g, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, W1, p->H, p->I, (uint64_t)p->n * 2, p->H / 2,
+                     (uint64_t)p->I * (p->H / 2), 128, 128, 2);
     if (rc != MOE_OK) return rc;
     p->w1_cached = W1;
   }
