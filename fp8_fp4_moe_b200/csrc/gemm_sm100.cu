@@ -1294,16 +1294,6 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, uint32_t n_ctas, uint32
   return *ok_smem != 0;
 }
 
-template <int KMAX, int U>
-__device__ __forceinline__ void fused_combine(const FusedArgs& a, long items, long first, long stride) {
-  for (long it = first; it < items; it += U * stride) {
-    long its[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) its[u] = it + u * stride;
-    combine_items<KMAX, U>(its, a.y, a.slot_pos, a.gates, a.out, a.T, a.H, a.k, a.shared);
-  }
-}
-
 constexpr int kScatterBulkSlices = 8;
 
 // Before its first linear1 tile, each epilogue warp of the grid scatters (and quantises) its
