@@ -247,12 +247,29 @@ cudaError_t launch_topk_rank(int mode, const float* logits, int n_parts, const f
                              float* gates,
                              int32_t* local_rank, int32_t* group_counts, uint32_t* status, int T, int E, int k,
                              cudaStream_t s);
-// T <= 32: launch_topk_rank followed by launch_dispatch_scan, as one single-block kernel.
+// The scatter step folded into the one-group kernel below (x == nullptr: not folded): the
+// arguments launch_scatter_quant takes beyond the routing results.
+struct FoldedScatter {
+  const uint16_t* x;
+  int32_t* slot_pos;
+  int32_t* perm;
+  uint8_t* xq;
+  uint8_t* xsf;
+  int H;
+  uint32_t* zero;
+  int n_zero;
+};
+// At most this many (token, 256-channel slice) items for the fold: the block's 32 warps take
+// them one by one, which beats a separate launch only while they are few.
+constexpr int kFoldScatterMaxItems = 128;
+// T <= 32: launch_topk_rank followed by launch_dispatch_scan, as one single-block kernel; with
+// fs.x set (T * slices <= kFoldScatterMaxItems), also launch_scatter_quant's work.
 cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_parts, const float* bias,
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
                                       int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                      int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s);
+                                      int4* ptile_info, int T, int E, int k, int shared, int bm, FoldedScatter fs,
+                                      cudaStream_t s);
 // counts, offsets, mtile_start (bm-row tiles), ptile_start (pairs of 128-row tiles) (n + 1
 // entries), the row-tile tables (see GemmArgs) and group_base[g][e] = rows of expert e in token
 // groups < g (relative to offsets[e]).

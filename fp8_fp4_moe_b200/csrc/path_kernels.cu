@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
     int mode, const float* __restrict__ logits, int n_parts, const float* __restrict__ bias, int32_t* topk_ids,
     float* gates, int32_t* __restrict__ local_rank, int32_t* __restrict__ group_counts, uint32_t* status,
     int32_t* group_base, int32_t* counts, int32_t* offsets, int32_t* mtile_start, int32_t* ptile_start,
-    int4* tile_info, int4* ptile_info, int T, int E, int k, int shared, int bm) {
+    int4* tile_info, int4* ptile_info, int T, int E, int k, int shared, int bm, FoldedScatter fs) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ TopkSmem sm;
@@ -213,6 +213,17 @@ __global__ void __launch_bounds__(1024) topk_scan_one_group_kernel(
   __syncthreads();
   expert_scan_block<1024>(counts, offsets, mtile_start, ptile_start, tile_info, ptile_info, T, E, shared, bm, wsum,
                           cnt_s);
+  if (fs.x != nullptr) {
+    // the scatter of a few tokens, here instead of in a kernel of its own: the positions and the
+    // tile starts this block wrote are visible to all of its threads after the barrier
+    if (fs.zero != nullptr)
+      for (int i = threadIdx.x; i < fs.n_zero; i += blockDim.x) fs.zero[i] = 0u;
+    __syncthreads();
+    const long items = (long)T * ((fs.H + 255) / 256);
+    for (long it = threadIdx.x / 32; it < items; it += blockDim.x / 32)
+      scatter_item(it, fs.x, topk_ids, local_rank, group_base, offsets, mtile_start, fs.slot_pos, fs.perm, fs.xq,
+                   fs.xsf, T, fs.H, E, k, shared, bm);
+  }
 }
 
 // --------------------------------------------------------------------------- scan
@@ -375,11 +386,13 @@ cudaError_t launch_topk_scan_one_group(int mode, const float* logits, int n_part
                                       int32_t* topk_ids, float* gates, int32_t* local_rank, int32_t* group_counts,
                                       uint32_t* status, int32_t* group_base, int32_t* counts, int32_t* offsets,
                                       int32_t* mtile_start, int32_t* ptile_start, int4* tile_info,
-                                      int4* ptile_info, int T, int E, int k, int shared, int bm, cudaStream_t s) {
+                                      int4* ptile_info, int T, int E, int k, int shared, int bm, FoldedScatter fs,
+                                      cudaStream_t s) {
   if (T > 32 || n_parts < 1 || (n_parts > 1 && E > kTopkMaxSplitE)) return cudaErrorInvalidValue;
+  if (fs.x != nullptr && (long)T * ((fs.H + 255) / 256) > kFoldScatterMaxItems) return cudaErrorInvalidValue;
   return launch_kernel(topk_scan_one_group_kernel, 1, 1024, 0, s, mode, logits, n_parts, bias, topk_ids, gates,
                        local_rank, group_counts, status, group_base, counts, offsets, mtile_start, ptile_start,
-                       tile_info, ptile_info, T, E, k, shared, bm);
+                       tile_info, ptile_info, T, E, k, shared, bm, fs);
 }
 
 cudaError_t launch_dispatch_scan(const int32_t* group_counts, int32_t* counts, int32_t* offsets,
