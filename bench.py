@@ -49,8 +49,11 @@ REF_STEP_TOKENS = {"tiny": 64, "mixtral": 1, "dsv3_t1": 1, "dsv3_t512": 1, "dsv3
 
 def kernels_per_forward(w) -> int:
     """router, top-k, column scan, expert scan, scatter, linear1, linear2, combine; with at
-    most 32 tokens top-k and the two scans are one kernel (prepare is skipped: weights static)."""
-    return 6 if w.T <= 32 else 8
+    most 32 tokens top-k and the two scans are one kernel, and with at most 32 (token, 256-channel
+    slice) items the scatter runs in it too (prepare is skipped: weights static)."""
+    if w.T <= 32:
+        return 5 if w.T * ((w.H + 255) // 256) <= 32 else 6
+    return 8
 
 
 def parse():
